@@ -1,0 +1,335 @@
+"""Pins of the oracle's MoE-layer steps against closed forms, brute force,
+invariants and library routines (torch's float8 cast, torch's silu), so that
+a dropped term, a wrong sign or index, or a transposed operand in the oracle
+fails one of them.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import gen
+from oracle import e4m3, moe
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+# ---------------------------------------------------------------- helpers
+
+def torch_decode(codes) -> np.ndarray:
+    t = torch.from_numpy(np.ascontiguousarray(codes, dtype=np.uint8))
+    return t.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+
+
+def torch_encode(v32: np.ndarray) -> np.ndarray:
+    v = np.clip(np.asarray(v32, np.float32), -448, 448)
+    return torch.from_numpy(np.ascontiguousarray(v)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
+def textbook_quant_row(v):
+    """One row, groups of 128: fp32 amax/448, fp32 divide, torch's RNE cast."""
+    v = np.asarray(v, np.float32)
+    codes, scales = [], []
+    for g0 in range(0, len(v), 128):
+        blk = v[g0:g0 + 128]
+        amax = np.float32(max(abs(float(t)) for t in blk))
+        s = np.float32(amax / np.float32(448))
+        scales.append(s)
+        codes.extend([0] * len(blk) if amax == 0 else list(torch_encode(blk / s)))
+    return np.array(codes, np.uint8), np.array(scales, np.float32)
+
+
+def textbook_ffn(x_row_f64, wg, sg, wu, su, wd, sd, F, H):
+    """One token through one SwiGLU expert with explicit loops over every index."""
+    q, s = textbook_quant_row(x_row_f64.astype(np.float32))
+    xd = torch_decode(q)
+    a = [xd[k] * float(s[k // 128]) for k in range(H)]
+    dg, du, dd = torch_decode(wg), torch_decode(wu), torch_decode(wd)
+    h = np.zeros(F)
+    for n in range(F):
+        g = sum(a[k] * dg[n, k] * float(sg[n // 128, k // 128]) for k in range(H))
+        u = sum(a[k] * du[n, k] * float(su[n // 128, k // 128]) for k in range(H))
+        h[n] = g / (1.0 + math.exp(-g)) * u
+    hq, hs = textbook_quant_row(h.astype(np.float32))
+    hd = torch_decode(hq)
+    b = [hd[n] * float(hs[n // 128]) for n in range(F)]
+    y = np.zeros(H)
+    for m in range(H):
+        y[m] = sum(b[n] * dd[m, n] * float(sd[m // 128, n // 128]) for n in range(F))
+    return y
+
+
+def small_layer(H=256, E=6, K=2, F=130, ld_f=144, seed=5):
+    sh = gen.LayerShape(H=H, E=E, K=K, F=F, ld_f=ld_f)
+    return gen.make_layer(sh, seed), sh
+
+
+# ---------------------------------------------------------------- config
+
+def test_layer_shape_matches_pages():
+    cfg = json.load(open(os.path.join(GOLDEN, "dots3_text_config.json")))
+    s = gen.DOTS3
+    assert (s.H, s.E, s.K, s.F) == (cfg["hidden_size"], cfg["n_routed_experts"],
+                                    cfg["num_experts_per_tok"], cfg["moe_intermediate_size"])
+    assert cfg["shared_experts_intermediate_size"] == s.F and cfg["n_shared_experts"] == 1
+    assert cfg["weight_block_size"] == [moe.GROUP, moe.GROUP]
+    assert cfg["routed_scaling_factor"] == 1.0 and cfg["norm_topk_prob"] is True
+    assert cfg["hidden_act"] == "silu" and cfg["mlp_bias"] is False
+
+
+# ---------------------------------------------------------------- quantiser
+
+def test_quantize_matches_textbook_rows():
+    rng = np.random.default_rng(2)
+    v = (rng.standard_normal((5, 300)) * np.exp(rng.uniform(-3, 3, (5, 1)))).astype(np.float32)
+    v[1, 128:256] = 0.0                       # an all-zero group
+    v[2, 256:] = 0.0; v[2, 299] = -7.5        # partial last group (44 channels)
+    q, s = moe.quantize_rows(v)
+    for r in range(5):
+        tq, ts = textbook_quant_row(v[r])
+        assert np.array_equal(q[r], tq) and np.array_equal(s[r], ts)
+    assert s[1, 1] == 0 and not q[1, 128:256].any()
+    assert s[2, 2] == np.float32(np.float32(7.5) / np.float32(448))
+
+
+def test_quantize_error_bound_and_amax_code():
+    rng = np.random.default_rng(3)
+    v = (rng.standard_normal((64, 512)) * 3).astype(np.float32)
+    q, s = moe.quantize_rows(v)
+    d = moe.dequant_rows(q, s)
+    # RNE to 3 mantissa bits: |error| <= 2^-4 |value| + half the subnormal step
+    bound = np.abs(v) * 2.0 ** -4 + np.repeat(s, 128, axis=1) * 2.0 ** -10 * 1.0001
+    assert np.all(np.abs(d - v) <= bound)
+    # the amax element of every group lands on +-448
+    for g in range(4):
+        j = np.argmax(np.abs(v[:, g * 128:(g + 1) * 128]), axis=1) + g * 128
+        assert np.all(np.abs(e4m3.DECODE[q[np.arange(64), j]]) == 448.0)
+
+
+def test_quantize_power_of_two_invariance():
+    rng = np.random.default_rng(4)
+    v = rng.standard_normal((8, 256)).astype(np.float32)
+    q0, s0 = moe.quantize_rows(v)
+    for k in (-20, -3, 5, 30):
+        q1, s1 = moe.quantize_rows(v * np.float32(2.0 ** k))
+        assert np.array_equal(q0, q1)
+        assert np.array_equal(s1, s0 * np.float32(2.0 ** k))
+
+
+# ---------------------------------------------------------------- routing
+
+def test_topk_vs_full_sort_with_ties():
+    rng = np.random.default_rng(5)
+    E, K = 24, 5
+    logits = rng.standard_normal((200, E)).round(1)       # many exact ties
+    probs = moe.softmax(logits)
+    idx, w, gap = moe.select_topk(probs, K)
+    for t in range(200):
+        ref = sorted(range(E), key=lambda e: (-probs[t, e], e))
+        assert list(idx[t]) == sorted(ref[:K])
+        assert gap[t] == probs[t, ref[K - 1]] - probs[t, ref[K]]
+
+
+def test_route_weights_closed_form():
+    rng = np.random.default_rng(6)
+    logits = rng.standard_normal((50, 32)) * 2
+    probs = moe.softmax(logits)
+    idx, w, _ = moe.select_topk(probs, 8)
+    assert np.allclose(w.sum(1), 1.0, atol=1e-15)
+    sel = np.take_along_axis(logits, idx.astype(np.int64), 1)
+    closed = np.exp(sel - sel.max(1, keepdims=True))
+    closed /= closed.sum(1, keepdims=True)
+    assert np.allclose(w, closed, rtol=1e-13, atol=0)
+    assert np.allclose(moe.softmax(logits), torch.softmax(torch.from_numpy(logits), 1).numpy(), rtol=1e-14)
+
+
+def test_route_zero_input():
+    sh = gen.TOY
+    x = np.zeros((4, sh.H), np.uint16)
+    r = moe.route(x, gen.make_router(sh, 0), sh.K)
+    assert np.array_equal(r.idx, np.tile(np.arange(sh.K), (4, 1)))
+    assert np.all(r.w == 1.0 / sh.K)
+
+
+def test_near_tie_flag():
+    sh = gen.TOY
+    router = np.zeros((sh.E, sh.H), np.float32)
+    router[:, 0] = np.linspace(1.0, -1.0, sh.E).astype(np.float32)
+    router[sh.K, 0] = router[sh.K - 1, 0]                # 4th and 5th exactly tied
+    x = np.zeros((2, sh.H), np.uint16)
+    x[:, 0] = gen.f32_to_bf16_bits(np.float32([1.0]))[0]
+    r = moe.route(x, router, sh.K)
+    assert r.near_tie.all() and np.all(r.gap == 0)
+    assert list(r.idx[0]) == list(range(sh.K))          # tie -> lower id
+    router[sh.K, 0] = -1.0
+    assert not moe.route(x, router, sh.K).near_tie.any()
+
+
+# ---------------------------------------------------------------- permutation
+
+def brute_permute(idx, E):
+    T, K = idx.shape
+    counts = [0] * E
+    for t in range(T):
+        for k in range(K):
+            counts[idx[t, k]] += 1
+    offsets = [0]
+    for e in range(E):
+        offsets.append(offsets[-1] + counts[e])
+    offsets.append(offsets[-1] + T)
+    cursor = offsets[:E]
+    perm = [None] * (T * K + T)
+    inv = np.zeros((T, K), np.int64)
+    for t in range(T):
+        for k in range(K):
+            e = idx[t, k]
+            perm[cursor[e]] = t
+            inv[t, k] = cursor[e]
+            cursor[e] += 1
+    for t in range(T):
+        perm[T * K + t] = t
+    return np.array(offsets), np.array(perm), inv
+
+
+def test_permute_vs_brute_and_invariants():
+    rng = np.random.default_rng(7)
+    T, K, E = 123, 4, 16
+    idx = np.sort(np.array([rng.choice(E, K, replace=False) for _ in range(T)]), axis=1)
+    p = moe.permute(idx, E)
+    o, pr, iv = brute_permute(idx, E)
+    assert np.array_equal(p.offsets, o) and np.array_equal(p.perm, pr) and np.array_equal(p.inv, iv)
+    R = T * K
+    assert sorted(p.inv.ravel().tolist()) == list(range(R))                 # bijection onto [0, R)
+    assert np.all(p.perm[p.inv] == np.arange(T)[:, None])                   # perm o inv = token
+    grp = np.searchsorted(p.offsets, p.inv, side="right") - 1
+    assert np.array_equal(grp, idx)                                         # row lies in its expert's group
+    for e in range(E):
+        seg = p.perm[p.offsets[e]:p.offsets[e + 1]]
+        assert np.all(np.diff(seg) > 0)                                     # token order inside a group
+    assert p.offsets[E] == R and p.offsets[E + 1] == R + T
+    assert np.array_equal(p.perm[R:], np.arange(T))
+
+
+def test_permute_empty_and_all_to_one():
+    p = moe.permute(np.zeros((0, 4), np.int32), 8)
+    assert p.offsets.tolist() == [0] * 10 and len(p.perm) == 0
+    idx = np.tile(np.array([[3, 5]]), (6, 1))
+    p = moe.permute(idx, 8)
+    assert p.offsets.tolist() == [0, 0, 0, 0, 6, 6, 12, 12, 12, 18]
+
+
+# ---------------------------------------------------------------- expert FFN
+
+def test_silu_matches_torch():
+    g = np.linspace(-80, 80, 1001)
+    assert np.allclose(moe.silu(g), torch.nn.functional.silu(torch.from_numpy(g)).numpy(), rtol=1e-15, atol=1e-300)
+
+
+def test_expert_ffn_vs_textbook_loops():
+    layer, sh = small_layer()
+    rng = np.random.default_rng(8)
+    # scales vary block to block so a transposed scale index shows up
+    for name in ("s_gate", "s_up", "s_down"):
+        arr = getattr(layer, name)
+        arr *= rng.uniform(0.5, 2.0, arr.shape).astype(np.float32)
+    x = gen.f32_to_bf16_bits(rng.standard_normal((3, sh.H)).astype(np.float32) * 2)
+    xf = moe.bf16_to_f64(x)
+    e = 4
+    tq, ts = moe.quantize_tokens(x)
+    f = moe.expert_ffn_rows(tq, ts, np.array([0] * (e + 1) + [3] * (sh.E + 1 - e)), layer, groups=[e])
+    for r in range(3):
+        ref = textbook_ffn(xf[r], layer.w_gate[e], layer.s_gate[e], layer.w_up[e], layer.s_up[e],
+                           layer.w_down[e], layer.s_down[e], sh.F, sh.H)
+        assert np.allclose(f["y"][r], ref, rtol=1e-12, atol=1e-12 * np.abs(ref).max())
+
+
+def test_gemm_exact_integers():
+    """Scales 1 and codes with values in {-4..4}: every dot product is an exact integer."""
+    rng = np.random.default_rng(9)
+    vals = np.array([0x00, 0x38, 0x40, 0x44, 0x48, 0xB8, 0xC0, 0xC4, 0xC8], np.uint8)  # 0,1,2,3,4,-1,-2,-3,-4
+    ints = np.array([0, 1, 2, 3, 4, -1, -2, -3, -4])
+    ia, ib = rng.integers(0, 9, (7, 384)), rng.integers(0, 9, (200, 384))
+    a = moe.dequant_rows(vals[ia], np.ones((7, 3), np.float32))
+    w = moe.dequant_block(vals[ib], np.ones((2, 3), np.float32), 200, 384)
+    assert np.array_equal(a @ w.T, (ints[ia] @ ints[ib].T).astype(np.float64))
+
+
+def test_dequant_block_index_order():
+    codes = np.full((256, 384), 0x38, np.uint8)           # all 1.0
+    s = np.arange(6, dtype=np.float32).reshape(2, 3) + 1  # s[n_blk, k_blk]
+    w = moe.dequant_block(codes, s, 200, 300)
+    assert w[0, 0] == 1 and w[0, 299] == 3 and w[199, 0] == 4 and w[130, 260] == 6
+
+
+def test_combine_closed_form():
+    T, K, H = 3, 2, 4
+    y = np.arange((T * K + T) * H, dtype=np.float64).reshape(T * K + T, H)
+    inv = np.array([[4, 0], [1, 5], [2, 3]])
+    w = np.array([[0.25, 0.75], [0.5, 0.5], [1.0, 0.0]])
+    out = moe.combine(y, inv, w)
+    for t in range(T):
+        ref = sum(w[t, k] * y[inv[t, k]] for k in range(K)) + y[T * K + t]
+        assert np.array_equal(out[t], ref)
+
+
+# ---------------------------------------------------------------- whole layer
+
+def test_zero_input_gives_zero_output(toy):
+    _, layer, _ = toy
+    x = np.zeros((5, layer.shape.H), np.uint16)
+    r = moe.layer_forward(x, layer)
+    assert np.all(r["out"] == 0.0) and np.all(r["xs"] == 0) and not r["xq"].any()
+
+
+def test_one_hot_router_selects_one_expert(toy):
+    _, layer0, x = toy
+    sh = layer0.shape
+    estar, c0 = 11, 0
+    router = np.zeros((sh.E, sh.H), np.float32)
+    router[estar, c0] = 200.0
+    layer = gen.Layer(sh, router, layer0.w_gate, layer0.s_gate, layer0.w_up, layer0.s_up,
+                      layer0.w_down, layer0.s_down)
+    xs = x[:3].copy()
+    xs[:, c0] = gen.f32_to_bf16_bits(np.float32([1.0]))[0]
+    r = moe.layer_forward(xs, layer)
+    assert np.array_equal(r["route"].idx, np.tile([0, 1, 2, estar], (3, 1)))
+    assert np.all(r["route"].w[:, 3] == 1.0) and np.all(r["route"].w[:, :3] < 1e-80)
+    xf = moe.bf16_to_f64(xs)
+    for t in range(3):
+        ref = sum(textbook_ffn(xf[t], layer.w_gate[g], layer.s_gate[g], layer.w_up[g], layer.s_up[g],
+                               layer.w_down[g], layer.s_down[g], sh.F, sh.H) for g in (estar, sh.E))
+        assert np.allclose(r["out"][t], ref, rtol=1e-11, atol=1e-11 * np.abs(ref).max())
+
+
+def test_permuted_path_equals_direct_per_token(toy):
+    _, layer, x = toy
+    r = moe.layer_forward(x, layer)
+    d = moe.token_outputs(x, layer, np.arange(x.shape[0]))
+    assert np.max(np.abs(d - r["out"])) <= 1e-12 * np.max(np.abs(r["out"]))
+
+
+def test_partial_blocks_equal_zero_padded_layer():
+    """F=250 (not a multiple of 128) equals the same layer zero-padded to F=256."""
+    layer, sh = small_layer(H=256, E=4, K=2, F=250, ld_f=256, seed=11)
+    sp = gen.LayerShape(H=256, E=4, K=2, F=256, ld_f=256)
+    pad = lambda a, axis: np.concatenate([a, np.zeros(a.shape[:axis] + (256 - a.shape[axis],) + a.shape[axis + 1:], a.dtype)], axis)
+    lp = gen.Layer(sp, layer.router_w, pad(layer.w_gate, 1), layer.s_gate, pad(layer.w_up, 1), layer.s_up,
+                   layer.w_down.copy(), layer.s_down)
+    lp.w_down[:, :, 250:] = 0
+    x = gen.make_x(9, 256, 3)
+    a, b = moe.layer_forward(x, layer)["out"], moe.layer_forward(x, lp)["out"]
+    assert np.max(np.abs(a - b)) <= 1e-13 * np.max(np.abs(a))
+    # the tail scale block was taken over the real rows only
+    w = gen.normal_f32(11, gen.STREAM_GATE, 5 * 250 * 256, 1 / 16).reshape(5, 250, 256)
+    assert layer.s_gate[2, 1, 0] == np.float32(np.abs(w[2, 128:250, :128]).max() / np.float32(448))
+
+
+def test_bf16_checkpoint_cross_check(toy):
+    _, layer, x = toy
+    a = moe.layer_forward(x, layer)["out"]
+    b = moe.layer_forward_bf16(x, layer)
+    rel = np.linalg.norm(a - b) / np.linalg.norm(b)
+    assert 1e-4 < rel < 8e-2
