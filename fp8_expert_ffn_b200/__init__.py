@@ -1,0 +1,195 @@
+"""Python binding of libfp8moe.so: argument marshalling only.
+
+Every step of the layer runs in the library's CUDA kernels; this module only
+turns tensors into device pointers and calls the C entry points of
+include/moe.h by the same names. There is no CPU path: if the shared library
+cannot be loaded, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libfp8moe.so")
+
+MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_MISALIGNED, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, \
+    MOE_ERR_DEVICE = range(7)
+
+ENTRY_POINTS = ("moe_status_string", "moe_layer_create", "moe_layer_destroy", "moe_workspace_size", "moe_route",
+                "moe_permute", "moe_expert_ffn", "moe_combine", "moe_layer_forward", "moe_get_device_status",
+                "moe_test_grouped_gemm_f32", "moe_test_workspace_h")
+
+
+class MoeError(RuntimeError):
+    def __init__(self, fn: str, code: int, text: str):
+        super().__init__(f"{fn}: {text} (status {code})")
+        self.code = code
+
+
+class moe_layer_desc(ctypes.Structure):
+    _fields_ = [("hidden", ctypes.c_int), ("n_routed", ctypes.c_int), ("n_shared", ctypes.c_int),
+                ("top_k", ctypes.c_int), ("ffn", ctypes.c_int), ("shared_ffn", ctypes.c_int),
+                ("block", ctypes.c_int), ("routed_scaling", ctypes.c_float), ("norm_topk", ctypes.c_int)]
+
+
+class moe_weights(ctypes.Structure):
+    _fields_ = [("w_gate", ctypes.c_void_p), ("w_up", ctypes.c_void_p), ("w_down", ctypes.c_void_p),
+                ("s_gate", ctypes.c_void_p), ("s_up", ctypes.c_void_p), ("s_down", ctypes.c_void_p),
+                ("router_w", ctypes.c_void_p), ("ld_h", ctypes.c_int), ("ld_f", ctypes.c_int)]
+
+
+_lib = None
+
+
+def lib(build_if_missing: bool = True):
+    """Load libfp8moe.so (building it in-tree first if it is missing or stale)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if build_if_missing:
+        from . import build as _build
+        if _build.stale():
+            _build.build()
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"fp8_expert_ffn_b200: CUDA library not built ({LIB_PATH})")
+    L = ctypes.CDLL(LIB_PATH)
+    P, I, S, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_float
+    L.moe_status_string.argtypes = [I]
+    L.moe_status_string.restype = ctypes.c_char_p
+    L.moe_layer_create.argtypes = [ctypes.POINTER(moe_layer_desc), ctypes.POINTER(moe_weights), ctypes.POINTER(P)]
+    L.moe_layer_destroy.argtypes = [P]
+    L.moe_workspace_size.argtypes = [P, I]
+    L.moe_workspace_size.restype = S
+    L.moe_route.argtypes = [P, P, I, I, P, P, P, P, S, P]
+    L.moe_permute.argtypes = [P, P, I, I, P, P, P, P, P, P, P, S, P]
+    L.moe_expert_ffn.argtypes = [P, P, P, P, I, P, P, S, P]
+    L.moe_combine.argtypes = [P, P, P, P, I, P, I, P]
+    L.moe_layer_forward.argtypes = [P, P, I, I, P, I, P, S, P]
+    L.moe_get_device_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_uint32)]
+    L.moe_test_grouped_gemm_f32.argtypes = [P, I, P, P, P, I, P, P, S, P]
+    L.moe_test_workspace_h.argtypes = [P, I, ctypes.POINTER(S), ctypes.POINTER(S)]
+    for name in ENTRY_POINTS:
+        if name not in ("moe_status_string", "moe_workspace_size"):
+            getattr(L, name).restype = I
+    _lib = L
+    return L
+
+
+def status_string(code: int) -> str:
+    return lib().moe_status_string(code).decode()
+
+
+def _check(fn: str, code: int):
+    if code != MOE_OK:
+        raise MoeError(fn, code, status_string(code))
+
+
+def _ptr(t) -> int:
+    if t is None:
+        return 0
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+@dataclass
+class LayerWeights:
+    """Device tensors of one layer (uint8 codes, float32 scales/router)."""
+    w_gate: object
+    w_up: object
+    w_down: object
+    s_gate: object
+    s_up: object
+    s_down: object
+    router_w: object
+
+
+class MoeLayer:
+    """Owns a moe_layer_t; keeps the weight tensors alive while it exists."""
+
+    def __init__(self, hidden, n_routed, top_k, ffn, weights: LayerWeights, ld_h=None, ld_f=None,
+                 routed_scaling=1.0):
+        self.H, self.E, self.K, self.F = hidden, n_routed, top_k, ffn
+        self.weights = weights
+        d = moe_layer_desc(hidden, n_routed, 1, top_k, ffn, ffn, 128, routed_scaling, 1)
+        w = moe_weights(_ptr(weights.w_gate), _ptr(weights.w_up), _ptr(weights.w_down), _ptr(weights.s_gate),
+                        _ptr(weights.s_up), _ptr(weights.s_down), _ptr(weights.router_w),
+                        hidden if ld_h is None else ld_h, ffn if ld_f is None else ld_f)
+        h = ctypes.c_void_p()
+        _check("moe_layer_create", lib().moe_layer_create(ctypes.byref(d), ctypes.byref(w), ctypes.byref(h)))
+        self.handle = h.value
+
+    def close(self):
+        if getattr(self, "handle", None):
+            lib().moe_layer_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def rows(self, T: int) -> int:
+        return T * (self.K + 1)
+
+
+def moe_workspace_size(layer: MoeLayer, T: int) -> int:
+    return int(lib().moe_workspace_size(layer.handle, T))
+
+
+def moe_route(layer, x, T, ldx, topk_idx, topk_w, router_logits, ws, ws_bytes, stream=None):
+    _check("moe_route", lib().moe_route(layer.handle, _ptr(x), T, ldx, _ptr(topk_idx), _ptr(topk_w),
+                                        _ptr(router_logits), _ptr(ws), ws_bytes, _stream(stream)))
+
+
+def moe_permute(layer, x, T, ldx, topk_idx, offsets, perm, inv, xq, xs, ws, ws_bytes, stream=None):
+    _check("moe_permute", lib().moe_permute(layer.handle, _ptr(x), T, ldx, _ptr(topk_idx), _ptr(offsets),
+                                            _ptr(perm), _ptr(inv), _ptr(xq), _ptr(xs), _ptr(ws), ws_bytes,
+                                            _stream(stream)))
+
+
+def moe_expert_ffn(layer, xq, xs, offsets, T, y, ws, ws_bytes, stream=None):
+    _check("moe_expert_ffn", lib().moe_expert_ffn(layer.handle, _ptr(xq), _ptr(xs), _ptr(offsets), T, _ptr(y),
+                                                  _ptr(ws), ws_bytes, _stream(stream)))
+
+
+def moe_combine(layer, y, inv, topk_w, T, out, ldo, stream=None):
+    _check("moe_combine", lib().moe_combine(layer.handle, _ptr(y), _ptr(inv), _ptr(topk_w), T, _ptr(out), ldo,
+                                            _stream(stream)))
+
+
+def moe_layer_forward(layer, x, T, ldx, out, ldo, ws, ws_bytes, stream=None):
+    _check("moe_layer_forward", lib().moe_layer_forward(layer.handle, _ptr(x), T, ldx, _ptr(out), ldo, _ptr(ws),
+                                                        ws_bytes, _stream(stream)))
+
+
+def moe_get_device_status(layer, stream=None):
+    """(status code, raw bits); synchronises the stream."""
+    bits = ctypes.c_uint32(0)
+    code = lib().moe_get_device_status(layer.handle, _stream(stream), ctypes.byref(bits))
+    return code, bits.value
+
+
+def moe_test_grouped_gemm_f32(layer, which, a, a_scales, offsets, T, out, ws, ws_bytes, stream=None):
+    _check("moe_test_grouped_gemm_f32",
+           lib().moe_test_grouped_gemm_f32(layer.handle, which, _ptr(a), _ptr(a_scales), _ptr(offsets), T,
+                                           _ptr(out), _ptr(ws), ws_bytes, _stream(stream)))
+
+
+def moe_test_workspace_h(layer, T):
+    """(h byte offset, hs byte offset) inside a workspace for T tokens."""
+    h, hs = ctypes.c_size_t(0), ctypes.c_size_t(0)
+    _check("moe_test_workspace_h", lib().moe_test_workspace_h(layer.handle, T, ctypes.byref(h), ctypes.byref(hs)))
+    return h.value, hs.value

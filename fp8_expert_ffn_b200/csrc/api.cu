@@ -1,0 +1,294 @@
+// C ABI of the FP8 MoE-layer library: argument validation, the layer handle,
+// workspace carving and the composition of the stages. No entry point
+// allocates device memory except moe_layer_create (one 4-byte status word).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdlib>
+#include <cstring>
+#include <new>
+
+#include "internal.h"
+
+namespace moe {
+
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+}  // namespace
+
+bool encode_tmap_u8(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t rows, uint64_t depth, uint64_t ld,
+                    uint64_t depth_stride) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {inner, rows, depth};
+  cuuint64_t strides[2] = {ld, depth_stride};
+  cuuint32_t box[3] = {128, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  const cuuint32_t rank = depth > 1 ? 3 : 2;
+  CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, rank, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+Scratch carve(const moe_layer_s* L, int T, void* base) {
+  Scratch s = {};
+  const int K = L->K, E = L->E;
+  const size_t rows = size_t(T) * (K + 1);
+  const size_t W = (size_t(T) + 31) / 32;
+  char* b = static_cast<char*>(base);
+  size_t off = 0;
+  auto take = [&](size_t bytes) -> void* {
+    off = align_up(off, 256);
+    void* p = b ? b + off : nullptr;
+    off += bytes;
+    return p;
+  };
+  s.route_partial = static_cast<float*>(take(sizeof(float) * size_t(route_splits(L, T)) * T * E));
+  s.bitmap = static_cast<uint32_t*>(take(sizeof(uint32_t) * E * W));
+  s.wprefix = static_cast<uint32_t*>(take(sizeof(uint32_t) * E * W));
+  s.counts = static_cast<int32_t*>(take(sizeof(int32_t) * E));
+  s.plan = static_cast<int32_t*>(take(sizeof(int32_t) * kPlanInts(E)));
+  s.h = static_cast<uint8_t*>(take(rows * L->ld_hh));
+  s.hs = static_cast<float*>(take(sizeof(float) * L->FB * rows));
+  s.idx = static_cast<int32_t*>(take(sizeof(int32_t) * size_t(T) * K));
+  s.topw = static_cast<float*>(take(sizeof(float) * size_t(T) * K));
+  s.offsets = static_cast<int32_t*>(take(sizeof(int32_t) * (E + 2)));
+  s.perm = static_cast<int32_t*>(take(sizeof(int32_t) * rows));
+  s.inv = static_cast<int32_t*>(take(sizeof(int32_t) * size_t(T) * K));
+  s.xq = static_cast<uint8_t*>(take(rows * L->H));
+  s.xs = static_cast<float*>(take(sizeof(float) * L->HB * rows));
+  s.y = static_cast<uint16_t*>(take(sizeof(uint16_t) * rows * L->H));
+  s.total = align_up(off, 256);
+  return s;
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+namespace {
+
+moe_status from_cuda(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+moe_status check_x(const moe_layer_s* L, const uint16_t* x, int ldx) {
+  if (!x) return MOE_ERR_INVALID_ARG;
+  if (ldx < L->H) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || (size_t(ldx) * 2) % 16 != 0) return MOE_ERR_MISALIGNED;
+  return MOE_OK;
+}
+
+moe_status check_ws(const moe_layer_s* L, int T, void* ws, size_t ws_bytes) {
+  if (!ws) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(ws)) return MOE_ERR_MISALIGNED;
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return MOE_ERR_MISALIGNED;
+  if (ws_bytes < carve(L, T, nullptr).total) return MOE_ERR_WORKSPACE;
+  return MOE_OK;
+}
+
+constexpr int kMaxT = 1 << 20;
+
+}  // namespace
+
+extern "C" {
+
+const char* moe_status_string(moe_status s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_MISALIGNED: return "pointer or stride not 16-byte aligned";
+    case MOE_ERR_UNSUPPORTED: return "unsupported layer shape";
+    case MOE_ERR_WORKSPACE: return "workspace too small";
+    case MOE_ERR_CUDA: return "CUDA call failed";
+    case MOE_ERR_DEVICE: return "a kernel reported bad data or a timed-out wait";
+  }
+  return "unknown status";
+}
+
+moe_status moe_layer_create(const moe_layer_desc* d, const moe_weights* w, moe_layer_t* out) {
+  if (!out) return MOE_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (!d || !w) return MOE_ERR_INVALID_ARG;
+  if (d->hidden <= 0 || d->n_routed <= 0 || d->top_k <= 0 || d->ffn <= 0) return MOE_ERR_INVALID_ARG;
+  if (d->hidden % 128 != 0 || d->hidden > 16384 || d->n_routed > 256 || d->n_shared != 1 || d->top_k > 8 ||
+      d->top_k > d->n_routed || d->ffn > 4096 || d->shared_ffn != d->ffn || d->block != 128 || d->norm_topk != 1)
+    return MOE_ERR_UNSUPPORTED;
+  if (!(d->routed_scaling == d->routed_scaling)) return MOE_ERR_INVALID_ARG;
+  if (!w->w_gate || !w->w_up || !w->w_down || !w->s_gate || !w->s_up || !w->s_down || !w->router_w)
+    return MOE_ERR_INVALID_ARG;
+  if (w->ld_h < d->hidden || w->ld_f < d->ffn) return MOE_ERR_INVALID_ARG;
+  if (w->ld_h % 16 != 0 || w->ld_f % 16 != 0) return MOE_ERR_MISALIGNED;
+  const void* ptrs[] = {w->w_gate, w->w_up, w->w_down, w->s_gate, w->s_up, w->s_down, w->router_w};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return MOE_ERR_MISALIGNED;
+
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+  cudaDeviceProp prop;
+  if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return MOE_ERR_CUDA;
+  if (prop.major != 10) return MOE_ERR_UNSUPPORTED;
+
+  moe_layer_s* L = new (std::nothrow) moe_layer_s();
+  if (!L) return MOE_ERR_CUDA;
+  L->d = *d;
+  L->w = *w;
+  L->H = d->hidden;
+  L->E = d->n_routed;
+  L->K = d->top_k;
+  L->F = d->ffn;
+  L->HB = d->hidden / 128;
+  L->FB = (d->ffn + 127) / 128;
+  L->ld_hh = L->FB * 128;
+  L->device = dev;
+  L->num_sms = prop.multiProcessorCount;
+  const uint64_t E1 = uint64_t(L->E) + 1;
+  if (!encode_tmap_u8(&L->tm_gate, w->w_gate, L->H, L->F, E1, w->ld_h, uint64_t(L->F) * w->ld_h) ||
+      !encode_tmap_u8(&L->tm_up, w->w_up, L->H, L->F, E1, w->ld_h, uint64_t(L->F) * w->ld_h) ||
+      !encode_tmap_u8(&L->tm_down, w->w_down, L->F, L->H, E1, w->ld_f, uint64_t(L->H) * w->ld_f)) {
+    delete L;
+    return MOE_ERR_CUDA;
+  }
+  if (cudaMalloc(&L->status, sizeof(uint32_t)) != cudaSuccess) {
+    delete L;
+    return MOE_ERR_CUDA;
+  }
+  if (cudaMemset(L->status, 0, sizeof(uint32_t)) != cudaSuccess) {
+    cudaFree(L->status);
+    delete L;
+    return MOE_ERR_CUDA;
+  }
+  *out = L;
+  return MOE_OK;
+}
+
+moe_status moe_layer_destroy(moe_layer_t L) {
+  if (!L) return MOE_OK;
+  cudaError_t e = cudaFree(L->status);
+  delete L;
+  return from_cuda(e);
+}
+
+size_t moe_workspace_size(moe_layer_t L, int T) {
+  if (!L || T < 0 || T > kMaxT) return 0;
+  return carve(L, T, nullptr).total;
+}
+
+moe_status moe_route(moe_layer_t L, const uint16_t* x, int T, int ldx, int32_t* idx, float* w, float* logits,
+                     void* ws, size_t ws_bytes, void* stream) {
+  if (!L || T < 0 || T > kMaxT) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  moe_status s;
+  if ((s = check_x(L, x, ldx)) != MOE_OK) return s;
+  if (!idx || !w) return MOE_ERR_INVALID_ARG;
+  if ((s = check_ws(L, T, ws, ws_bytes)) != MOE_OK) return s;
+  Scratch sc = carve(L, T, ws);
+  return from_cuda(launch_route(L, x, T, ldx, idx, w, logits, sc.route_partial, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_permute(moe_layer_t L, const uint16_t* x, int T, int ldx, const int32_t* idx, int32_t* offsets,
+                       int32_t* perm, int32_t* inv, uint8_t* xq, float* xs, void* ws, size_t ws_bytes,
+                       void* stream) {
+  if (!L || T < 0 || T > kMaxT) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  moe_status s;
+  if ((s = check_x(L, x, ldx)) != MOE_OK) return s;
+  if (!idx || !offsets || !perm || !inv || !xq || !xs) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(xq)) return MOE_ERR_MISALIGNED;
+  if ((s = check_ws(L, T, ws, ws_bytes)) != MOE_OK) return s;
+  Scratch sc = carve(L, T, ws);
+  return from_cuda(
+      launch_permute(L, x, T, ldx, idx, offsets, perm, inv, xq, xs, sc, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_expert_ffn(moe_layer_t L, const uint8_t* xq, const float* xs, const int32_t* offsets, int T,
+                          uint16_t* y, void* ws, size_t ws_bytes, void* stream) {
+  if (!L || T < 0 || T > kMaxT) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!xq || !xs || !offsets || !y) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(xq) || !aligned16(y)) return MOE_ERR_MISALIGNED;
+  moe_status s;
+  if ((s = check_ws(L, T, ws, ws_bytes)) != MOE_OK) return s;
+  Scratch sc = carve(L, T, ws);
+  return from_cuda(launch_expert_ffn(L, xq, xs, offsets, T, y, sc, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_combine(moe_layer_t L, const uint16_t* y, const int32_t* inv, const float* w, int T, uint16_t* out,
+                       int ldo, void* stream) {
+  if (!L || T < 0 || T > kMaxT) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!y || !inv || !w || !out || ldo < L->H) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(y) || !aligned16(out) || (size_t(ldo) * 2) % 16 != 0) return MOE_ERR_MISALIGNED;
+  return from_cuda(launch_combine(L, y, inv, w, T, out, ldo, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_layer_forward(moe_layer_t L, const uint16_t* x, int T, int ldx, uint16_t* out, int ldo, void* ws,
+                             size_t ws_bytes, void* stream) {
+  if (!L || T < 0 || T > kMaxT) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  moe_status s;
+  if ((s = check_x(L, x, ldx)) != MOE_OK) return s;
+  if (!out || ldo < L->H) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(out) || (size_t(ldo) * 2) % 16 != 0) return MOE_ERR_MISALIGNED;
+  if ((s = check_ws(L, T, ws, ws_bytes)) != MOE_OK) return s;
+  Scratch sc = carve(L, T, ws);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_route(L, x, T, ldx, sc.idx, sc.topw, nullptr, sc.route_partial, st);
+  if (e == cudaSuccess) e = launch_permute(L, x, T, ldx, sc.idx, sc.offsets, sc.perm, sc.inv, sc.xq, sc.xs, sc, st);
+  if (e == cudaSuccess) e = launch_expert_ffn(L, sc.xq, sc.xs, sc.offsets, T, sc.y, sc, st);
+  if (e == cudaSuccess) e = launch_combine(L, sc.y, sc.inv, sc.topw, T, out, ldo, st);
+  return from_cuda(e);
+}
+
+moe_status moe_get_device_status(moe_layer_t L, void* stream, uint32_t* detail) {
+  if (!L) return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return MOE_ERR_CUDA;
+  uint32_t v = 0;
+  if (cudaMemcpy(&v, L->status, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+  if (v && cudaMemset(L->status, 0, sizeof(v)) != cudaSuccess) return MOE_ERR_CUDA;
+  if (detail) *detail = v;
+  return v ? MOE_ERR_DEVICE : MOE_OK;
+}
+
+moe_status moe_test_grouped_gemm_f32(moe_layer_t L, int which, const uint8_t* a, const float* as,
+                                     const int32_t* offsets, int T, float* out, void* ws, size_t ws_bytes,
+                                     void* stream) {
+  if (!L || T < 0 || T > kMaxT || (which != 0 && which != 1)) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!a || !as || !offsets || !out) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(a)) return MOE_ERR_MISALIGNED;
+  moe_status s;
+  if ((s = check_ws(L, T, ws, ws_bytes)) != MOE_OK) return s;
+  Scratch sc = carve(L, T, ws);
+  return from_cuda(launch_test_gemm_f32(L, which, a, as, offsets, T, out, sc, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_test_workspace_h(moe_layer_t L, int T, size_t* h_offset, size_t* hs_offset) {
+  if (!L || T < 1 || T > kMaxT || !h_offset || !hs_offset) return MOE_ERR_INVALID_ARG;
+  Scratch s = carve(L, T, nullptr);
+  *h_offset = reinterpret_cast<size_t>(s.h);
+  *hs_offset = reinterpret_cast<size_t>(s.hs);
+  return MOE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,507 @@
+// Grouped FP8 GEMMs of the expert FFN with per-128-K-block scale promotion.
+//
+// Fine-grained FP8 (transformers PR #47844, "What does this PR do?"): E4M3
+// weights with one fp32 scale per 128 x 128 block and dynamically quantised
+// activations with one fp32 scale per token per 128 channels. Both scales are
+// constant over one 128-wide K block, so a GEMM over K = sum of K blocks is
+//   C[r, n] = sum_kb  P_kb[r, n] * sw[n/128, kb] * sa[r, kb],
+//   P_kb[r, n] = sum_{k in kb} qa[r, k] * qw[n, k]   (E4M3 x E4M3, fp32).
+// The tensor cores compute each P_kb (tcgen05.mma kind::f8f6f4, 4 MMAs of
+// K = 32 into a TMEM buffer); epilogue warps read it back and promote it into
+// an FP32 register accumulator with the scalar sw * sa of their row. The
+// scales are arbitrary fp32 values, which the hardware's power-of-two block
+// scaling cannot represent, hence the software promotion.
+//
+// Expert FFN (Dots3NoteTextConfig: hidden_act silu, mlp_bias False,
+// moe_intermediate_size 1536; SwiGLU experts with gate_proj, up_proj,
+// down_proj):
+//   gate/up GEMM: tile = 128 rows x (128 gate + 128 up channels of one
+//     128-channel block); the epilogue forms h = silu(G) * U in fp32 and
+//     quantises it per row per 128 channels (s = amax/448, E4M3 RNE), so the
+//     quantisation group is exactly one tile's channel block;
+//   down GEMM: tile = 128 rows x 256 output columns (two 128-column weight
+//     blocks); the epilogue rounds y to bf16.
+//
+// Kernel layout (one CTA per SM, persistent over a device-side tile list):
+//   warp 0      TMA producer: A tile 128 x 128 B, two B tiles 128 x 128 B per
+//               stage, 4-stage mbarrier ring (48 KB per stage, 128-byte swizzle)
+//   warp 1      TMEM allocator (512 columns) and single-thread MMA issuer;
+//               two 256-column TMEM buffers hold consecutive K-block partials
+//   warps 2-9   epilogue: warp w reads TMEM lanes 32*(w%4).. (its rows) and
+//               one half of the 256 columns; promotion, then the fused
+//               SwiGLU+quant or bf16 store.
+// Tile order: per group (expert), chunks of up to 8 row tiles, then the
+// n tiles, then the row tiles of the chunk -- the row tiles that share one
+// weight tile run side by side, so that weight tile comes from HBM once.
+//
+// Every wait is bounded (1 s); a timeout sets the layer's status word and
+// all roles leave their loops; the producer then waits for its own copies in
+// flight, the MMA thread for its own MMAs, and the TMEM is released.
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+
+namespace {
+
+constexpr int BM = 128;                    // rows per tile
+constexpr int BK = 128;                    // K bytes per stage = one scale block
+constexpr int BN = 256;                    // columns per tile (two 128-column halves)
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BK;           // 16 KB
+constexpr int BH_BYTES = 128 * BK;         // 16 KB per B half
+constexpr int STAGE_BYTES = A_BYTES + 2 * BH_BYTES;
+constexpr int EPI_WARPS = 8;
+constexpr int THREADS = 64 + EPI_WARPS * 32;
+constexpr int MCHUNK = 8;                  // row tiles per chunk of the tile order
+constexpr int MAX_GROUPS = 257;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t IDESC = idesc_e4m3_f32(BM, BN);
+constexpr int SMEM_DYN = STAGES * STAGE_BYTES + 1024;
+
+enum { MODE_GATEUP = 0, MODE_DOWN = 1 };
+enum { EPI_FUSED = 0, EPI_F32 = 1 };
+
+struct GemmArgs {
+  const int32_t* offsets;  // [ngroups + 1] row offsets of the groups
+  const int32_t* prefix;   // [ngroups + 1] exclusive tile prefix; [ngroups] = total
+  int ngroups;
+  int ntn;                 // n tiles per group
+  int nkb;                 // K blocks
+  int rows;                // rows in the permuted buffers
+  const float* as;         // activation scales [nkb][rows]
+  const float* ws0;        // weight scales [group][ws_nb][ws_kb]
+  const float* ws1;
+  int ws_nb, ws_kb;
+  int nb_count;            // valid 128-column output blocks (down GEMM)
+  uint8_t* h;              // gate/up: quantised h [rows][ld_h]
+  float* hs;               // gate/up: h scales [ntn][rows]
+  int ld_h;
+  uint16_t* y;             // down: y [rows][ld_y] bf16
+  int ld_y;
+  float* out;              // test: promoted accumulators [rows][ld_out]
+  int ld_out;
+  uint32_t* status;
+};
+
+struct TileInfo {
+  int g, nt, row0, nvalid;
+};
+
+__device__ __forceinline__ TileInfo decode_tile(int i, const int* s_prefix, const int* s_off, int ngroups, int ntn) {
+  int lo = 0, hi = ngroups - 1;
+  while (lo < hi) {  // last group whose prefix is <= i
+    const int mid = (lo + hi + 1) >> 1;
+    if (s_prefix[mid] <= i) lo = mid; else hi = mid - 1;
+  }
+  TileInfo t;
+  t.g = lo;
+  const int local = i - s_prefix[lo];
+  const int n_g = s_off[lo + 1] - s_off[lo];
+  const int mt = (n_g + BM - 1) / BM;
+  const int per_chunk = MCHUNK * ntn;
+  const int chunk = local / per_chunk;
+  const int within = local - chunk * per_chunk;
+  const int mc = min(MCHUNK, mt - chunk * MCHUNK);
+  t.nt = within / mc;
+  const int m = chunk * MCHUNK + (within - t.nt * mc);
+  t.row0 = s_off[lo] + m * BM;
+  t.nvalid = min(BM, n_g - m * BM);
+  return t;
+}
+
+// Bounded wait that ignores the abort flag (used to drain in-flight work).
+__device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity, uint32_t* status) {
+  int never = 0;
+  mbar_wait(bar, parity, &never, status);
+}
+
+template <int MODE, int EPI>
+__global__ void __launch_bounds__(THREADS, 1)
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
+                        const __grid_constant__ CUtensorMap tmB1, const GemmArgs p) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t full_bar[STAGES];
+  __shared__ __align__(8) uint64_t empty_bar[STAGES];
+  __shared__ __align__(8) uint64_t tfull_bar[2];
+  __shared__ __align__(8) uint64_t tempty_bar[2];
+  __shared__ __align__(8) uint64_t amax_bar[2];
+  __shared__ __align__(8) uint64_t done_bar;
+  __shared__ uint32_t tmem_base_s;
+  __shared__ int s_off[MAX_GROUPS + 1];
+  __shared__ int s_prefix[MAX_GROUPS + 1];
+  __shared__ float s_amax[2][2][BM];
+  __shared__ int s_abort_store;
+  __shared__ uint32_t s_consumed;
+  volatile int* s_abort = &s_abort_store;
+
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  for (int i = threadIdx.x; i <= p.ngroups; i += blockDim.x) {
+    s_off[i] = p.offsets[i];
+    s_prefix[i] = p.prefix[i];
+  }
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull_bar[b], 1);
+      mbar_init(&tempty_bar[b], EPI_WARPS);
+      mbar_init(&amax_bar[b], EPI_WARPS);
+    }
+    mbar_init(&done_bar, 1);
+    s_abort_store = 0;
+    s_consumed = 0;
+    fence_mbar_init();
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB0);
+    tma_prefetch_desc(&tmB1);
+  }
+  if (warp == 1) tmem_alloc(&tmem_base_s, TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = tmem_base_s;
+  const int total = s_prefix[p.ngroups];
+  uint32_t issued = 0;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      uint32_t it = 0;
+      bool ok = true;
+      for (int i = blockIdx.x; ok && i < total; i += gridDim.x) {
+        const TileInfo t = decode_tile(i, s_prefix, s_off, p.ngroups, p.ntn);
+        for (int kb = 0; kb < p.nkb; ++kb) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1u;
+          if (!mbar_wait(&empty_bar[s], ph ^ 1u, s_abort, p.status)) { ok = false; break; }
+          uint8_t* a = smem + s * STAGE_BYTES;
+          uint8_t* b = a + A_BYTES;
+          mbar_arrive_expect_tx(&full_bar[s], STAGE_BYTES);
+          tma_load_2d(a, &tmA, &full_bar[s], kb * BK, t.row0);
+          if (MODE == MODE_GATEUP) {
+            tma_load_3d(b, &tmB0, &full_bar[s], kb * BK, t.nt * 128, t.g);
+            tma_load_3d(b + BH_BYTES, &tmB1, &full_bar[s], kb * BK, t.nt * 128, t.g);
+          } else {
+            tma_load_3d(b, &tmB0, &full_bar[s], kb * BK, (2 * t.nt) * 128, t.g);
+            tma_load_3d(b + BH_BYTES, &tmB0, &full_bar[s], kb * BK, (2 * t.nt + 1) * 128, t.g);
+          }
+          ++it;
+        }
+      }
+      issued = it;
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      uint32_t it = 0, tb = 0;
+      bool ok = true;
+      for (int i = blockIdx.x; ok && i < total; i += gridDim.x) {
+        for (int kb = 0; kb < p.nkb; ++kb) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1u;
+          const uint32_t buf = tb & 1u, tph = (tb >> 1) & 1u;
+          if (!mbar_wait(&tempty_bar[buf], tph ^ 1u, s_abort, p.status)) { ok = false; break; }
+          if (!mbar_wait(&full_bar[s], ph, s_abort, p.status)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smem + s * STAGE_BYTES);
+          const uint64_t ad = smem_desc_sw128(a_addr);
+          const uint64_t bd = smem_desc_sw128(a_addr + A_BYTES);
+          const uint32_t d = tmem_base + buf * BN;
+#pragma unroll
+          for (int k = 0; k < BK / 32; ++k)   // advance 32 bytes of K = 2 in the 16-byte address field
+            mma_e4m3(d, ad + uint64_t(2 * k), bd + uint64_t(2 * k), IDESC, k > 0 ? 1u : 0u);
+          tc_commit(&empty_bar[s]);
+          tc_commit(&tfull_bar[buf]);
+          ++it;
+          ++tb;
+        }
+      }
+      s_consumed = it;
+      tc_commit(&done_bar);                 // all MMAs issued above have completed
+      mbar_wait_drain(&done_bar, 0, p.status);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int ew = warp - 2;
+    const int q = warp & 3;          // TMEM lane quarter this warp may access
+    const int half = ew >> 2;        // column half of the tile
+    const int r_in = q * 32 + lane;  // row within the tile
+    uint32_t tb = 0;
+    uint32_t tile_iter = 0;
+    bool ok = true;
+    for (int i = blockIdx.x; ok && i < total; i += gridDim.x, ++tile_iter) {
+      const TileInfo t = decode_tile(i, s_prefix, s_off, p.ngroups, p.ntn);
+      const bool warp_active = q * 32 < t.nvalid;
+      const bool valid = r_in < t.nvalid;
+      const int row = t.row0 + r_in;
+      const float* w0;
+      const float* w1;
+      int nb = 0;
+      if (MODE == MODE_GATEUP) {
+        w0 = p.ws0 + (size_t(t.g) * p.ws_nb + t.nt) * p.ws_kb;
+        w1 = p.ws1 + (size_t(t.g) * p.ws_nb + t.nt) * p.ws_kb;
+      } else {
+        nb = 2 * t.nt + half;
+        w0 = p.ws0 + (size_t(t.g) * p.ws_nb + min(nb, p.ws_nb - 1)) * p.ws_kb;
+        w1 = w0;
+      }
+      float acc[128];
+#pragma unroll
+      for (int j = 0; j < 128; ++j) acc[j] = 0.0f;
+
+      for (int kb = 0; kb < p.nkb; ++kb) {
+        const uint32_t buf = tb & 1u, tph = (tb >> 1) & 1u;
+        const float sa = valid ? __ldg(p.as + size_t(kb) * p.rows + row) : 0.0f;
+        const float f0 = __ldg(w0 + kb) * sa;
+        const float f1 = __ldg(w1 + kb) * sa;
+        if (!mbar_wait(&tfull_bar[buf], tph, s_abort, p.status)) { ok = false; break; }
+        tc_fence_after();
+        if (warp_active) {
+          const uint32_t tbase = tmem_base + (uint32_t(q * 32) << 16) + buf * BN;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const uint32_t col = (MODE == MODE_GATEUP) ? uint32_t((c >> 1) * 128 + half * 64 + (c & 1) * 32)
+                                                       : uint32_t(half * 128 + c * 32);
+            float v[32];
+            tmem_ld32(tbase + col, v);
+            tmem_ld_wait();
+            const float f = (MODE == MODE_GATEUP && c >= 2) ? f1 : f0;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) acc[c * 32 + j] = fmaf(v[j], f, acc[c * 32 + j]);
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty_bar[buf]);
+        ++tb;
+      }
+      if (!ok) break;
+
+      if (EPI == EPI_F32) {
+        if (valid) {
+          float* dst = p.out + size_t(row) * p.ld_out;
+          if (MODE == MODE_GATEUP) {
+#pragma unroll
+            for (int j = 0; j < 64; ++j) {
+              dst[t.nt * 256 + half * 64 + j] = acc[j];
+              dst[t.nt * 256 + 128 + half * 64 + j] = acc[64 + j];
+            }
+          } else if (nb < p.nb_count) {
+#pragma unroll
+            for (int j = 0; j < 128; ++j) dst[nb * 128 + j] = acc[j];
+          }
+        }
+      } else if (MODE == MODE_GATEUP) {
+        // h = silu(G) * U for this thread's 64 channels, then the row's
+        // 128-channel amax across the two column halves.
+        float amax = 0.0f;
+#pragma unroll
+        for (int j = 0; j < 64; ++j) {
+          const float g = acc[j];
+          const float hv = g / (1.0f + expf(-g)) * acc[64 + j];
+          acc[j] = hv;
+          amax = fmaxf(amax, fabsf(hv));
+        }
+        const uint32_t xb = tile_iter & 1u;
+        s_amax[xb][half][r_in] = amax;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&amax_bar[xb]);
+        if (!mbar_wait(&amax_bar[xb], (tile_iter >> 1) & 1u, s_abort, p.status)) { ok = false; break; }
+        amax = fmaxf(amax, s_amax[xb][half ^ 1][r_in]);
+        if (valid) {
+          uint32_t pk[16];
+          float s = 0.0f;
+          if (amax > 0.0f) {
+            s = __fdiv_rn(amax, 448.0f);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const uint32_t lo = e4m3x2(__fdiv_rn(acc[4 * j], s), __fdiv_rn(acc[4 * j + 1], s));
+              const uint32_t hi = e4m3x2(__fdiv_rn(acc[4 * j + 2], s), __fdiv_rn(acc[4 * j + 3], s));
+              pk[j] = lo | (hi << 16);
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) pk[j] = 0u;
+          }
+          uint8_t* dst = p.h + size_t(row) * p.ld_h + t.nt * 128 + half * 64;
+#pragma unroll
+          for (int v = 0; v < 4; ++v)
+            *reinterpret_cast<uint4*>(dst + 16 * v) = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+          if (half == 0) p.hs[size_t(t.nt) * p.rows + row] = s;
+        }
+      } else {
+        if (valid && nb < p.nb_count) {
+          uint16_t* dst = p.y + size_t(row) * p.ld_y + nb * 128;
+#pragma unroll
+          for (int v = 0; v < 16; ++v) {
+            uint32_t o[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              o[j] = uint32_t(f32_to_bf16_bits(acc[8 * v + 2 * j])) |
+                     (uint32_t(f32_to_bf16_bits(acc[8 * v + 2 * j + 1])) << 16);
+            *reinterpret_cast<uint4*>(dst + 8 * v) = make_uint4(o[0], o[1], o[2], o[3]);
+          }
+        }
+      }
+    }
+  }
+
+  // ------------------------------------------------------------ teardown
+  __syncthreads();
+  if (warp == 0 && lane == 0) {
+    // copies issued but never consumed (only after an abort) must land first
+    for (uint32_t j = s_consumed; j < issued; ++j) mbar_wait_drain(&full_bar[j % STAGES], (j / STAGES) & 1u, p.status);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+// Exclusive tile prefix of both GEMMs from the group offsets:
+// plan[0 .. ng]          gate/up (ntn_gu n tiles per group)
+// plan[ng+1 .. 2ng+1]    down    (ntn_dn n tiles per group)
+__global__ void __launch_bounds__(512) tile_plan_kernel(const int32_t* __restrict__ offsets, int ng, int ntn_gu,
+                                                        int ntn_dn, int32_t* __restrict__ plan) {
+  __shared__ int sums[2][16];
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  int mt = 0;
+  if (tid < ng) mt = (offsets[tid + 1] - offsets[tid] + BM - 1) / BM;
+  int v[2] = {mt * ntn_gu, mt * ntn_dn};
+  int incl[2] = {v[0], v[1]};
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const int o = __shfl_up_sync(0xFFFFFFFFu, incl[j], off);
+      if (lane >= off) incl[j] += o;
+    }
+  }
+  if (lane == 31) { sums[0][wid] = incl[0]; sums[1][wid] = incl[1]; }
+  __syncthreads();
+  int base[2] = {0, 0};
+  for (int j = 0; j < wid; ++j) { base[0] += sums[0][j]; base[1] += sums[1][j]; }
+  if (tid < ng) {
+    plan[tid] = base[0] + incl[0] - v[0];
+    plan[ng + 1 + tid] = base[1] + incl[1] - v[1];
+  }
+  if (tid == ng - 1) {
+    plan[ng] = base[0] + incl[0];
+    plan[ng + 1 + ng] = base[1] + incl[1];
+  }
+}
+
+template <int MODE, int EPI>
+cudaError_t launch_gemm(const moe_layer_s* L, const CUtensorMap& tmA, const CUtensorMap& tmB0,
+                        const CUtensorMap& tmB1, const GemmArgs& a, cudaStream_t st) {
+  static bool configured = false;  // per process; the attribute is per function
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<MODE, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         SMEM_DYN);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  // upper bound on the number of tiles: every group may add one partial row tile
+  const long long bound = (static_cast<long long>(a.rows) / BM + a.ngroups) * a.ntn;
+  const int grid = int(bound < L->num_sms ? bound : L->num_sms);
+  if (grid <= 0) return cudaSuccess;
+  grouped_gemm_kernel<MODE, EPI><<<grid, THREADS, SMEM_DYN, st>>>(tmA, tmB0, tmB1, a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+static GemmArgs gateup_args(const moe_layer_s* L, const int32_t* offsets, const int32_t* plan, int rows,
+                            const float* xs) {
+  GemmArgs a = {};
+  a.offsets = offsets;
+  a.prefix = plan;
+  a.ngroups = L->E + 1;
+  a.ntn = L->FB;
+  a.nkb = L->HB;
+  a.rows = rows;
+  a.as = xs;
+  a.ws0 = L->w.s_gate;
+  a.ws1 = L->w.s_up;
+  a.ws_nb = L->FB;
+  a.ws_kb = L->HB;
+  a.nb_count = L->FB;
+  a.status = L->status;
+  return a;
+}
+
+static GemmArgs down_args(const moe_layer_s* L, const int32_t* offsets, const int32_t* plan, int rows,
+                          const float* hs) {
+  GemmArgs a = {};
+  a.offsets = offsets;
+  a.prefix = plan + (L->E + 2);
+  a.ngroups = L->E + 1;
+  a.ntn = (L->HB + 1) / 2;
+  a.nkb = L->FB;
+  a.rows = rows;
+  a.as = hs;
+  a.ws0 = L->w.s_down;
+  a.ws1 = L->w.s_down;
+  a.ws_nb = L->HB;
+  a.ws_kb = L->FB;
+  a.nb_count = L->HB;
+  a.status = L->status;
+  return a;
+}
+
+static cudaError_t launch_plan(const moe_layer_s* L, const int32_t* offsets, int32_t* plan, cudaStream_t st) {
+  tile_plan_kernel<<<1, 512, 0, st>>>(offsets, L->E + 1, L->FB, (L->HB + 1) / 2, plan);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_expert_ffn(const moe_layer_s* L, const uint8_t* xq, const float* xs, const int32_t* offsets,
+                              int T, uint16_t* y, const Scratch& s, cudaStream_t st) {
+  const int rows = T * (L->K + 1);
+  cudaError_t e = launch_plan(L, offsets, s.plan, st);
+  if (e != cudaSuccess) return e;
+  CUtensorMap tmX, tmH;
+  if (!encode_tmap_u8(&tmX, xq, L->H, rows, 1, L->H, 0)) return cudaErrorInvalidValue;
+  if (!encode_tmap_u8(&tmH, s.h, L->F, rows, 1, L->ld_hh, 0)) return cudaErrorInvalidValue;
+  GemmArgs gu = gateup_args(L, offsets, s.plan, rows, xs);
+  gu.h = s.h;
+  gu.hs = s.hs;
+  gu.ld_h = L->ld_hh;
+  e = launch_gemm<MODE_GATEUP, EPI_FUSED>(L, tmX, L->tm_gate, L->tm_up, gu, st);
+  if (e != cudaSuccess) return e;
+  GemmArgs dn = down_args(L, offsets, s.plan, rows, s.hs);
+  dn.y = y;
+  dn.ld_y = L->H;
+  return launch_gemm<MODE_DOWN, EPI_FUSED>(L, tmH, L->tm_down, L->tm_down, dn, st);
+}
+
+cudaError_t launch_test_gemm_f32(const moe_layer_s* L, int which, const uint8_t* a_ptr, const float* as,
+                                 const int32_t* offsets, int T, float* out, const Scratch& s, cudaStream_t st) {
+  const int rows = T * (L->K + 1);
+  cudaError_t e = launch_plan(L, offsets, s.plan, st);
+  if (e != cudaSuccess) return e;
+  CUtensorMap tmA;
+  if (which == 0) {
+    if (!encode_tmap_u8(&tmA, a_ptr, L->H, rows, 1, L->H, 0)) return cudaErrorInvalidValue;
+    GemmArgs a = gateup_args(L, offsets, s.plan, rows, as);
+    a.out = out;
+    a.ld_out = 2 * L->FB * 128;
+    return launch_gemm<MODE_GATEUP, EPI_F32>(L, tmA, L->tm_gate, L->tm_up, a, st);
+  }
+  if (!encode_tmap_u8(&tmA, a_ptr, L->F, rows, 1, L->ld_hh, 0)) return cudaErrorInvalidValue;
+  GemmArgs a = down_args(L, offsets, s.plan, rows, as);
+  a.out = out;
+  a.ld_out = L->H;
+  return launch_gemm<MODE_DOWN, EPI_F32>(L, tmA, L->tm_down, L->tm_down, a, st);
+}
+
+}  // namespace moe

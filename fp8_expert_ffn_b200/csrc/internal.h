@@ -1,0 +1,74 @@
+// Host-side layer handle and the launchers each .cu file provides.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+
+#include "../../include/moe.h"
+
+struct moe_layer_s {
+  moe_layer_desc d;
+  moe_weights w;
+  int H, E, K, F;
+  int HB;        // H / 128
+  int FB;        // ceil(F / 128)
+  int ld_hh;     // row stride of the quantised SwiGLU output h: FB * 128
+  int device;
+  int num_sms;
+  uint32_t* status;  // device status word
+  CUtensorMap tm_gate;  // [E+1][F][ld_h] E4M3, box 128 x 128 x 1
+  CUtensorMap tm_up;
+  CUtensorMap tm_down;  // [E+1][H][ld_f] E4M3, box 128 x 128 x 1
+};
+
+namespace moe {
+
+// Workspace carving shared by every entry point.
+struct Scratch {
+  // route
+  float* route_partial;   // [S][T][E]
+  // permute
+  uint32_t* bitmap;       // [E][W]
+  uint32_t* wprefix;      // [E][W]
+  int32_t* counts;        // [E]
+  // expert ffn
+  int32_t* plan;          // tile plans (two GEMMs)
+  uint8_t* h;             // [rows][ld_hh]
+  float* hs;              // [FB][rows]
+  // forward intermediates
+  int32_t* idx;           // [T][K]
+  float* topw;            // [T][K]
+  int32_t* offsets;       // [E+2]
+  int32_t* perm;          // [rows]
+  int32_t* inv;           // [T][K]
+  uint8_t* xq;            // [rows][H]
+  float* xs;              // [HB][rows]
+  uint16_t* y;            // [rows][H]
+  size_t total;
+};
+
+int route_splits(const moe_layer_s* L, int T);
+Scratch carve(const moe_layer_s* L, int T, void* base);
+constexpr int kPlanInts(int E) { return 2 * (E + 2) + 8; }
+
+cudaError_t launch_route(const moe_layer_s* L, const uint16_t* x, int T, int ldx, int32_t* idx, float* w,
+                         float* logits, float* partial, cudaStream_t st);
+cudaError_t launch_permute(const moe_layer_s* L, const uint16_t* x, int T, int ldx, const int32_t* idx,
+                           int32_t* offsets, int32_t* perm, int32_t* inv, uint8_t* xq, float* xs,
+                           const Scratch& s, cudaStream_t st);
+cudaError_t launch_expert_ffn(const moe_layer_s* L, const uint8_t* xq, const float* xs, const int32_t* offsets,
+                              int T, uint16_t* y, const Scratch& s, cudaStream_t st);
+cudaError_t launch_test_gemm_f32(const moe_layer_s* L, int which, const uint8_t* a, const float* as,
+                                 const int32_t* offsets, int T, float* out, const Scratch& s, cudaStream_t st);
+cudaError_t launch_combine(const moe_layer_s* L, const uint16_t* y, const int32_t* inv, const float* w, int T,
+                           uint16_t* out, int ldo, cudaStream_t st);
+
+// TMA descriptor for a row-major byte matrix [rows][inner] with row stride
+// `ld` bytes, 128 x 128 boxes, 128-byte swizzle (3-D when depth > 1).
+bool encode_tmap_u8(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t rows, uint64_t depth,
+                    uint64_t ld, uint64_t depth_stride);
+
+}  // namespace moe

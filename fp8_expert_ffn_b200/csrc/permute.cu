@@ -1,0 +1,176 @@
+// Token permutation by expert with the dynamic activation quantiser fused
+// into the gather.
+//
+// Grouping tokens by expert is the "dispatch" of the pages' DeepEP transport
+// (SGLang cookbook "Dots3-Note", "2. Configuration Tips", MoE runner); on one
+// GPU it is a counting sort. Activation quantisation follows transformers
+// PR #47844 ("What does this PR do?": dynamic activations, E4M3): per token
+// per 128 channels, s = fp32(amax) / 448, q = E4M3_RNE_satfinite(x / s), both
+// divisions IEEE fp32; an all-zero group gives s = 0 and q = 0.
+//
+// Determinism without ordering atomics: every (token, expert) pair sets one
+// bit of a per-expert token bitmap (atomicOr, order-independent). The row of
+// (t, k) inside expert e's group is the number of earlier tokens that chose
+// e: a prefix popcount over e's bitmap words. Kernels:
+//   1. permute_bitmap   one thread per (t, k): validate, set the bit
+//   2. permute_count    one CTA per expert: per-word prefix popcounts, count
+//   3. permute_offsets  one CTA: exclusive scan of counts -> offsets[E+2]
+//   4. permute_gather   one warp per token: rows of its K slots and its
+//                       shared-expert row, inv/perm, then the 128-channel
+//                       groups of x quantised once and stored to all rows.
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+
+namespace {
+
+__global__ void permute_bitmap_kernel(const int32_t* __restrict__ idx, int T, int K, int E, int W,
+                                      uint32_t* __restrict__ bitmap, uint32_t* status) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= T * K) return;
+  const int t = i / K;
+  const int e = idx[i];
+  if (e < 0 || e >= E) {
+    set_status(status, STATUS_BAD_EXPERT);
+    return;
+  }
+  const uint32_t bit = 1u << (t & 31);
+  const uint32_t old = atomicOr(&bitmap[size_t(e) * W + (t >> 5)], bit);
+  if (old & bit) set_status(status, STATUS_DUP_EXPERT);
+}
+
+// One CTA (256 threads) per expert: wprefix[e][w] = set bits of e's words
+// before word w; counts[e] = all set bits.
+__global__ void __launch_bounds__(256) permute_count_kernel(const uint32_t* __restrict__ bitmap, int W,
+                                                            uint32_t* __restrict__ wprefix,
+                                                            int32_t* __restrict__ counts) {
+  __shared__ uint32_t warp_sums[8];
+  const int e = blockIdx.x, tid = threadIdx.x;
+  const uint32_t* row = bitmap + size_t(e) * W;
+  uint32_t* out = wprefix + size_t(e) * W;
+  const int per = (W + 255) / 256;
+  const int w0 = min(W, tid * per), w1 = min(W, w0 + per);
+  uint32_t local = 0;
+  for (int w = w0; w < w1; ++w) local += __popc(row[w]);
+  // exclusive scan of `local` over the CTA
+  const int lane = tid & 31, wid = tid >> 5;
+  uint32_t incl = local;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    uint32_t v = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+    if (lane >= off) incl += v;
+  }
+  if (lane == 31) warp_sums[wid] = incl;
+  __syncthreads();
+  uint32_t base = 0;
+  for (int j = 0; j < wid; ++j) base += warp_sums[j];
+  uint32_t run = base + incl - local;
+  for (int w = w0; w < w1; ++w) {
+    out[w] = run;
+    run += __popc(row[w]);
+  }
+  if (tid == 255) counts[e] = int32_t(base + incl);
+}
+
+// offsets[g] = sum of counts[0..g), offsets[E+1] = offsets[E] + T.
+__global__ void __launch_bounds__(256) permute_offsets_kernel(const int32_t* __restrict__ counts, int E, int T,
+                                                              int32_t* __restrict__ offsets) {
+  __shared__ int32_t warp_sums[8];
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  const int v = tid < E ? counts[tid] : 0;
+  int incl = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    int o = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+    if (lane >= off) incl += o;
+  }
+  if (lane == 31) warp_sums[wid] = incl;
+  __syncthreads();
+  int base = 0;
+  for (int j = 0; j < wid; ++j) base += warp_sums[j];
+  if (tid < E) offsets[tid] = base + incl - v;
+  if (tid == E - 1) {
+    offsets[E] = base + incl;
+    offsets[E + 1] = base + incl + T;
+  }
+}
+
+// One warp per token. Lane k < K owns slot k; lane K owns the shared row.
+__global__ void __launch_bounds__(256) permute_gather_kernel(
+    const uint16_t* __restrict__ x, int T, int ldx, int H, const int32_t* __restrict__ idx, int K, int E, int W,
+    const uint32_t* __restrict__ bitmap, const uint32_t* __restrict__ wprefix, const int32_t* __restrict__ offsets,
+    int rows, int32_t* __restrict__ perm, int32_t* __restrict__ inv, uint8_t* __restrict__ xq,
+    float* __restrict__ xs) {
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (t >= T) return;
+  int my_row = -1;
+  if (lane < K) {
+    const int e = idx[size_t(t) * K + lane];
+    bool ok = (e >= 0 && e < E);
+    for (int j = 0; j < lane && ok; ++j) ok = (idx[size_t(t) * K + j] != e);  // first slot of a repeat wins
+    if (ok) {
+      const uint32_t word = bitmap[size_t(e) * W + (t >> 5)];
+      my_row = offsets[e] + int(wprefix[size_t(e) * W + (t >> 5)]) + __popc(word & ((1u << (t & 31)) - 1u));
+    }
+    inv[size_t(t) * K + lane] = my_row;
+  } else if (lane == K) {
+    my_row = offsets[E] + t;
+  }
+  if (my_row >= 0) perm[my_row] = t;
+  // rows of this token, known to every lane
+  int rowv[9];
+#pragma unroll
+  for (int j = 0; j < 9; ++j) rowv[j] = __shfl_sync(0xFFFFFFFFu, my_row, j);
+
+  const uint16_t* xr = x + size_t(t) * ldx;
+  const int HB = H / 128;
+  for (int g = 0; g < HB; ++g) {
+    // lane holds channels g*128 + lane*4 .. +3
+    const uint2 raw = *reinterpret_cast<const uint2*>(xr + g * 128 + lane * 4);
+    float v[4] = {bf16_bits_to_f32(uint16_t(raw.x & 0xFFFFu)), bf16_bits_to_f32(uint16_t(raw.x >> 16)),
+                  bf16_bits_to_f32(uint16_t(raw.y & 0xFFFFu)), bf16_bits_to_f32(uint16_t(raw.y >> 16))};
+    float amax = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
+    uint32_t packed = 0;
+    float s = 0.0f;
+    if (amax > 0.0f) {
+      s = __fdiv_rn(amax, 448.0f);
+      const uint32_t lo = e4m3x2(__fdiv_rn(v[0], s), __fdiv_rn(v[1], s));
+      const uint32_t hi = e4m3x2(__fdiv_rn(v[2], s), __fdiv_rn(v[3], s));
+      packed = lo | (hi << 16);
+    }
+#pragma unroll
+    for (int j = 0; j < 9; ++j) {
+      if (j > K) break;
+      const int r = rowv[j];
+      if (r < 0) continue;
+      *reinterpret_cast<uint32_t*>(xq + size_t(r) * H + g * 128 + lane * 4) = packed;
+      if (lane == j) xs[size_t(g) * rows + r] = s;
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_permute(const moe_layer_s* L, const uint16_t* x, int T, int ldx, const int32_t* idx,
+                           int32_t* offsets, int32_t* perm, int32_t* inv, uint8_t* xq, float* xs,
+                           const Scratch& s, cudaStream_t st) {
+  const int K = L->K, E = L->E, W = (T + 31) / 32;
+  const int rows = T * (K + 1);
+  cudaError_t e = cudaMemsetAsync(s.bitmap, 0, sizeof(uint32_t) * size_t(E) * W, st);
+  if (e != cudaSuccess) return e;
+  permute_bitmap_kernel<<<(T * K + 255) / 256, 256, 0, st>>>(idx, T, K, E, W, s.bitmap, L->status);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  permute_count_kernel<<<E, 256, 0, st>>>(s.bitmap, W, s.wprefix, s.counts);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  permute_offsets_kernel<<<1, 256, 0, st>>>(s.counts, E, T, offsets);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  permute_gather_kernel<<<(T + 7) / 8, 256, 0, st>>>(x, T, ldx, L->H, idx, K, E, W, s.bitmap, s.wprefix, offsets,
+                                                     rows, perm, inv, xq, xs);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,200 @@
+/*
+ * fp8_expert_ffn_b200 — forward pass of one fine-grained-FP8 Mixture-of-Experts
+ * layer (dots3-note preview shape) on a B200 (sm_100a).
+ *
+ * The layer (transformers docs page "Dots 3 Note Preview", Dots3NoteTextConfig;
+ * model card dots-studio/dots3-note-prev, "Model Overview"): hidden size H,
+ * E routed SwiGLU experts plus 1 shared expert, top-K routing with the K
+ * weights renormalised (norm_topk_prob), expert FFN width F, no biases.
+ * Weights are a fine-grained FP8 checkpoint (transformers PR #47844, "What
+ * does this PR do?"): E4M3 codes with one fp32 scale per 128 x 128 block;
+ * activations are quantised at run time per token per 128 channels.
+ *
+ * Readings taken where the pages are silent (all fixed here):
+ *   - router logits are FP32; top-K by logit (equivalently by softmax
+ *     probability), ties to the lower expert id; the K weights are the
+ *     softmax over the K selected logits (= softmax over all E experts
+ *     renormalised over the selection), times routed_scaling;
+ *   - the K slots of a token are listed in ascending expert id;
+ *   - E4M3 is the OCP "FN" flavour (max 448, no infinities); quantisation
+ *     is s = fp32(amax)/448 (IEEE fp32 divide), q = E4M3_RNE_satfinite(v/s)
+ *     (IEEE fp32 divide); an all-zero group gives s = 0 and q = 0;
+ *   - scales are dequantisation multipliers: value ~ decode(q) * s;
+ *   - the SwiGLU output h is quantised the same way from fp32, per row per
+ *     128 channels, before the down projection;
+ *   - the shared expert (index E in every weight array) is added with
+ *     weight 1; its rows follow the routed rows in token order.
+ *
+ * Conventions for every call:
+ *   - all data pointers are DEVICE pointers owned by the caller; the library
+ *     never allocates after moe_layer_create (which allocates one 4-byte
+ *     device status word and nothing else);
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default);
+ *     calls are asynchronous on that stream and never synchronise the host;
+ *   - bf16 tensors are passed as uint16_t bit patterns;
+ *   - row strides (ld*) are in elements; every byte stride must be a
+ *     multiple of 16 and every base pointer 16-byte aligned, else
+ *     MOE_ERR_MISALIGNED;
+ *   - T = 0 is a no-op that returns MOE_OK;
+ *   - inputs must be finite; NaN/Inf inputs give unspecified results;
+ *   - errors found by the host are returned before anything is launched;
+ *     errors found on the device (an expert id out of range, a repeated
+ *     expert in one token's slots, a pipeline wait that timed out) set the
+ *     layer's device status word, skip the offending work and are read back
+ *     with moe_get_device_status.
+ *
+ * Row count: R = T*K routed rows plus T shared rows, rows = T*(K+1).
+ */
+#ifndef FP8_EXPERT_FFN_MOE_H
+#define FP8_EXPERT_FFN_MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,  /* null pointer, bad size or count */
+  MOE_ERR_MISALIGNED = 2,   /* pointer or byte stride not 16-byte aligned */
+  MOE_ERR_UNSUPPORTED = 3,  /* a layer shape this build does not handle */
+  MOE_ERR_WORKSPACE = 4,    /* workspace smaller than moe_workspace_size */
+  MOE_ERR_CUDA = 5,         /* a CUDA runtime/driver call failed */
+  MOE_ERR_DEVICE = 6        /* a kernel reported bad data or a timed-out wait */
+} moe_status;
+
+/* Layer description; mirrors Dots3NoteTextConfig (transformers docs page
+ * "Dots 3 Note Preview"): hidden_size, n_routed_experts, n_shared_experts,
+ * num_experts_per_tok, moe_intermediate_size, shared_experts_intermediate_size,
+ * routed_scaling_factor, norm_topk_prob; block = the 128 x 128 weight block
+ * edge of transformers PR #47844. This build requires: hidden % 128 == 0,
+ * 128 <= hidden <= 16384, 1 <= n_routed <= 256, n_shared == 1,
+ * 1 <= top_k <= min(8, n_routed), 1 <= ffn <= 4096, shared_ffn == ffn,
+ * block == 128, norm_topk == 1; otherwise MOE_ERR_UNSUPPORTED. */
+typedef struct {
+  int hidden;           /* H */
+  int n_routed;         /* E */
+  int n_shared;         /* must be 1 */
+  int top_k;            /* K */
+  int ffn;              /* F */
+  int shared_ffn;       /* must equal ffn */
+  int block;            /* must be 128 */
+  float routed_scaling; /* multiplies the renormalised routed weights */
+  int norm_topk;        /* must be 1 */
+} moe_layer_desc;
+
+/* Caller-owned device weights; they must outlive the layer handle. Expert
+ * index E is the shared expert. Codes are E4M3 bytes; scales are fp32
+ * dequantisation multipliers, one per 128 x 128 block (edge blocks cover the
+ * real rows/columns only):
+ *   w_gate, w_up : [E+1][F][ld_h]   bytes, ld_h >= H, ld_h % 16 == 0
+ *   s_gate, s_up : [E+1][ceil(F/128)][H/128]
+ *   w_down       : [E+1][H][ld_f]   bytes, ld_f >= F, ld_f % 16 == 0
+ *   s_down       : [E+1][H/128][ceil(F/128)]
+ *   router_w     : [E][H] fp32, row-major                                  */
+typedef struct {
+  const uint8_t* w_gate;
+  const uint8_t* w_up;
+  const uint8_t* w_down;
+  const float* s_gate;
+  const float* s_up;
+  const float* s_down;
+  const float* router_w;
+  int ld_h;
+  int ld_f;
+} moe_weights;
+
+typedef struct moe_layer_s* moe_layer_t;
+
+/* Static description of a status code (never NULL). */
+const char* moe_status_string(moe_status s);
+
+/* Validates desc/weights, queries the current device (must be sm_100),
+ * encodes the weights' TMA descriptors once and allocates the 4-byte device
+ * status word. On error *out is NULL. */
+moe_status moe_layer_create(const moe_layer_desc* desc, const moe_weights* w, moe_layer_t* out);
+
+/* Frees the handle (not the caller's weights). NULL is accepted. */
+moe_status moe_layer_destroy(moe_layer_t layer);
+
+/* Bytes of workspace that moe_layer_forward needs for T tokens; it also
+ * covers the scratch of moe_permute and moe_expert_ffn. 0 on bad input. */
+size_t moe_workspace_size(moe_layer_t layer, int T);
+
+/* Router: logits = x . router_w^T in FP32, top-K experts per token (ties to
+ * the lower id, slots in ascending id), weights = softmax over the K selected
+ * logits times routed_scaling.
+ *   x             [T][ldx] bf16, ldx >= H
+ *   topk_idx      [T][K] int32 (out)
+ *   topk_w        [T][K] fp32  (out)
+ *   router_logits [T][E] fp32  (out, may be NULL)
+ *   ws, ws_bytes  scratch, at least moe_workspace_size(layer, T) bytes    */
+moe_status moe_route(moe_layer_t layer, const uint16_t* x, int T, int ldx, int32_t* topk_idx, float* topk_w,
+                     float* router_logits, void* ws, size_t ws_bytes, void* stream);
+
+/* Token permutation by expert with fused activation quantisation.
+ * Counting sort of the T*K (token, slot) pairs by expert id, stable in token
+ * order; group E (shared expert) holds rows [T*K, T*K+T) in token order.
+ *   topk_idx  [T][K] int32 (in); ids outside [0,E) or repeated within a
+ *             token set MOE_ERR_DEVICE and are skipped
+ *   offsets   [E+2] int32 (out): group g is rows [offsets[g], offsets[g+1])
+ *   perm      [rows] int32 (out): row -> token
+ *   inv       [T][K] int32 (out): (token, slot) -> row
+ *   xq        [rows][H] E4M3 bytes (out): x of the row's token, quantised
+ *             per 128 channels
+ *   xs        [H/128][rows] fp32 (out, group-major): the row's scales      */
+moe_status moe_permute(moe_layer_t layer, const uint16_t* x, int T, int ldx, const int32_t* topk_idx,
+                       int32_t* offsets, int32_t* perm, int32_t* inv, uint8_t* xq, float* xs, void* ws,
+                       size_t ws_bytes, void* stream);
+
+/* Grouped expert FFN over the permuted rows: for each group g and row r in
+ * it, h = silu(xq Wg_g^T) * (xq Wu_g^T) with per-128-K-block scale promotion,
+ * h quantised per 128 channels (E4M3, fp32 scale), y = h Wd_g^T in FP32,
+ * rounded to bf16.
+ *   xq, xs, offsets as written by moe_permute for the same T
+ *   y         [rows][H] bf16 (out)                                         */
+moe_status moe_expert_ffn(moe_layer_t layer, const uint8_t* xq, const float* xs, const int32_t* offsets, int T,
+                          uint16_t* y, void* ws, size_t ws_bytes, void* stream);
+
+/* out[t] = bf16_RNE( sum_k topk_w[t,k] * y[inv[t,k]] + y[T*K + t] ), FP32
+ * sum in slot order, shared row last.
+ *   out [T][ldo] bf16, ldo >= H                                            */
+moe_status moe_combine(moe_layer_t layer, const uint16_t* y, const int32_t* inv, const float* topk_w, int T,
+                       uint16_t* out, int ldo, void* stream);
+
+/* The whole layer: moe_route -> moe_permute -> moe_expert_ffn -> moe_combine,
+ * with every intermediate in the workspace. */
+moe_status moe_layer_forward(moe_layer_t layer, const uint16_t* x, int T, int ldx, uint16_t* out, int ldo,
+                             void* ws, size_t ws_bytes, void* stream);
+
+/* Synchronises `stream`, returns MOE_ERR_DEVICE if any kernel of this layer
+ * flagged an error since the last call (and clears the flag), else MOE_OK.
+ * If `detail` is not NULL it receives the raw status bits. */
+moe_status moe_get_device_status(moe_layer_t layer, void* stream, uint32_t* detail);
+
+/* Test hook for the grouped FP8 GEMM with per-128-K-block promotion: writes
+ * the promoted FP32 accumulators instead of the fused epilogue.
+ *   which = 0: gate/up GEMM; a = xq [rows][H], as = [H/128][rows];
+ *              out [rows][2*ceil(F/128)*128] fp32, channel block c of the
+ *              gate result at columns [256c, 256c+128), of the up result at
+ *              [256c+128, 256c+256)
+ *   which = 1: down GEMM; a = h [rows][ceil(F/128)*128] (bytes beyond F are
+ *              ignored), as = [ceil(F/128)][rows]; out [rows][H] fp32
+ * offsets gives the groups as in moe_permute; rows = T*(K+1). */
+moe_status moe_test_grouped_gemm_f32(moe_layer_t layer, int which, const uint8_t* a, const float* as,
+                                     const int32_t* offsets, int T, float* out, void* ws, size_t ws_bytes,
+                                     void* stream);
+
+/* Test hook: byte offsets, inside a workspace for T tokens, of the quantised
+ * SwiGLU output that moe_expert_ffn leaves there: h [rows][ceil(F/128)*128]
+ * E4M3 bytes (channels >= F are zero) and its scales hs [ceil(F/128)][rows]
+ * fp32. They stay valid until the workspace is reused. */
+moe_status moe_test_workspace_h(moe_layer_t layer, int T, size_t* h_offset, size_t* hs_offset);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP8_EXPERT_FFN_MOE_H */

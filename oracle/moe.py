@@ -32,6 +32,8 @@ Steps and the readings taken where the pages are silent:
 """
 from __future__ import annotations
 
+import os
+from concurrent.futures import ThreadPoolExecutor
 from dataclasses import dataclass
 
 import numpy as np
@@ -40,6 +42,17 @@ from . import e4m3
 
 GROUP = 128          # activation group / weight block edge
 NEAR_TIE = 1e-6      # near-tie flag threshold on p_(K) - p_(K+1)
+# Experts are independent, so the per-expert work runs on a thread pool
+# (numpy releases the GIL in the table lookups and the matmuls).
+WORKERS = max(1, min(32, os.cpu_count() or 1))
+
+
+def _pool_map(fn, items):
+    items = list(items)
+    if WORKERS == 1 or len(items) < 2:
+        return [fn(i) for i in items]
+    with ThreadPoolExecutor(WORKERS) as ex:
+        return list(ex.map(fn, items))
 
 
 # ---------------------------------------------------------------------------
@@ -94,10 +107,14 @@ def dequant_rows(codes: np.ndarray, scales: np.ndarray, C: int = None) -> np.nda
 
 
 def dequant_block(codes: np.ndarray, scales: np.ndarray, rows: int, cols: int) -> np.ndarray:
-    """Weight matrix codes [rows, >=cols] with one scale per 128x128 block -> f64 [rows, cols]."""
-    v = e4m3.decode(np.asarray(codes)[:rows, :cols])
-    s = np.repeat(np.repeat(np.asarray(scales, np.float64), GROUP, axis=0), GROUP, axis=1)[:rows, :cols]
-    return v * s
+    """Weight matrix codes [rows, >=cols] with one scale per 128x128 block -> f64 [rows, cols].
+    Element (n, k) is decode(codes[n, k]) * scales[n // 128, k // 128]."""
+    rb, cb = -(-rows // GROUP), -(-cols // GROUP)
+    padded = np.zeros((rb * GROUP, cb * GROUP), np.uint8)
+    padded[:rows, :cols] = np.asarray(codes)[:rows, :cols]
+    v = e4m3.decode(padded)
+    v.reshape(rb, GROUP, cb, GROUP).__imul__(np.asarray(scales, np.float64)[:rb, None, :cb, None])
+    return v[:rows, :cols]
 
 
 # ---------------------------------------------------------------------------
@@ -211,16 +228,42 @@ def expert_ffn_rows(xq, xs, offsets, layer, groups=None):
     hs = np.zeros((rows, sh.FB), np.float32)
     y = np.zeros((rows, H), np.float64)
     groups = range(sh.E + 1) if groups is None else groups
-    for g in groups:
+
+    def one(g):
         r0, r1 = int(offsets[g]), int(offsets[g + 1])
         if r1 == r0:
-            continue
+            return None
         a = dequant_rows(xq[r0:r1], xs[r0:r1], H)
         hg = expert_gate_up(a, layer.w_gate[g], layer.s_gate[g], layer.w_up[g], layer.s_up[g], F, H)
         q, s = quantize_rows(hg.astype(np.float32))
-        h[r0:r1], hq[r0:r1], hs[r0:r1] = hg, q, s
-        y[r0:r1] = expert_down(dequant_rows(q, s, F), layer.w_down[g], layer.s_down[g], H, F)
+        yg = expert_down(dequant_rows(q, s, F), layer.w_down[g], layer.s_down[g], H, F)
+        return r0, r1, hg, q, s, yg
+
+    for res in _pool_map(one, groups):
+        if res is not None:
+            r0, r1, hg, q, s, yg = res
+            h[r0:r1], hq[r0:r1], hs[r0:r1], y[r0:r1] = hg, q, s, yg
     return {"h": h, "hq": hq, "hs": hs, "y": y}
+
+
+def expert_down_rows(hq, hs, offsets, layer, groups=None):
+    """Down projection alone over permuted rows (h given as codes + scales)."""
+    sh = layer.shape
+    rows = int(offsets[-1])
+    y = np.zeros((rows, sh.H), np.float64)
+    groups = range(sh.E + 1) if groups is None else groups
+
+    def one(g):
+        r0, r1 = int(offsets[g]), int(offsets[g + 1])
+        if r1 == r0:
+            return None
+        return r0, r1, expert_down(dequant_rows(hq[r0:r1], hs[r0:r1], sh.F), layer.w_down[g], layer.s_down[g],
+                                   sh.H, sh.F)
+
+    for res in _pool_map(one, groups):
+        if res is not None:
+            y[res[0]:res[1]] = res[2]
+    return y
 
 
 def combine(y: np.ndarray, inv: np.ndarray, w: np.ndarray) -> np.ndarray:
@@ -278,13 +321,17 @@ def token_outputs(x_bits: np.ndarray, layer, tokens, idx=None, w=None) -> np.nda
             users.setdefault(int(idx_s[i, k]), []).append((i, float(w_s[i, k])))
     users.setdefault(sh.E, [])
     users[sh.E] = [(i, 1.0) for i in range(n)]
-    for g, lst in users.items():
+    def one(item):
+        g, lst = item
         rows = np.array([i for i, _ in lst])
         wt = np.array([c for _, c in lst])
         hg = expert_gate_up(a[rows], layer.w_gate[g], layer.s_gate[g], layer.w_up[g], layer.s_up[g], sh.F, sh.H)
         q, s = quantize_rows(hg.astype(np.float32))
         yg = expert_down(dequant_rows(q, s, sh.F), layer.w_down[g], layer.s_down[g], sh.H, sh.F)
-        np.add.at(out, rows, wt[:, None] * yg)
+        return rows, wt[:, None] * yg
+
+    for rows, contrib in _pool_map(one, sorted(users.items())):
+        np.add.at(out, rows, contrib)
     return out
 
 
@@ -308,12 +355,16 @@ def layer_forward_bf16(x_bits: np.ndarray, layer, tokens=None, idx=None, w=None)
         for k in range(sh.K):
             users.setdefault(int(idx_s[i, k]), []).append((i, float(w_s[i, k])))
     users[sh.E] = [(i, 1.0) for i in range(len(tokens))]
-    for g, lst in users.items():
+    def one(item):
+        g, lst = item
         rows = np.array([i for i, _ in lst])
         wt = np.array([c for _, c in lst])
         Wg = f64_to_bf16_f64(dequant_block(layer.w_gate[g], layer.s_gate[g], sh.F, sh.H))
         Wu = f64_to_bf16_f64(dequant_block(layer.w_up[g], layer.s_up[g], sh.F, sh.H))
         Wd = f64_to_bf16_f64(dequant_block(layer.w_down[g], layer.s_down[g], sh.H, sh.F))
         hg = silu(a[rows] @ Wg.T) * (a[rows] @ Wu.T)
-        np.add.at(out, rows, wt[:, None] * (hg @ Wd.T))
+        return rows, wt[:, None] * (hg @ Wd.T)
+
+    for rows, contrib in _pool_map(one, sorted(users.items())):
+        np.add.at(out, rows, contrib)
     return out

@@ -1,0 +1,384 @@
+"""Parity of the CUDA path (through the C ABI) with the FP64 oracle.
+
+Each stage is checked with teacher forcing: the oracle gets the GPU's own
+upstream outputs. Routing indices, permutation maps and quantised activation
+bytes must match bit-exactly (tokens whose top-K gap is below 1e-6 are
+excluded from the routing comparison); the layer output must be within
+relative Frobenius 5e-3 and max-abs 2e-2 * rms of the oracle.
+"""
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+import gen  # noqa: E402
+from oracle import moe  # noqa: E402
+
+pytestmark = pytest.mark.gpu
+
+if not torch.cuda.is_available():  # collected on CPU machines, never run there
+    pytest.skip("needs a GPU", allow_module_level=True)
+
+import fp8_expert_ffn_b200 as fx  # noqa: E402
+from fp8_expert_ffn_b200 import torch_utils as tu  # noqa: E402
+import gpu_case as gc  # noqa: E402
+
+RNG = np.random.default_rng(1234)
+
+
+# ----------------------------------------------------------------------------- fixtures
+
+_cases = {}
+
+
+def get_case(name):
+    if name not in _cases:
+        wl, layer, x = gen.workload_inputs(name)
+        dev = _device_layers.get((wl.shape, wl.w_seed, wl.zipf))
+        if dev is None:
+            same_experts = [d for (s, w, z), d in _device_layers.items() if (s, w) == (wl.shape, wl.w_seed)]
+            dev = tu.upload_layer(layer, share_experts=same_experts[0] if same_experts else None)
+            _device_layers[(wl.shape, wl.w_seed, wl.zipf)] = dev
+        _cases[name] = (wl, layer, gc.Case(layer, x, dev))
+    return _cases[name]
+
+
+_device_layers = {}
+
+FULL = ["toy", "decode"]                    # every token / row checked
+SAMPLED = ["prefill", "zipf", "edge", "edge_f1500"]
+ALL = FULL + SAMPLED
+
+
+def token_sample(T, n):
+    if T <= n:
+        return np.arange(T)
+    s = RNG.choice(T, n, replace=False)
+    return np.sort(np.concatenate([s, [0, T - 1]]))
+
+
+# ----------------------------------------------------------------------------- routing
+
+@pytest.mark.parametrize("name", ALL)
+def test_route(name):
+    wl, layer, c = get_case(name)
+    r = moe.route(c.x_bits, layer.router_w, layer.shape.K)
+    keep = ~r.near_tie
+    idx = c.np("idx")
+    assert np.array_equal(idx[keep], r.idx[keep]), \
+        f"{np.sum(np.any(idx[keep] != r.idx[keep], axis=1))} unflagged tokens routed differently"
+    w = c.np("w")
+    assert np.allclose(w[keep], r.w[keep], rtol=2e-5, atol=1e-6)
+    assert np.allclose(w.sum(1), 1.0, atol=2e-6)
+    lg = c.np("logits")
+    assert np.max(np.abs(lg - r.logits)) <= 1e-4 * max(1.0, np.abs(r.logits).max())
+
+
+# ----------------------------------------------------------------------------- permutation
+
+@pytest.mark.parametrize("name", ALL)
+def test_permute(name):
+    wl, layer, c = get_case(name)
+    sh, T = layer.shape, c.T
+    p = moe.permute(c.np("idx"), sh.E)
+    assert np.array_equal(c.np("offsets"), p.offsets)
+    assert np.array_equal(c.np("perm"), p.perm)
+    assert np.array_equal(c.np("inv"), p.inv)
+    tq, ts = moe.quantize_tokens(c.x_bits)
+    perm = p.perm
+    rows = np.arange(c.rows) if name in FULL else np.sort(RNG.choice(c.rows, min(c.rows, 8192), replace=False))
+    xq = c.xq[torch.from_numpy(rows).cuda()].cpu().numpy()
+    assert np.array_equal(xq, tq[perm[rows]]), "quantised activation bytes differ"
+    xs = c.np("xs")[:, rows].T
+    assert np.array_equal(xs.view(np.uint32), ts[perm[rows]].view(np.uint32)), "activation scales differ"
+
+
+# ----------------------------------------------------------------------------- expert FFN
+
+@pytest.mark.parametrize("name", ALL)
+def test_expert_ffn(name):
+    wl, layer, c = get_case(name)
+    sh, T = layer.shape, c.T
+    toks = np.arange(T) if name in FULL else token_sample(T, 40)
+    rows = np.unique(gc.rows_of_tokens(c.np("inv"), T, sh.K, toks))
+    off = c.np("offsets")
+    xq = c.xq[torch.from_numpy(rows).cuda()].cpu().numpy()
+    xs = c.np("xs")[:, rows].T.copy()
+    ref = gc.oracle_ffn_on_rows(layer, np.arange(len(rows)), xq, xs,
+                                np.searchsorted(rows, off).astype(np.int64))
+    # h bytes: not gated bit-exactly (FP32 vs FP64 accumulation), but nearly all
+    # equal and the rest one E4M3 step away
+    hq = c.hq[torch.from_numpy(rows).cuda()].cpu().numpy()[:, :sh.F]
+    match = np.mean(hq == ref["hq"])
+    assert match >= 0.995, f"h code match {match:.5f}"
+    assert gc.e4m3_step_diff(hq, ref["hq"]).max() <= 1
+    # y against the oracle fed with the GPU's h (teacher forcing of the down GEMM)
+    hs = c.hs.cpu().numpy()[:, rows].T.copy()
+    E1 = sh.E + 1
+    groups = np.searchsorted(off, rows, side="right") - 1
+    sub_off = np.zeros(E1 + 1, np.int64)
+    sub_off[1:] = np.cumsum(np.bincount(groups, minlength=E1)[:E1])
+    y_tf = moe.expert_down_rows(hq, hs, sub_off, layer, groups=np.unique(groups))
+    y = tu.bf16_bits(c.y[torch.from_numpy(rows).cuda()])
+    yg = moe.bf16_to_f64(y)
+    rms = np.sqrt(np.mean(y_tf ** 2))
+    assert np.all(np.abs(yg - y_tf) <= 2.0 ** -8 * np.abs(y_tf) + 1e-4 * rms), "y differs beyond bf16 rounding"
+    # and against the oracle's own h
+    gc.assert_output_close(yg, ref["y"], f"{name}: y")
+
+
+# ----------------------------------------------------------------------------- combine and layer
+
+@pytest.mark.parametrize("name", ALL)
+def test_combine(name):
+    wl, layer, c = get_case(name)
+    T = c.T
+    toks = np.arange(T) if name in FULL else token_sample(T, 2048)
+    y = moe.bf16_to_f64(tu.bf16_bits(c.y))
+    ref = moe.combine(y, c.np("inv"), c.np("w").astype(np.float64))[toks]
+    out = moe.bf16_to_f64(c.np("out"))[toks]
+    rms = np.sqrt(np.mean(ref ** 2))
+    assert np.all(np.abs(out - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-5 * rms)
+
+
+@pytest.mark.parametrize("name", ALL)
+def test_layer_end_to_end(name):
+    wl, layer, c = get_case(name)
+    T = c.T
+    toks = np.arange(T) if name in FULL else token_sample(T, 48)
+    r = moe.route(c.x_bits[toks], layer.router_w, layer.shape.K)
+    keep = toks[~r.near_tie]
+    ref = moe.token_outputs(c.x_bits, layer, keep)
+    out = moe.bf16_to_f64(c.np("out"))[keep]
+    gc.assert_output_close(out, ref, f"{name}: layer output")
+    # the fused entry point gives the same bytes as the four stages
+    ws = tu.workspace(c.dev, T)
+    o2 = torch.empty_like(c.out)
+    fx.moe_layer_forward(c.dev, c.x, T, layer.shape.H, o2, layer.shape.H, ws, ws.numel())
+    assert torch.equal(o2.view(torch.int16), c.out.view(torch.int16))
+
+
+def test_bf16_checkpoint_cross_check():
+    """FP8 path vs the oracle's BF16-weight path (no activation quantisation)
+    on the F=1500 variant: catches a wrong dequantisation (scale index or
+    partial block) that both FP8 paths could share."""
+    wl, layer, c = get_case("edge_f1500")
+    toks = token_sample(c.T, 24)
+    r = moe.route(c.x_bits[toks], layer.router_w, layer.shape.K)
+    keep = toks[~r.near_tie]
+    ref = moe.layer_forward_bf16(c.x_bits, layer, tokens=keep)
+    out = moe.bf16_to_f64(c.np("out"))[keep]
+    rel = np.linalg.norm(out - ref) / np.linalg.norm(ref)
+    assert rel < 8e-2, rel
+
+
+# ----------------------------------------------------------------------------- GEMM promotion
+
+def _integer_layer():
+    """Toy-shaped layer whose codes decode to integers in [-4, 4] with every
+    scale 1: all products and sums are exact in FP32."""
+    sh = gen.TOY
+    rng = np.random.default_rng(7)
+    vals = np.array([0x00, 0x38, 0x40, 0x44, 0x48, 0xB8, 0xC0, 0xC4, 0xC8], np.uint8)
+    pick = lambda shape: vals[rng.integers(0, 9, shape)]
+    E1 = sh.E + 1
+    return gen.Layer(sh, gen.make_router(sh, 0), pick((E1, sh.F, sh.H)), np.ones((E1, sh.FB, sh.HB), np.float32),
+                     pick((E1, sh.F, sh.H)), np.ones((E1, sh.FB, sh.HB), np.float32),
+                     pick((E1, sh.H, sh.ld_f)), np.ones((E1, sh.HB, sh.FB), np.float32)), vals
+
+
+def _group_offsets(sh, T, rng):
+    rows = T * (sh.K + 1)
+    sizes = np.zeros(sh.E + 1, np.int64)
+    sizes[3] = 150          # two row tiles
+    sizes[0] = 0            # empty groups
+    rest = rows - sizes.sum()
+    cuts = np.sort(rng.choice(rest + 1, sh.E - 2, replace=True))
+    parts = np.diff(np.concatenate([[0], cuts, [rest]]))
+    sizes[[g for g in range(sh.E + 1) if g not in (0, 3)]] = parts
+    off = np.zeros(sh.E + 2, np.int64)
+    off[1:] = np.cumsum(sizes)
+    return off.astype(np.int32)
+
+
+@pytest.mark.parametrize("which", [0, 1])
+def test_grouped_gemm_exact_integers(which):
+    layer, vals = _integer_layer()
+    sh = layer.shape
+    dev = tu.upload_layer(layer)
+    rng = np.random.default_rng(3 + which)
+    T = 60
+    rows = T * (sh.K + 1)
+    off = _group_offsets(sh, T, rng)
+    Kdim = sh.H if which == 0 else sh.FB * 128
+    a = vals[rng.integers(0, 9, (rows, Kdim))]
+    nkb = Kdim // 128
+    a_s = np.ones((nkb, rows), np.float32)
+    ncols = 2 * sh.FB * 128 if which == 0 else sh.H
+    out = torch.full((rows, ncols), float("nan"), device="cuda")
+    ws = tu.workspace(dev, T)
+    fx.moe_test_grouped_gemm_f32(dev, which, tu.to_device(a), tu.to_device(a_s), tu.to_device(off), T, out, ws,
+                                 ws.numel())
+    got = out.cpu().numpy().astype(np.float64)
+    ints = moe.e4m3.decode(np.arange(256, dtype=np.uint8))
+    A = ints[a].astype(np.int64)
+    for g in range(sh.E + 1):
+        r0, r1 = off[g], off[g + 1]
+        if r0 == r1:
+            continue
+        if which == 0:
+            Wg = ints[layer.w_gate[g]].astype(np.int64)
+            Wu = ints[layer.w_up[g]].astype(np.int64)
+            G, U = A[r0:r1] @ Wg.T, A[r0:r1] @ Wu.T
+            for cb in range(sh.FB):
+                assert np.array_equal(got[r0:r1, cb * 256:cb * 256 + 128], G[:, cb * 128:(cb + 1) * 128])
+                assert np.array_equal(got[r0:r1, cb * 256 + 128:cb * 256 + 256], U[:, cb * 128:(cb + 1) * 128])
+        else:
+            Wd = ints[layer.w_down[g][:, :sh.F]].astype(np.int64)
+            assert np.array_equal(got[r0:r1], A[r0:r1, :sh.F] @ Wd.T)
+
+
+@pytest.mark.parametrize("which", [0, 1])
+def test_grouped_gemm_promotion_random_scales(which):
+    """Non-uniform scales: a transposed or shifted scale index would show."""
+    wl, layer0, _ = gen.workload_inputs("toy")
+    sh = layer0.shape
+    rng = np.random.default_rng(11 + which)
+    layer = gen.Layer(sh, layer0.router_w, layer0.w_gate, layer0.s_gate * rng.uniform(0.25, 4, layer0.s_gate.shape)
+                      .astype(np.float32), layer0.w_up, layer0.s_up, layer0.w_down,
+                      layer0.s_down * rng.uniform(0.25, 4, layer0.s_down.shape).astype(np.float32))
+    dev = tu.upload_layer(layer)
+    T = 60
+    rows = T * (sh.K + 1)
+    off = _group_offsets(sh, T, rng)
+    Kdim = sh.H if which == 0 else sh.FB * 128
+    a = rng.integers(0, 256, (rows, Kdim)).astype(np.uint8)
+    a[(a & 0x7F) == 0x7F] = 0x30     # no NaN codes
+    nkb = Kdim // 128
+    a_s = rng.uniform(0.001, 0.1, (nkb, rows)).astype(np.float32)
+    ncols = 2 * sh.FB * 128 if which == 0 else sh.H
+    out = torch.zeros((rows, ncols), device="cuda")
+    ws = tu.workspace(dev, T)
+    fx.moe_test_grouped_gemm_f32(dev, which, tu.to_device(a), tu.to_device(a_s), tu.to_device(off), T, out, ws,
+                                 ws.numel())
+    got = out.cpu().numpy().astype(np.float64)
+    A = moe.dequant_rows(a, a_s.T.copy())
+    for g in range(sh.E + 1):
+        r0, r1 = off[g], off[g + 1]
+        if r0 == r1:
+            continue
+        if which == 0:
+            G = A[r0:r1] @ moe.dequant_block(layer.w_gate[g], layer.s_gate[g], sh.F, sh.H).T
+            U = A[r0:r1] @ moe.dequant_block(layer.w_up[g], layer.s_up[g], sh.F, sh.H).T
+            ref = np.concatenate([np.concatenate([G[:, cb * 128:(cb + 1) * 128], U[:, cb * 128:(cb + 1) * 128]], 1)
+                                  for cb in range(sh.FB)], 1)
+        else:
+            ref = A[r0:r1, :sh.F] @ moe.dequant_block(layer.w_down[g], layer.s_down[g], sh.H, sh.F).T
+        err = np.abs(got[r0:r1] - ref)
+        assert err.max() <= 1e-5 * np.abs(ref).max() + 1e-30, (g, err.max(), np.abs(ref).max())
+
+
+# ----------------------------------------------------------------------------- special inputs
+
+def test_zero_input_exact_zero_output():
+    wl, layer, _ = gen.workload_inputs("toy")
+    x = np.zeros((17, layer.shape.H), np.uint16)
+    c = gc.Case(layer, x)
+    assert np.array_equal(c.np("idx"), np.tile(np.arange(layer.shape.K), (17, 1)))
+    assert np.all(c.np("w") == np.float32(1.0 / layer.shape.K))
+    assert not c.np("out").any()                  # +0 everywhere
+
+
+def test_one_hot_router():
+    wl, layer0, x = gen.workload_inputs("toy")
+    sh = layer0.shape
+    estar = 11
+    router = np.zeros((sh.E, sh.H), np.float32)
+    router[estar, 0] = 200.0
+    layer = gen.Layer(sh, router, layer0.w_gate, layer0.s_gate, layer0.w_up, layer0.s_up, layer0.w_down,
+                      layer0.s_down)
+    xs = x.copy()
+    xs[:, 0] = gen.f32_to_bf16_bits(np.float32([1.0]))[0]
+    c = gc.Case(layer, xs)
+    assert np.array_equal(c.np("idx"), np.tile([0, 1, 2, estar], (xs.shape[0], 1)))
+    assert np.all(c.np("w") == np.float32([0, 0, 0, 1]))
+    ref = moe.layer_forward(xs, layer)["out"]
+    gc.assert_output_close(moe.bf16_to_f64(c.np("out")), ref, "one-hot router")
+    c2 = gc.Case(layer, xs, c.dev)
+    assert np.array_equal(c.np("out"), c2.np("out"))
+
+
+def test_batch_invariance_ragged_tail():
+    """The first 4096 tokens of the T=4099 run equal a T=4096 run bit for bit."""
+    wl, layer, c = get_case("edge")
+    c2 = gc.Case(layer, c.x_bits[:4096], c.dev)
+    assert np.array_equal(c.np("out")[:4096], c2.np("out"))
+
+
+def test_partial_blocks_equal_zero_padded_layer():
+    """FFN 1500 (partial 128x128 blocks) equals the same layer zero-padded to 1536."""
+    wl, layer, c = get_case("edge_f1500")
+    sh = layer.shape
+    sp = gen.LayerShape(H=sh.H, E=sh.E, K=sh.K, F=1536, ld_f=1536)
+    pad = np.zeros((sh.E + 1, 36, sh.H), np.uint8)
+    lp = gen.Layer(sp, layer.router_w, np.concatenate([layer.w_gate, pad], 1), layer.s_gate,
+                   np.concatenate([layer.w_up, pad], 1), layer.s_up, layer.w_down, layer.s_down)
+    assert not lp.w_down[:, :, 1500:].any()
+    x = c.x_bits[:512]
+    a = gc.Case(layer, x, c.dev)
+    b = gc.Case(lp, x)
+    assert np.array_equal(a.np("out"), b.np("out"))
+    del b
+
+
+# ----------------------------------------------------------------------------- errors
+
+def test_bad_expert_ids_set_device_status():
+    wl, layer, c = get_case("toy")
+    sh, T = layer.shape, 8
+    idx = torch.tensor(np.tile(np.arange(sh.K), (T, 1)), dtype=torch.int32, device="cuda")
+    idx[2, 1] = sh.E            # out of range
+    idx[5, 3] = idx[5, 0]       # repeated within a token
+    rows = T * (sh.K + 1)
+    off = torch.empty(sh.E + 2, dtype=torch.int32, device="cuda")
+    perm = torch.full((rows,), -7, dtype=torch.int32, device="cuda")
+    inv = torch.empty((T, sh.K), dtype=torch.int32, device="cuda")
+    xq = torch.empty((rows, sh.H), dtype=torch.uint8, device="cuda")
+    xs = torch.empty((sh.HB, rows), dtype=torch.float32, device="cuda")
+    ws = tu.workspace(c.dev, T)
+    fx.moe_permute(c.dev, c.x[:T], T, sh.H, idx, off, perm, inv, xq, xs, ws, ws.numel())
+    code, bits = fx.moe_get_device_status(c.dev)
+    assert code == fx.MOE_ERR_DEVICE and bits & 1 and bits & 2
+    assert inv[2, 1].item() == -1 and inv[5, 3].item() == -1
+    code, bits = fx.moe_get_device_status(c.dev)   # cleared by the read
+    assert code == fx.MOE_OK and bits == 0
+
+
+def test_host_validation():
+    wl, layer, c = get_case("toy")
+    sh = layer.shape
+    T = 4
+    ws = tu.workspace(c.dev, T)
+    out = torch.empty((T, sh.H), dtype=torch.bfloat16, device="cuda")
+    xmis = torch.empty(T * sh.H + 8, dtype=torch.bfloat16, device="cuda")[1:1 + T * sh.H]
+    with pytest.raises(fx.MoeError) as e:
+        fx.moe_layer_forward(c.dev, xmis, T, sh.H, out, sh.H, ws, ws.numel())
+    assert e.value.code == fx.MOE_ERR_MISALIGNED
+    with pytest.raises(fx.MoeError) as e:
+        fx.moe_layer_forward(c.dev, c.x, T, sh.H, out, sh.H, ws, ws.numel() - 256)
+    assert e.value.code == fx.MOE_ERR_WORKSPACE
+    with pytest.raises(fx.MoeError) as e:
+        fx.moe_layer_forward(c.dev, c.x, T, sh.H - 8, out, sh.H, ws, ws.numel())
+    assert e.value.code == fx.MOE_ERR_INVALID_ARG
+    fx.moe_layer_forward(c.dev, c.x, 0, sh.H, out, sh.H, ws, ws.numel())   # T = 0: no-op
+
+
+def test_forward_is_deterministic():
+    wl, layer, c = get_case("prefill")
+    ws = tu.workspace(c.dev, c.T)
+    outs = []
+    for _ in range(2):
+        o = torch.empty_like(c.out)
+        fx.moe_layer_forward(c.dev, c.x, c.T, layer.shape.H, o, layer.shape.H, ws, ws.numel())
+        outs.append(o)
+    assert torch.equal(outs[0].view(torch.int16), outs[1].view(torch.int16))
