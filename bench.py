@@ -1,0 +1,468 @@
+"""Benchmark of the FP8 MoE-layer forward (dots3-note preview shape) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload decode|prefill|zipf|edge] [--no-secondary]
+
+One step = one whole forward of the layer (route, permute + quantise, gate/up
+GEMM + SwiGLU + quantise, down GEMM, combine) over one batch of T tokens
+whose inputs already sit in HBM. With N > 1 (torchrun, one rank per GPU) every
+rank runs an independent replica of the layer on its own batch: the layer has
+no exchange step on one node at this scale, so the job is weak-scaled and the
+value is all ranks' tokens over the slowest rank's device time.
+
+Prints one JSON line (rank 0).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer tokens/s at T=64 and T=16384; % of HBM / dense-FP8 tensor roofline"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+FP8_OVER_BF16 = 2.0          # nominal dense FP8 / BF16 tensor throughput ratio on B200
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--warmup", type=int, default=10)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default="decode", choices=["decode", "prefill", "zipf", "edge", "decode_e64"])
+    p.add_argument("--no-secondary", action="store_true", help="skip the T=16384 Zipf measurement")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+def peaks():
+    if os.path.exists(PEAKS_FILE):
+        d = json.load(open(PEAKS_FILE))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": FALLBACK_HBM_GBS, "bf16_tflops": FALLBACK_BF16_TFLOPS,
+            "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ----------------------------------------------------------------------------- distributed plumbing
+
+def dist_setup(n):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if n > 1 and world != n:
+        raise SystemExit(f"--gpus {n} needs torchrun with {n} ranks (WORLD_SIZE={world})")
+    return world, rank, local
+
+
+class Dist:
+    def __init__(self, world, rank, local, backend="nccl"):
+        import torch
+        import torch.distributed as dist
+        self.world, self.rank, self.local = world, rank, local
+        self.dist = dist if world > 1 else None
+        if self.dist:
+            from datetime import timedelta
+            dist.init_process_group(backend, timeout=timedelta(seconds=600))
+
+    def barrier(self):
+        if self.dist:
+            self.dist.barrier()
+
+    def max(self, v: float) -> float:
+        if not self.dist:
+            return v
+        import torch
+        t = torch.tensor([v], dtype=torch.float64, device="cuda")
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def sum(self, v: float) -> float:
+        if not self.dist:
+            return v
+        import torch
+        t = torch.tensor([v], dtype=torch.float64, device="cuda")
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.SUM)
+        return float(t.item())
+
+    def close(self):
+        if self.dist:
+            self.dist.destroy_process_group()
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples of this GPU's clocks and throttle reasons while running."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        import tempfile
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.15)
+        self.proc.terminate()
+        self.proc.wait()
+        rows = []
+        for line in open(self.path):
+            parts = [s.strip() for s in line.split(",")]
+            if len(parts) == 8:
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[0]) for r in rows if r[0].replace(".", "").isdigit()]
+        mx = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[4 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------- workload
+
+def algorithmic_work(layer, T, offsets):
+    """Bytes and FLOPs of one forward, counted from the problem (not from the
+    kernels): weights of the touched experts read once, activations and
+    outputs once; FLOPs of the expert GEMMs only (2 * rows * N * K)."""
+    sh = layer.shape
+    H, F, E, K = sh.H, sh.F, sh.E, sh.K
+    rows = T * (K + 1)
+    counts = np.diff(offsets)
+    touched = int(np.count_nonzero(counts[:E])) + (1 if counts[E] > 0 else 0)
+    gu_w = 2 * F * H + 2 * sh.FB * sh.HB * 4          # gate + up codes and scales of one expert
+    dn_w = H * F + sh.HB * sh.FB * 4                  # down codes and scales
+    gu_bytes = touched * gu_w + rows * (H + 4 * sh.HB) + rows * (sh.FB * 128 + 4 * sh.FB)
+    dn_bytes = touched * dn_w + rows * (sh.FB * 128 + 4 * sh.FB) + rows * H * 2
+    route_bytes = E * H * 4 + T * H * 2 + T * K * 8
+    permute_bytes = T * H * 2 + rows * (H + 4 * sh.HB) + T * K * 8 + rows * 4
+    combine_bytes = rows * H * 2 + T * H * 2 + T * K * 8
+    gu_flops = 2.0 * rows * (2 * F) * H
+    dn_flops = 2.0 * rows * H * F
+    return {"touched_groups": touched, "rows": rows,
+            "bytes": {"route": route_bytes, "permute": permute_bytes, "gate_up": gu_bytes, "down": dn_bytes,
+                      "combine": combine_bytes},
+            "flops": {"gate_up": gu_flops, "down": dn_flops}}
+
+
+def load_layer(name, d, rank):
+    """Host inputs on every rank; with several ranks rank 0 generates the
+    expert weights and broadcasts them over NCCL (same checkpoint everywhere)."""
+    import gen
+    import torch
+    from fp8_expert_ffn_b200 import torch_utils as tu
+    import fp8_expert_ffn_b200 as fx
+    wl = gen.WORKLOADS[name]
+    sh = wl.shape
+    x = gen.make_x(wl.T, sh.H, wl.x_seed + 1000 * rank, wl.outliers, wl.zipf)
+    if d.world == 1 or rank == 0:
+        host = gen.make_layer(sh, wl.w_seed, zipf=wl.zipf)
+    else:
+        host = None
+    if d.world == 1:
+        return wl, host, tu.upload_layer(host), x
+    shapes = {"w_gate": ((sh.E + 1, sh.F, sh.H), torch.uint8), "w_up": ((sh.E + 1, sh.F, sh.H), torch.uint8),
+              "w_down": ((sh.E + 1, sh.H, sh.ld_f), torch.uint8),
+              "s_gate": ((sh.E + 1, sh.FB, sh.HB), torch.float32), "s_up": ((sh.E + 1, sh.FB, sh.HB), torch.float32),
+              "s_down": ((sh.E + 1, sh.HB, sh.FB), torch.float32), "router_w": ((sh.E, sh.H), torch.float32)}
+    tens = {}
+    for k, (shape, dt) in shapes.items():
+        tens[k] = tu.to_device(getattr(host, k)) if rank == 0 else torch.empty(shape, dtype=dt, device="cuda")
+        d.dist.broadcast(tens[k], 0)
+    w = fx.LayerWeights(**tens)
+    dev = fx.MoeLayer(sh.H, sh.E, sh.K, sh.F, w, ld_h=sh.H, ld_f=sh.ld_f)
+    return wl, host, dev, x
+
+
+class Stages:
+    """Buffers and the per-stage calls of one forward (the same kernels that
+    moe_layer_forward launches, with CUDA events between the stages)."""
+    NAMES = ("route", "permute", "gate_up", "down", "combine")
+    KERNELS_PER_STEP = 9      # route 2, permute 4, gate/up 1, down 1, combine 1
+
+    def __init__(self, dev, sh, T, x):
+        import torch
+        import fp8_expert_ffn_b200 as fx
+        from fp8_expert_ffn_b200 import torch_utils as tu
+        self.fx, self.dev, self.sh, self.T, self.x = fx, dev, sh, T, x
+        K, E, H = sh.K, sh.E, sh.H
+        rows = T * (K + 1)
+        c = "cuda"
+        self.ws = tu.workspace(dev, T)
+        self.idx = torch.empty((T, K), dtype=torch.int32, device=c)
+        self.w = torch.empty((T, K), dtype=torch.float32, device=c)
+        self.offsets = torch.empty(E + 2, dtype=torch.int32, device=c)
+        self.perm = torch.empty(rows, dtype=torch.int32, device=c)
+        self.inv = torch.empty((T, K), dtype=torch.int32, device=c)
+        self.xq = torch.empty((rows, H), dtype=torch.uint8, device=c)
+        self.xs = torch.empty((sh.HB, rows), dtype=torch.float32, device=c)
+        self.h = torch.empty((rows, sh.FB * 128), dtype=torch.uint8, device=c)
+        self.hs = torch.empty((sh.FB, rows), dtype=torch.float32, device=c)
+        self.y = torch.empty((rows, H), dtype=torch.bfloat16, device=c)
+        self.out = torch.empty((T, H), dtype=torch.bfloat16, device=c)
+
+    def step(self, ev=None):
+        fx, d, T, H, nb = self.fx, self.dev, self.T, self.sh.H, self.ws.numel()
+        if ev: ev[0].record()
+        fx.moe_route(d, self.x, T, H, self.idx, self.w, None, self.ws, nb)
+        if ev: ev[1].record()
+        fx.moe_permute(d, self.x, T, H, self.idx, self.offsets, self.perm, self.inv, self.xq, self.xs, self.ws, nb)
+        if ev: ev[2].record()
+        fx.moe_gate_up(d, self.xq, self.xs, self.offsets, T, self.h, self.hs)
+        if ev: ev[3].record()
+        fx.moe_down(d, self.h, self.hs, self.offsets, T, self.y)
+        if ev: ev[4].record()
+        fx.moe_combine(d, self.y, self.inv, self.w, T, self.out, H)
+        if ev: ev[5].record()
+
+
+def time_stages(st: Stages, steps: int, warmup: int, d: Dist, sampler=None):
+    import torch
+    for _ in range(warmup):
+        st.step()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(steps)]
+    d.barrier()
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.start()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for i in range(steps):
+        st.step(evs[i])
+    t1.record()
+    torch.cuda.synchronize()
+    clocks = sampler.stop() if sampler else None
+    d.barrier()
+    torch.cuda.synchronize()
+    total_ms = t0.elapsed_time(t1)
+    per = {n: sum(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(steps)) / steps
+           for j, n in enumerate(Stages.NAMES)}
+    code, bits = st.fx.moe_get_device_status(st.dev)
+    if code != 0:
+        raise RuntimeError(f"device status {bits:#x}")
+    return total_ms, per, clocks
+
+
+def time_e2e(dev, sh, x_bits, steps, warmup, d: Dist):
+    """Through moe_layer_forward with host buffers: pinned host x -> device,
+    forward, device -> pinned host out, all inside the timed region."""
+    import torch
+    import fp8_expert_ffn_b200 as fx
+    from fp8_expert_ffn_b200 import torch_utils as tu
+    T, H = x_bits.shape
+    x_host = torch.from_numpy(np.ascontiguousarray(x_bits).view(np.int16)).view(torch.bfloat16).pin_memory()
+    out_host = torch.empty((T, H), dtype=torch.bfloat16).pin_memory()
+    x_dev = torch.empty((T, H), dtype=torch.bfloat16, device="cuda")
+    out_dev = torch.empty((T, H), dtype=torch.bfloat16, device="cuda")
+    ws = tu.workspace(dev, T)
+
+    def one():
+        x_dev.copy_(x_host, non_blocking=True)
+        fx.moe_layer_forward(dev, x_dev, T, H, out_dev, H, ws, ws.numel())
+        out_host.copy_(out_dev, non_blocking=True)
+
+    for _ in range(warmup):
+        one()
+    torch.cuda.synchronize()
+    d.barrier()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        one()
+    b.record()
+    torch.cuda.synchronize()
+    d.barrier()
+    return a.elapsed_time(b), T * H * 2, T * H * 2
+
+
+def cpu_baseline(host_layer, x_bits, budget_s=20.0):
+    """The oracle (FP64 numpy) on a bounded sample of the workload's tokens,
+    timed on this host's cores."""
+    from oracle import moe
+    n, dt = 1, 0.0
+    tokens = np.arange(x_bits.shape[0])
+    while True:
+        t = time.perf_counter()
+        moe.token_outputs(x_bits, host_layer, tokens[:n])
+        dt = time.perf_counter() - t
+        if dt * 2 > budget_s or n * 2 > len(tokens):
+            break
+        n *= 2
+    return {"value": n / dt, "unit": "tokens/s", "cores": moe.WORKERS, "kind": "oracle",
+            "sample": f"{n} of the {len(tokens)} tokens through the whole layer (route, quantise, expert FFNs, "
+                      f"combine; FP64), {dt:.1f} s"}
+
+
+# ----------------------------------------------------------------------------- arms
+
+def run_ours(args):
+    import torch
+    world, rank, local = dist_setup(args.gpus)
+    torch.cuda.set_device(local)
+    d = Dist(world, rank, local)
+    pk = peaks()
+    wl, host, dev, x_bits = load_layer(args.workload, d, rank)
+    from fp8_expert_ffn_b200 import torch_utils as tu
+    sh = wl.shape
+    T = wl.T
+    x = tu.bf16_tensor(x_bits)
+    st = Stages(dev, sh, T, x)
+    visible = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+    sampler = ClockSampler(visible.split(",")[local] if visible else local)
+    total_ms, per, clocks = time_stages(st, args.steps, args.warmup, d, sampler)
+    total_ms = d.max(total_ms)
+    tokens = d.sum(float(T * args.steps))
+    value = tokens / (total_ms / 1e3)
+    off = st.offsets.cpu().numpy()
+    work = algorithmic_work(wl, T, off)
+    # the dominant kernel: decode-sized batches are bound by streaming the
+    # gate/up weights (HBM); large batches by the FP8 tensor pipe
+    kern = max(("gate_up", "down"), key=lambda k: per[k])
+    kern_ms = d.max(per[kern])
+    hbm_bound = work["flops"][kern] / work["bytes"][kern] < (FP8_OVER_BF16 * pk["bf16_tflops"] * 1e12) / (
+        pk["hbm_gbs"] * 1e9)
+    if hbm_bound:
+        ach = work["bytes"][kern] / (kern_ms / 1e3) / 1e9
+        roof = {"bound": "hbm", "kernel": kern, "achieved": round(ach, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": round(ach / pk["hbm_gbs"], 4), "traffic": None,
+                "algorithmic_bytes_per_launch": work["bytes"][kern], "ms_per_launch": round(kern_ms, 5),
+                "peak_source": f"{pk['source']} hbm_gbs"}
+    else:
+        peak = FP8_OVER_BF16 * pk["bf16_tflops"]
+        ach = work["flops"][kern] / (kern_ms / 1e3) / 1e12
+        roof = {"bound": "tensor", "kernel": kern, "achieved": round(ach, 1), "peak": round(peak, 1),
+                "unit": "TFLOP/s", "frac": round(ach / peak, 4), "traffic": None,
+                "algorithmic_flops_per_launch": work["flops"][kern], "ms_per_launch": round(kern_ms, 5),
+                "peak_source": f"{pk['source']} bf16_tflops x {FP8_OVER_BF16} (nominal FP8/BF16 ratio)"}
+    e2e_ms, bi, bo = time_e2e(dev, sh, x_bits, args.steps, args.warmup, d)
+    e2e_ms = d.max(e2e_ms)
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "e4m3 (fp32 accumulate)", "data": "synthetic",
+        "config": {"workload": f"{wl.name}: {wl.note}", "T": T, "hidden": sh.H, "experts": f"{sh.E}+1",
+                   "top_k": sh.K, "ffn": sh.F, "weights": "FP8 E4M3, 128x128 fp32 block scales, seeded synthetic",
+                   "l2": "inputs larger than L2 (each step streams the touched experts' weights, GBs >> 126 MB)",
+                   "parallelism": f"replicas x{world}", "touched_groups": work["touched_groups"]},
+        "stage_ms": {k: round(v, 5) for k, v in per.items()},
+        "roofline": roof,
+        "e2e": {"value": round(tokens / (e2e_ms / 1e3), 1), "unit": "tokens/s", "h2d_bytes_per_step": bi,
+                "d2h_bytes_per_step": bo, "ms_per_step": round(e2e_ms / args.steps, 5)},
+        "gpu_launches": Stages.KERNELS_PER_STEP * args.steps,
+        "clocks": clocks,
+    }
+    if not args.no_secondary and args.workload != "zipf":
+        del st
+        sec = secondary(d, rank, args, pk)
+        if sec:
+            line["secondary"] = sec
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(host, x_bits)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    d.close()
+
+
+def secondary(d, rank, args, pk):
+    """The long-prefill workload (T=16384, Zipf-skewed routing), timed the same way."""
+    import torch
+    from fp8_expert_ffn_b200 import torch_utils as tu
+    wl, host, dev, x_bits = load_layer("zipf", d, rank)
+    st = Stages(dev, wl.shape, wl.T, tu.bf16_tensor(x_bits))
+    steps = max(3, min(args.steps, 20))
+    total_ms, per, _ = time_stages(st, steps, max(3, min(args.warmup, 5)), d)
+    total_ms = d.max(total_ms)
+    off = st.offsets.cpu().numpy()
+    work = algorithmic_work(wl, wl.T, off)
+    flops = work["flops"]["gate_up"] + work["flops"]["down"]
+    gemm_ms = d.max(per["gate_up"] + per["down"])
+    peak = FP8_OVER_BF16 * pk["bf16_tflops"]
+    kern = max(("gate_up", "down"), key=lambda k: per[k])
+    kms = d.max(per[kern])
+    ach = work["flops"][kern] / (kms / 1e3) / 1e12
+    counts = np.diff(off)[:wl.shape.E]
+    return {"workload": f"{wl.name}: {wl.note}", "T": wl.T, "steps": steps,
+            "value": round(d.sum(float(wl.T * steps)) / (total_ms / 1e3), 1), "unit": "tokens/s",
+            "ms_per_step": round(total_ms / steps, 5), "stage_ms": {k: round(v, 5) for k, v in per.items()},
+            "expert_gemm_tflops": round(flops / (gemm_ms / 1e3) / 1e12, 1),
+            "roofline": {"bound": "tensor", "kernel": kern, "achieved": round(ach, 1), "peak": round(peak, 1),
+                         "unit": "TFLOP/s", "frac": round(ach / peak, 4),
+                         "peak_source": f"{pk['source']} bf16_tflops x {FP8_OVER_BF16}"},
+            "load_max_over_mean": round(float(counts.max() / counts.mean()), 2),
+            "empty_experts": int((counts == 0).sum())}
+
+
+def run_reference(args):
+    """The oracle timed on this host's cores as the reference arm (rank 0 only)."""
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    import gen
+    from oracle import moe
+    wl = gen.WORKLOADS[args.workload]
+    host = gen.make_layer(wl.shape, wl.w_seed, zipf=wl.zipf)
+    x_bits = gen.make_x(wl.T, wl.shape.H, wl.x_seed, wl.outliers, wl.zipf)
+    per_step = 1                       # tokens per step: a bounded sample of the batch
+    for i in range(args.warmup):
+        moe.token_outputs(x_bits, host, [i % wl.T])
+    t = time.perf_counter()
+    for i in range(args.steps):
+        moe.token_outputs(x_bits, host, [(args.warmup + i) % wl.T])
+    dt = time.perf_counter() - t
+    value = per_step * args.steps / dt
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": f"{wl.name}: {wl.note}", "T": wl.T, "hidden": wl.shape.H,
+                       "experts": f"{wl.shape.E}+1", "top_k": wl.shape.K, "ffn": wl.shape.F},
+            "cpu_baseline": {"value": round(value, 4), "unit": "tokens/s", "kind": "oracle", "cores": moe.WORKERS,
+                             "sample": f"{per_step} token per step through the whole layer (FP64 oracle)"},
+            "e2e": {"value": round(value, 4), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -19,7 +19,7 @@ MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_MISALIGNED, MOE_ERR_UNSUPPORTED, MOE_ERR_WO
 
 ENTRY_POINTS = ("moe_status_string", "moe_layer_create", "moe_layer_destroy", "moe_workspace_size", "moe_route",
                 "moe_permute", "moe_expert_ffn", "moe_combine", "moe_layer_forward", "moe_get_device_status",
-                "moe_test_grouped_gemm_f32", "moe_test_workspace_h")
+                "moe_gate_up", "moe_down", "moe_test_grouped_gemm_f32")
 
 
 class MoeError(RuntimeError):
@@ -68,8 +68,9 @@ def lib(build_if_missing: bool = True):
     L.moe_combine.argtypes = [P, P, P, P, I, P, I, P]
     L.moe_layer_forward.argtypes = [P, P, I, I, P, I, P, S, P]
     L.moe_get_device_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_uint32)]
-    L.moe_test_grouped_gemm_f32.argtypes = [P, I, P, P, P, I, P, P, S, P]
-    L.moe_test_workspace_h.argtypes = [P, I, ctypes.POINTER(S), ctypes.POINTER(S)]
+    L.moe_gate_up.argtypes = [P, P, P, P, I, P, P, P]
+    L.moe_down.argtypes = [P, P, P, P, I, P, P]
+    L.moe_test_grouped_gemm_f32.argtypes = [P, I, P, P, P, I, P, P]
     for name in ENTRY_POINTS:
         if name not in ("moe_status_string", "moe_workspace_size"):
             getattr(L, name).restype = I
@@ -182,14 +183,16 @@ def moe_get_device_status(layer, stream=None):
     return code, bits.value
 
 
-def moe_test_grouped_gemm_f32(layer, which, a, a_scales, offsets, T, out, ws, ws_bytes, stream=None):
+def moe_gate_up(layer, xq, xs, offsets, T, h, hs, stream=None):
+    _check("moe_gate_up", lib().moe_gate_up(layer.handle, _ptr(xq), _ptr(xs), _ptr(offsets), T, _ptr(h), _ptr(hs),
+                                            _stream(stream)))
+
+
+def moe_down(layer, h, hs, offsets, T, y, stream=None):
+    _check("moe_down", lib().moe_down(layer.handle, _ptr(h), _ptr(hs), _ptr(offsets), T, _ptr(y), _stream(stream)))
+
+
+def moe_test_grouped_gemm_f32(layer, which, a, a_scales, offsets, T, out, stream=None):
     _check("moe_test_grouped_gemm_f32",
            lib().moe_test_grouped_gemm_f32(layer.handle, which, _ptr(a), _ptr(a_scales), _ptr(offsets), T,
-                                           _ptr(out), _ptr(ws), ws_bytes, _stream(stream)))
-
-
-def moe_test_workspace_h(layer, T):
-    """(h byte offset, hs byte offset) inside a workspace for T tokens."""
-    h, hs = ctypes.c_size_t(0), ctypes.c_size_t(0)
-    _check("moe_test_workspace_h", lib().moe_test_workspace_h(layer.handle, T, ctypes.byref(h), ctypes.byref(hs)))
-    return h.value, hs.value
+                                           _ptr(out), _stream(stream)))

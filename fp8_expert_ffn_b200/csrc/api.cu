@@ -68,7 +68,6 @@ Scratch carve(const moe_layer_s* L, int T, void* base) {
   s.bitmap = static_cast<uint32_t*>(take(sizeof(uint32_t) * E * W));
   s.wprefix = static_cast<uint32_t*>(take(sizeof(uint32_t) * E * W));
   s.counts = static_cast<int32_t*>(take(sizeof(int32_t) * E));
-  s.plan = static_cast<int32_t*>(take(sizeof(int32_t) * kPlanInts(E)));
   s.h = static_cast<uint8_t*>(take(rows * L->ld_hh));
   s.hs = static_cast<float*>(take(sizeof(float) * L->FB * rows));
   s.idx = static_cast<int32_t*>(take(sizeof(int32_t) * size_t(T) * K));
@@ -220,6 +219,24 @@ moe_status moe_permute(moe_layer_t L, const uint16_t* x, int T, int ldx, const i
       launch_permute(L, x, T, ldx, idx, offsets, perm, inv, xq, xs, sc, static_cast<cudaStream_t>(stream)));
 }
 
+moe_status moe_gate_up(moe_layer_t L, const uint8_t* xq, const float* xs, const int32_t* offsets, int T,
+                       uint8_t* h, float* hs, void* stream) {
+  if (!L || T < 0 || T > kMaxT) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!xq || !xs || !offsets || !h || !hs) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(xq) || !aligned16(h)) return MOE_ERR_MISALIGNED;
+  return from_cuda(launch_gate_up(L, xq, xs, offsets, T, h, hs, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_down(moe_layer_t L, const uint8_t* h, const float* hs, const int32_t* offsets, int T, uint16_t* y,
+                    void* stream) {
+  if (!L || T < 0 || T > kMaxT) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!h || !hs || !offsets || !y) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(h) || !aligned16(y)) return MOE_ERR_MISALIGNED;
+  return from_cuda(launch_down(L, h, hs, offsets, T, y, static_cast<cudaStream_t>(stream)));
+}
+
 moe_status moe_expert_ffn(moe_layer_t L, const uint8_t* xq, const float* xs, const int32_t* offsets, int T,
                           uint16_t* y, void* ws, size_t ws_bytes, void* stream) {
   if (!L || T < 0 || T > kMaxT) return MOE_ERR_INVALID_ARG;
@@ -229,7 +246,10 @@ moe_status moe_expert_ffn(moe_layer_t L, const uint8_t* xq, const float* xs, con
   moe_status s;
   if ((s = check_ws(L, T, ws, ws_bytes)) != MOE_OK) return s;
   Scratch sc = carve(L, T, ws);
-  return from_cuda(launch_expert_ffn(L, xq, xs, offsets, T, y, sc, static_cast<cudaStream_t>(stream)));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_gate_up(L, xq, xs, offsets, T, sc.h, sc.hs, st);
+  if (e == cudaSuccess) e = launch_down(L, sc.h, sc.hs, offsets, T, y, st);
+  return from_cuda(e);
 }
 
 moe_status moe_combine(moe_layer_t L, const uint16_t* y, const int32_t* inv, const float* w, int T, uint16_t* out,
@@ -254,7 +274,8 @@ moe_status moe_layer_forward(moe_layer_t L, const uint16_t* x, int T, int ldx, u
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e = launch_route(L, x, T, ldx, sc.idx, sc.topw, nullptr, sc.route_partial, st);
   if (e == cudaSuccess) e = launch_permute(L, x, T, ldx, sc.idx, sc.offsets, sc.perm, sc.inv, sc.xq, sc.xs, sc, st);
-  if (e == cudaSuccess) e = launch_expert_ffn(L, sc.xq, sc.xs, sc.offsets, T, sc.y, sc, st);
+  if (e == cudaSuccess) e = launch_gate_up(L, sc.xq, sc.xs, sc.offsets, T, sc.h, sc.hs, st);
+  if (e == cudaSuccess) e = launch_down(L, sc.h, sc.hs, sc.offsets, T, sc.y, st);
   if (e == cudaSuccess) e = launch_combine(L, sc.y, sc.inv, sc.topw, T, out, ldo, st);
   return from_cuda(e);
 }
@@ -271,24 +292,12 @@ moe_status moe_get_device_status(moe_layer_t L, void* stream, uint32_t* detail) 
 }
 
 moe_status moe_test_grouped_gemm_f32(moe_layer_t L, int which, const uint8_t* a, const float* as,
-                                     const int32_t* offsets, int T, float* out, void* ws, size_t ws_bytes,
-                                     void* stream) {
+                                     const int32_t* offsets, int T, float* out, void* stream) {
   if (!L || T < 0 || T > kMaxT || (which != 0 && which != 1)) return MOE_ERR_INVALID_ARG;
   if (T == 0) return MOE_OK;
   if (!a || !as || !offsets || !out) return MOE_ERR_INVALID_ARG;
   if (!aligned16(a)) return MOE_ERR_MISALIGNED;
-  moe_status s;
-  if ((s = check_ws(L, T, ws, ws_bytes)) != MOE_OK) return s;
-  Scratch sc = carve(L, T, ws);
-  return from_cuda(launch_test_gemm_f32(L, which, a, as, offsets, T, out, sc, static_cast<cudaStream_t>(stream)));
-}
-
-moe_status moe_test_workspace_h(moe_layer_t L, int T, size_t* h_offset, size_t* hs_offset) {
-  if (!L || T < 1 || T > kMaxT || !h_offset || !hs_offset) return MOE_ERR_INVALID_ARG;
-  Scratch s = carve(L, T, nullptr);
-  *h_offset = reinterpret_cast<size_t>(s.h);
-  *hs_offset = reinterpret_cast<size_t>(s.hs);
-  return MOE_OK;
+  return from_cuda(launch_test_gemm_f32(L, which, a, as, offsets, T, out, static_cast<cudaStream_t>(stream)));
 }
 
 }  // extern "C"

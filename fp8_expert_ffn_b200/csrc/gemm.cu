@@ -64,7 +64,6 @@ enum { EPI_FUSED = 0, EPI_F32 = 1 };
 
 struct GemmArgs {
   const int32_t* offsets;  // [ngroups + 1] row offsets of the groups
-  const int32_t* prefix;   // [ngroups + 1] exclusive tile prefix; [ngroups] = total
   int ngroups;
   int ntn;                 // n tiles per group
   int nkb;                 // K blocks
@@ -138,9 +137,26 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  for (int i = threadIdx.x; i <= p.ngroups; i += blockDim.x) {
-    s_off[i] = p.offsets[i];
-    s_prefix[i] = p.prefix[i];
+  // Group offsets and the exclusive prefix of the tile counts (every CTA
+  // derives the same tile list from the device-side offsets).
+  {
+    __shared__ int s_wsum[THREADS / 32];
+    const int g = threadIdx.x;
+    int v = 0;
+    if (g <= p.ngroups) s_off[g] = p.offsets[g];
+    if (g < p.ngroups) v = ((p.offsets[g + 1] - p.offsets[g] + BM - 1) / BM) * p.ntn;
+    int incl = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int o = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+      if ((threadIdx.x & 31) >= off) incl += o;
+    }
+    if ((threadIdx.x & 31) == 31) s_wsum[threadIdx.x >> 5] = incl;
+    __syncthreads();
+    int base = 0;
+    for (int j = 0; j < (threadIdx.x >> 5); ++j) base += s_wsum[j];
+    if (g < p.ngroups) s_prefix[g] = base + incl - v;
+    if (g == p.ngroups - 1) s_prefix[p.ngroups] = base + incl;
   }
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -368,39 +384,6 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
 }
 
-// Exclusive tile prefix of both GEMMs from the group offsets:
-// plan[0 .. ng]          gate/up (ntn_gu n tiles per group)
-// plan[ng+1 .. 2ng+1]    down    (ntn_dn n tiles per group)
-__global__ void __launch_bounds__(512) tile_plan_kernel(const int32_t* __restrict__ offsets, int ng, int ntn_gu,
-                                                        int ntn_dn, int32_t* __restrict__ plan) {
-  __shared__ int sums[2][16];
-  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-  int mt = 0;
-  if (tid < ng) mt = (offsets[tid + 1] - offsets[tid] + BM - 1) / BM;
-  int v[2] = {mt * ntn_gu, mt * ntn_dn};
-  int incl[2] = {v[0], v[1]};
-#pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-#pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      const int o = __shfl_up_sync(0xFFFFFFFFu, incl[j], off);
-      if (lane >= off) incl[j] += o;
-    }
-  }
-  if (lane == 31) { sums[0][wid] = incl[0]; sums[1][wid] = incl[1]; }
-  __syncthreads();
-  int base[2] = {0, 0};
-  for (int j = 0; j < wid; ++j) { base[0] += sums[0][j]; base[1] += sums[1][j]; }
-  if (tid < ng) {
-    plan[tid] = base[0] + incl[0] - v[0];
-    plan[ng + 1 + tid] = base[1] + incl[1] - v[1];
-  }
-  if (tid == ng - 1) {
-    plan[ng] = base[0] + incl[0];
-    plan[ng + 1 + ng] = base[1] + incl[1];
-  }
-}
-
 template <int MODE, int EPI>
 cudaError_t launch_gemm(const moe_layer_s* L, const CUtensorMap& tmA, const CUtensorMap& tmB0,
                         const CUtensorMap& tmB1, const GemmArgs& a, cudaStream_t st) {
@@ -421,11 +404,9 @@ cudaError_t launch_gemm(const moe_layer_s* L, const CUtensorMap& tmA, const CUte
 
 }  // namespace
 
-static GemmArgs gateup_args(const moe_layer_s* L, const int32_t* offsets, const int32_t* plan, int rows,
-                            const float* xs) {
+static GemmArgs gateup_args(const moe_layer_s* L, const int32_t* offsets, int rows, const float* xs) {
   GemmArgs a = {};
   a.offsets = offsets;
-  a.prefix = plan;
   a.ngroups = L->E + 1;
   a.ntn = L->FB;
   a.nkb = L->HB;
@@ -440,11 +421,9 @@ static GemmArgs gateup_args(const moe_layer_s* L, const int32_t* offsets, const 
   return a;
 }
 
-static GemmArgs down_args(const moe_layer_s* L, const int32_t* offsets, const int32_t* plan, int rows,
-                          const float* hs) {
+static GemmArgs down_args(const moe_layer_s* L, const int32_t* offsets, int rows, const float* hs) {
   GemmArgs a = {};
   a.offsets = offsets;
-  a.prefix = plan + (L->E + 2);
   a.ngroups = L->E + 1;
   a.ntn = (L->HB + 1) / 2;
   a.nkb = L->FB;
@@ -459,46 +438,42 @@ static GemmArgs down_args(const moe_layer_s* L, const int32_t* offsets, const in
   return a;
 }
 
-static cudaError_t launch_plan(const moe_layer_s* L, const int32_t* offsets, int32_t* plan, cudaStream_t st) {
-  tile_plan_kernel<<<1, 512, 0, st>>>(offsets, L->E + 1, L->FB, (L->HB + 1) / 2, plan);
-  return cudaGetLastError();
+cudaError_t launch_gate_up(const moe_layer_s* L, const uint8_t* xq, const float* xs, const int32_t* offsets, int T,
+                           uint8_t* h, float* hs, cudaStream_t st) {
+  const int rows = T * (L->K + 1);
+  CUtensorMap tmX;
+  if (!encode_tmap_u8(&tmX, xq, L->H, rows, 1, L->H, 0)) return cudaErrorInvalidValue;
+  GemmArgs a = gateup_args(L, offsets, rows, xs);
+  a.h = h;
+  a.hs = hs;
+  a.ld_h = L->ld_hh;
+  return launch_gemm<MODE_GATEUP, EPI_FUSED>(L, tmX, L->tm_gate, L->tm_up, a, st);
 }
 
-cudaError_t launch_expert_ffn(const moe_layer_s* L, const uint8_t* xq, const float* xs, const int32_t* offsets,
-                              int T, uint16_t* y, const Scratch& s, cudaStream_t st) {
+cudaError_t launch_down(const moe_layer_s* L, const uint8_t* h, const float* hs, const int32_t* offsets, int T,
+                        uint16_t* y, cudaStream_t st) {
   const int rows = T * (L->K + 1);
-  cudaError_t e = launch_plan(L, offsets, s.plan, st);
-  if (e != cudaSuccess) return e;
-  CUtensorMap tmX, tmH;
-  if (!encode_tmap_u8(&tmX, xq, L->H, rows, 1, L->H, 0)) return cudaErrorInvalidValue;
-  if (!encode_tmap_u8(&tmH, s.h, L->F, rows, 1, L->ld_hh, 0)) return cudaErrorInvalidValue;
-  GemmArgs gu = gateup_args(L, offsets, s.plan, rows, xs);
-  gu.h = s.h;
-  gu.hs = s.hs;
-  gu.ld_h = L->ld_hh;
-  e = launch_gemm<MODE_GATEUP, EPI_FUSED>(L, tmX, L->tm_gate, L->tm_up, gu, st);
-  if (e != cudaSuccess) return e;
-  GemmArgs dn = down_args(L, offsets, s.plan, rows, s.hs);
-  dn.y = y;
-  dn.ld_y = L->H;
-  return launch_gemm<MODE_DOWN, EPI_FUSED>(L, tmH, L->tm_down, L->tm_down, dn, st);
+  CUtensorMap tmH;
+  if (!encode_tmap_u8(&tmH, h, L->F, rows, 1, L->ld_hh, 0)) return cudaErrorInvalidValue;
+  GemmArgs a = down_args(L, offsets, rows, hs);
+  a.y = y;
+  a.ld_y = L->H;
+  return launch_gemm<MODE_DOWN, EPI_FUSED>(L, tmH, L->tm_down, L->tm_down, a, st);
 }
 
 cudaError_t launch_test_gemm_f32(const moe_layer_s* L, int which, const uint8_t* a_ptr, const float* as,
-                                 const int32_t* offsets, int T, float* out, const Scratch& s, cudaStream_t st) {
+                                 const int32_t* offsets, int T, float* out, cudaStream_t st) {
   const int rows = T * (L->K + 1);
-  cudaError_t e = launch_plan(L, offsets, s.plan, st);
-  if (e != cudaSuccess) return e;
   CUtensorMap tmA;
   if (which == 0) {
     if (!encode_tmap_u8(&tmA, a_ptr, L->H, rows, 1, L->H, 0)) return cudaErrorInvalidValue;
-    GemmArgs a = gateup_args(L, offsets, s.plan, rows, as);
+    GemmArgs a = gateup_args(L, offsets, rows, as);
     a.out = out;
     a.ld_out = 2 * L->FB * 128;
     return launch_gemm<MODE_GATEUP, EPI_F32>(L, tmA, L->tm_gate, L->tm_up, a, st);
   }
   if (!encode_tmap_u8(&tmA, a_ptr, L->F, rows, 1, L->ld_hh, 0)) return cudaErrorInvalidValue;
-  GemmArgs a = down_args(L, offsets, s.plan, rows, as);
+  GemmArgs a = down_args(L, offsets, rows, as);
   a.out = out;
   a.ld_out = L->H;
   return launch_gemm<MODE_DOWN, EPI_F32>(L, tmA, L->tm_down, L->tm_down, a, st);

@@ -35,7 +35,6 @@ struct Scratch {
   uint32_t* wprefix;      // [E][W]
   int32_t* counts;        // [E]
   // expert ffn
-  int32_t* plan;          // tile plans (two GEMMs)
   uint8_t* h;             // [rows][ld_hh]
   float* hs;              // [FB][rows]
   // forward intermediates
@@ -52,17 +51,18 @@ struct Scratch {
 
 int route_splits(const moe_layer_s* L, int T);
 Scratch carve(const moe_layer_s* L, int T, void* base);
-constexpr int kPlanInts(int E) { return 2 * (E + 2) + 8; }
 
 cudaError_t launch_route(const moe_layer_s* L, const uint16_t* x, int T, int ldx, int32_t* idx, float* w,
                          float* logits, float* partial, cudaStream_t st);
 cudaError_t launch_permute(const moe_layer_s* L, const uint16_t* x, int T, int ldx, const int32_t* idx,
                            int32_t* offsets, int32_t* perm, int32_t* inv, uint8_t* xq, float* xs,
                            const Scratch& s, cudaStream_t st);
-cudaError_t launch_expert_ffn(const moe_layer_s* L, const uint8_t* xq, const float* xs, const int32_t* offsets,
-                              int T, uint16_t* y, const Scratch& s, cudaStream_t st);
+cudaError_t launch_gate_up(const moe_layer_s* L, const uint8_t* xq, const float* xs, const int32_t* offsets, int T,
+                           uint8_t* h, float* hs, cudaStream_t st);
+cudaError_t launch_down(const moe_layer_s* L, const uint8_t* h, const float* hs, const int32_t* offsets, int T,
+                        uint16_t* y, cudaStream_t st);
 cudaError_t launch_test_gemm_f32(const moe_layer_s* L, int which, const uint8_t* a, const float* as,
-                                 const int32_t* offsets, int T, float* out, const Scratch& s, cudaStream_t st);
+                                 const int32_t* offsets, int T, float* out, cudaStream_t st);
 cudaError_t launch_combine(const moe_layer_s* L, const uint16_t* y, const int32_t* inv, const float* w, int T,
                            uint16_t* out, int ldo, cudaStream_t st);
 

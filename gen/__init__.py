@@ -195,6 +195,10 @@ WORKLOADS = {
                      note="T=4099 (ragged)"),
     "edge_f1500": Workload("edge_f1500", 4099, DOTS3_F1500, x_seed=4, w_seed=2, outliers=8,
                            note="T=4099 on the FFN=1500 variant (partial 128x128 blocks)"),
+    # a smaller decode-shaped case (64 routed experts, 1.5 GB of weights) for
+    # profiler captures that must stay a few GB on the device
+    "decode_e64": Workload("decode_e64", 16, LayerShape(H=5120, E=64, K=8, F=1536, ld_f=1536), x_seed=5,
+                           w_seed=3, outliers=8, note="T=16, 64+1 experts, hidden 5120, FFN 1536 (profiling case)"),
 }
 
 

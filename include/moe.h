@@ -158,6 +158,20 @@ moe_status moe_permute(moe_layer_t layer, const uint16_t* x, int T, int ldx, con
 moe_status moe_expert_ffn(moe_layer_t layer, const uint8_t* xq, const float* xs, const int32_t* offsets, int T,
                           uint16_t* y, void* ws, size_t ws_bytes, void* stream);
 
+/* The two halves of moe_expert_ffn, for callers that keep h themselves.
+ * moe_gate_up: h = quantise(silu(xq Wg^T) * (xq Wu^T)) per row per 128
+ * channels.
+ *   h   [rows][ceil(F/128)*128] E4M3 bytes (out); channels >= F are zero
+ *   hs  [ceil(F/128)][rows] fp32 (out, group-major)
+ * moe_down: y = h Wd^T (FP32 with block-scale promotion) rounded to bf16.
+ *   y   [rows][H] bf16 (out)
+ * Neither needs a workspace; both read the groups from the device-side
+ * offsets written by moe_permute. */
+moe_status moe_gate_up(moe_layer_t layer, const uint8_t* xq, const float* xs, const int32_t* offsets, int T,
+                       uint8_t* h, float* hs, void* stream);
+moe_status moe_down(moe_layer_t layer, const uint8_t* h, const float* hs, const int32_t* offsets, int T,
+                    uint16_t* y, void* stream);
+
 /* out[t] = bf16_RNE( sum_k topk_w[t,k] * y[inv[t,k]] + y[T*K + t] ), FP32
  * sum in slot order, shared row last.
  *   out [T][ldo] bf16, ldo >= H                                            */
@@ -184,14 +198,7 @@ moe_status moe_get_device_status(moe_layer_t layer, void* stream, uint32_t* deta
  *              ignored), as = [ceil(F/128)][rows]; out [rows][H] fp32
  * offsets gives the groups as in moe_permute; rows = T*(K+1). */
 moe_status moe_test_grouped_gemm_f32(moe_layer_t layer, int which, const uint8_t* a, const float* as,
-                                     const int32_t* offsets, int T, float* out, void* ws, size_t ws_bytes,
-                                     void* stream);
-
-/* Test hook: byte offsets, inside a workspace for T tokens, of the quantised
- * SwiGLU output that moe_expert_ffn leaves there: h [rows][ceil(F/128)*128]
- * E4M3 bytes (channels >= F are zero) and its scales hs [ceil(F/128)][rows]
- * fp32. They stay valid until the workspace is reused. */
-moe_status moe_test_workspace_h(moe_layer_t layer, int T, size_t* h_offset, size_t* hs_offset);
+                                     const int32_t* offsets, int T, float* out, void* stream);
 
 #ifdef __cplusplus
 }

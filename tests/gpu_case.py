@@ -45,24 +45,15 @@ class Case:
         self.xs = torch.empty((sh.HB, rows), dtype=torch.float32, device=d)
         fx.moe_permute(self.dev, self.x, T, H, self.idx, self.offsets, self.perm, self.inv, self.xq, self.xs,
                        self.ws, nb)
+        self.hq = torch.empty((rows, sh.FB * 128), dtype=torch.uint8, device=d)
+        self.hs = torch.empty((sh.FB, rows), dtype=torch.float32, device=d)
+        fx.moe_gate_up(self.dev, self.xq, self.xs, self.offsets, T, self.hq, self.hs)
         self.y = torch.empty((rows, H), dtype=torch.bfloat16, device=d)
-        fx.moe_expert_ffn(self.dev, self.xq, self.xs, self.offsets, T, self.y, self.ws, nb)
-        # h and its scales stay in the workspace; copy them out before anything reuses it
-        self.hq, self.hs = self._workspace_h()
+        fx.moe_down(self.dev, self.hq, self.hs, self.offsets, T, self.y)
         self.out = torch.empty((T, H), dtype=torch.bfloat16, device=d)
         fx.moe_combine(self.dev, self.y, self.inv, self.w, T, self.out, H)
         code, bits = fx.moe_get_device_status(self.dev)
         assert code == fx.MOE_OK, f"device status {bits:#x}"
-
-    def _workspace_h(self):
-        """The quantised SwiGLU output h [rows][ld_hh] and hs [FB][rows] that
-        moe_expert_ffn leaves in the workspace."""
-        sh, rows = self.sh, self.rows
-        h_off, hs_off = fx.moe_test_workspace_h(self.dev, self.T)
-        ld_hh = sh.FB * 128
-        hq = self.ws[h_off:h_off + rows * ld_hh].view(rows, ld_hh).clone()
-        hs = self.ws[hs_off:hs_off + 4 * sh.FB * rows].view(torch.float32).view(sh.FB, rows).clone()
-        return hq, hs
 
     # host copies
     def np(self, name):
@@ -98,15 +89,30 @@ def oracle_ffn_on_rows(layer, rows, xq, xs_rows_major, offsets):
     return {k: v[inv_order] for k, v in f.items()}
 
 
+def bf16_half_ulp(v: np.ndarray) -> np.ndarray:
+    """Half a unit in the last place of bf16 (8 significant bits) at |v|."""
+    a = np.maximum(np.abs(np.asarray(v, np.float64)), 2.0 ** -126)
+    return 2.0 ** (np.floor(np.log2(a)) - 8)
+
+
 def assert_output_close(got: np.ndarray, ref: np.ndarray, what: str, rel_fro=REL_FRO, max_abs_rms=MAX_ABS_RMS):
+    """The layer's parity bar on a bf16 output against the unrounded FP64
+    oracle: relative Frobenius error <= rel_fro, and max-abs error <=
+    max_abs_rms * rms(ref) applied to the value before its one rounding to
+    bf16, i.e. |got - ref| <= max_abs_rms * rms + half a bf16 ulp of ref.
+    (Without the half ulp no bf16 output could pass once |ref| > 5.1 rms.)"""
     got = np.asarray(got, np.float64)
     ref = np.asarray(ref, np.float64)
     assert np.all(np.isfinite(got)), f"{what}: non-finite values"
     rms = np.sqrt(np.mean(ref ** 2))
     rel = np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-300)
-    mx = np.max(np.abs(got - ref)) if got.size else 0.0
+    err = np.abs(got - ref)
+    excess = err - bf16_half_ulp(ref)
+    mx = float(np.max(excess)) if got.size else 0.0
     assert rel <= rel_fro, f"{what}: relative Frobenius error {rel:.3e} > {rel_fro}"
-    assert mx <= max_abs_rms * rms, f"{what}: max abs error {mx:.3e} > {max_abs_rms} * rms {rms:.3e}"
+    assert mx <= max_abs_rms * rms, \
+        f"{what}: max abs error beyond bf16 rounding {mx:.3e} > {max_abs_rms} * rms {rms:.3e}" \
+        f" (raw max abs {err.max():.3e})"
     return rel, mx / rms
 
 

@@ -151,11 +151,14 @@ def test_layer_end_to_end(name):
     ref = moe.token_outputs(c.x_bits, layer, keep)
     out = moe.bf16_to_f64(c.np("out"))[keep]
     gc.assert_output_close(out, ref, f"{name}: layer output")
-    # the fused entry point gives the same bytes as the four stages
+    # the composed entry points give the same bytes as the stage calls
     ws = tu.workspace(c.dev, T)
     o2 = torch.empty_like(c.out)
     fx.moe_layer_forward(c.dev, c.x, T, layer.shape.H, o2, layer.shape.H, ws, ws.numel())
     assert torch.equal(o2.view(torch.int16), c.out.view(torch.int16))
+    y2 = torch.empty_like(c.y)
+    fx.moe_expert_ffn(c.dev, c.xq, c.xs, c.offsets, T, y2, ws, ws.numel())
+    assert torch.equal(y2.view(torch.int16), c.y.view(torch.int16))
 
 
 def test_bf16_checkpoint_cross_check():
@@ -216,9 +219,7 @@ def test_grouped_gemm_exact_integers(which):
     a_s = np.ones((nkb, rows), np.float32)
     ncols = 2 * sh.FB * 128 if which == 0 else sh.H
     out = torch.full((rows, ncols), float("nan"), device="cuda")
-    ws = tu.workspace(dev, T)
-    fx.moe_test_grouped_gemm_f32(dev, which, tu.to_device(a), tu.to_device(a_s), tu.to_device(off), T, out, ws,
-                                 ws.numel())
+    fx.moe_test_grouped_gemm_f32(dev, which, tu.to_device(a), tu.to_device(a_s), tu.to_device(off), T, out)
     got = out.cpu().numpy().astype(np.float64)
     ints = moe.e4m3.decode(np.arange(256, dtype=np.uint8))
     A = ints[a].astype(np.int64)
@@ -258,9 +259,7 @@ def test_grouped_gemm_promotion_random_scales(which):
     a_s = rng.uniform(0.001, 0.1, (nkb, rows)).astype(np.float32)
     ncols = 2 * sh.FB * 128 if which == 0 else sh.H
     out = torch.zeros((rows, ncols), device="cuda")
-    ws = tu.workspace(dev, T)
-    fx.moe_test_grouped_gemm_f32(dev, which, tu.to_device(a), tu.to_device(a_s), tu.to_device(off), T, out, ws,
-                                 ws.numel())
+    fx.moe_test_grouped_gemm_f32(dev, which, tu.to_device(a), tu.to_device(a_s), tu.to_device(off), T, out)
     got = out.cpu().numpy().astype(np.float64)
     A = moe.dequant_rows(a, a_s.T.copy())
     for g in range(sh.E + 1):
