@@ -67,38 +67,47 @@ def dist_setup(n):
 
 
 class Dist:
-    def __init__(self, world, rank, local, backend="nccl"):
-        import torch
+    """One process per GPU; every rank runs its own replica of the layer. The
+    only collectives are the barriers around the timed region and the
+    reductions of the timing (max over ranks) and of the token count (sum)."""
+
+    def __init__(self, world, rank, local, backend="nccl", timeout_s=600):
         import torch.distributed as dist
         self.world, self.rank, self.local = world, rank, local
         self.dist = dist if world > 1 else None
+        self.device = "cuda" if backend == "nccl" else "cpu"
         if self.dist:
             from datetime import timedelta
-            dist.init_process_group(backend, timeout=timedelta(seconds=600))
+            dist.init_process_group(backend, timeout=timedelta(seconds=timeout_s))
 
     def barrier(self):
         if self.dist:
             self.dist.barrier()
 
-    def max(self, v: float) -> float:
+    def _reduce(self, v: float, op) -> float:
         if not self.dist:
             return v
         import torch
-        t = torch.tensor([v], dtype=torch.float64, device="cuda")
-        self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
+        t = torch.tensor([v], dtype=torch.float64, device=self.device)
+        self.dist.all_reduce(t, op=op)
         return float(t.item())
 
+    def max(self, v: float) -> float:
+        return v if not self.dist else self._reduce(v, self.dist.ReduceOp.MAX)
+
     def sum(self, v: float) -> float:
-        if not self.dist:
-            return v
-        import torch
-        t = torch.tensor([v], dtype=torch.float64, device="cuda")
-        self.dist.all_reduce(t, op=self.dist.ReduceOp.SUM)
-        return float(t.item())
+        return v if not self.dist else self._reduce(v, self.dist.ReduceOp.SUM)
 
     def close(self):
         if self.dist:
             self.dist.destroy_process_group()
+
+
+def job_throughput(d: "Dist", tokens_this_rank: float, ms_this_rank: float):
+    """Whole-job tokens/s: all ranks' tokens over the slowest rank's time."""
+    ms = d.max(ms_this_rank)
+    tokens = d.sum(tokens_this_rank)
+    return tokens / (ms / 1e3), ms, tokens
 
 
 # ----------------------------------------------------------------------------- clocks
@@ -341,9 +350,7 @@ def run_ours(args):
     visible = os.environ.get("CUDA_VISIBLE_DEVICES", "")
     sampler = ClockSampler(visible.split(",")[local] if visible else local)
     total_ms, per, clocks = time_stages(st, args.steps, args.warmup, d, sampler)
-    total_ms = d.max(total_ms)
-    tokens = d.sum(float(T * args.steps))
-    value = tokens / (total_ms / 1e3)
+    value, total_ms, tokens = job_throughput(d, float(T * args.steps), total_ms)
     off = st.offsets.cpu().numpy()
     work = algorithmic_work(wl, T, off)
     # the dominant kernel: decode-sized batches are bound by streaming the

@@ -17,7 +17,10 @@ NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-cudart", "shared",
-         "--expt-relaxed-constexpr", "-Werror", "all-warnings"]
+         "--expt-relaxed-constexpr", "-Werror", "all-warnings", "-Xcompiler", "-fvisibility=hidden"]
+
+
+PER_FILE = {}
 
 
 def sources():
@@ -44,7 +47,7 @@ def build(force: bool = False, verbose_ptxas: bool = False) -> str:
     extra = ["-Xptxas", "-v"] if verbose_ptxas else []
     for src in sources():
         obj = os.path.join(BUILD_DIR, os.path.basename(src) + ".o")
-        cmd = [NVCC, *ARCH, *FLAGS, *extra, "-c", src, "-o", obj]
+        cmd = [NVCC, *ARCH, *FLAGS, *PER_FILE.get(os.path.basename(src), []), *extra, "-c", src, "-o", obj]
         subprocess.check_call(cmd)
         objs.append(obj)
     tmp = LIB + f".tmp{os.getpid()}"

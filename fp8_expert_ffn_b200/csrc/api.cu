@@ -1,6 +1,7 @@
 // C ABI of the FP8 MoE-layer library: argument validation, the layer handle,
 // workspace carving and the composition of the stages. No entry point
-// allocates device memory except moe_layer_create (one 4-byte status word).
+// allocates device memory except moe_layer_create (a 4-byte status word and
+// the router weight's bf16 split).
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -36,19 +37,24 @@ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 }  // namespace
 
-bool encode_tmap_u8(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t rows, uint64_t depth, uint64_t ld,
-                    uint64_t depth_stride) {
+bool encode_tmap(CUtensorMap* tm, bool bf16, const void* base, uint64_t inner, uint64_t rows, uint64_t depth,
+                 uint64_t ld_bytes, uint64_t depth_stride_bytes) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[3] = {inner, rows, depth};
-  cuuint64_t strides[2] = {ld, depth_stride};
-  cuuint32_t box[3] = {128, 128, 1};
+  cuuint64_t strides[2] = {ld_bytes, depth_stride_bytes};
+  cuuint32_t box[3] = {bf16 ? 64u : 128u, 128, 1};   // 128 bytes of K per box row
   cuuint32_t estr[3] = {1, 1, 1};
   const cuuint32_t rank = depth > 1 ? 3 : 2;
-  CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, rank, const_cast<void*>(base), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult r = fn(tm, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, rank,
+                  const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+bool encode_tmap_u8(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t rows, uint64_t depth, uint64_t ld,
+                    uint64_t depth_stride) {
+  return encode_tmap(tm, false, base, inner, rows, depth, ld, depth_stride);
 }
 
 Scratch carve(const moe_layer_s* L, int T, void* base) {
@@ -109,6 +115,7 @@ constexpr int kMaxT = 1 << 20;
 
 }  // namespace
 
+#pragma GCC visibility push(default)
 extern "C" {
 
 const char* moe_status_string(moe_status s) {
@@ -167,12 +174,17 @@ moe_status moe_layer_create(const moe_layer_desc* d, const moe_weights* w, moe_l
     delete L;
     return MOE_ERR_CUDA;
   }
-  if (cudaMalloc(&L->status, sizeof(uint32_t)) != cudaSuccess) {
-    delete L;
-    return MOE_ERR_CUDA;
-  }
-  if (cudaMemset(L->status, 0, sizeof(uint32_t)) != cudaSuccess) {
+  const size_t split_bytes = 3 * size_t(L->E) * L->H * sizeof(uint16_t);
+  bool ok = cudaMalloc(&L->status, sizeof(uint32_t)) == cudaSuccess;
+  ok = ok && cudaMalloc(&L->router_split, split_bytes) == cudaSuccess;
+  ok = ok && cudaMemset(L->status, 0, sizeof(uint32_t)) == cudaSuccess;
+  ok = ok && launch_router_split(w->router_w, L->E, L->H, L->router_split, nullptr) == cudaSuccess;
+  ok = ok && cudaDeviceSynchronize() == cudaSuccess;
+  ok = ok && encode_tmap(&L->tm_router, true, L->router_split, L->H, L->E, 3, uint64_t(L->H) * 2,
+                         uint64_t(L->E) * L->H * 2);
+  if (!ok) {
     cudaFree(L->status);
+    cudaFree(L->router_split);
     delete L;
     return MOE_ERR_CUDA;
   }
@@ -183,8 +195,9 @@ moe_status moe_layer_create(const moe_layer_desc* d, const moe_weights* w, moe_l
 moe_status moe_layer_destroy(moe_layer_t L) {
   if (!L) return MOE_OK;
   cudaError_t e = cudaFree(L->status);
+  cudaError_t e2 = cudaFree(L->router_split);
   delete L;
-  return from_cuda(e);
+  return from_cuda(e != cudaSuccess ? e : e2);
 }
 
 size_t moe_workspace_size(moe_layer_t L, int T) {
@@ -301,3 +314,4 @@ moe_status moe_test_grouped_gemm_f32(moe_layer_t L, int which, const uint8_t* a,
 }
 
 }  // extern "C"
+#pragma GCC visibility pop

@@ -16,7 +16,8 @@ namespace {
 
 constexpr int CB_THREADS = 128;
 
-// One CTA per token; each thread owns 8-channel (16-byte) chunks.
+// CTA (token, chunk of CB_THREADS*8 channels); each thread owns one
+// 8-channel (16-byte) piece and loads its K+1 rows at once.
 __global__ void __launch_bounds__(CB_THREADS) combine_kernel(const uint16_t* __restrict__ y,
                                                              const int32_t* __restrict__ inv,
                                                              const float* __restrict__ w, int T, int K, int H,
@@ -30,13 +31,21 @@ __global__ void __launch_bounds__(CB_THREADS) combine_kernel(const uint16_t* __r
   }
   __syncthreads();
   const size_t shared_row = size_t(T) * K + t;
-  for (int c = threadIdx.x * 8; c < H; c += CB_THREADS * 8) {
+  const int c = (blockIdx.y * CB_THREADS + threadIdx.x) * 8;
+  if (c < H) {
+    uint4 raws[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int r = k < K ? s_row[k] : -1;
+      raws[k] = r >= 0 ? *reinterpret_cast<const uint4*>(y + size_t(r) * H + c) : make_uint4(0, 0, 0, 0);
+    }
+    const uint4 raw_shared = *reinterpret_cast<const uint4*>(y + shared_row * H + c);
     float acc[8] = {};
-    for (int k = 0; k < K; ++k) {
-      const int r = s_row[k];
-      if (r < 0) continue;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      if (k >= K || s_row[k] < 0) continue;
       const float wk = s_w[k];
-      const uint4 raw = *reinterpret_cast<const uint4*>(y + size_t(r) * H + c);
+      const uint4 raw = raws[k];
       const uint32_t p[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
@@ -44,8 +53,7 @@ __global__ void __launch_bounds__(CB_THREADS) combine_kernel(const uint16_t* __r
         acc[2 * j + 1] = fmaf(wk, bf16_bits_to_f32(uint16_t(p[j] >> 16)), acc[2 * j + 1]);
       }
     }
-    const uint4 raw = *reinterpret_cast<const uint4*>(y + shared_row * H + c);
-    const uint32_t p[4] = {raw.x, raw.y, raw.z, raw.w};
+    const uint32_t p[4] = {raw_shared.x, raw_shared.y, raw_shared.z, raw_shared.w};
     uint32_t o[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
@@ -61,7 +69,8 @@ __global__ void __launch_bounds__(CB_THREADS) combine_kernel(const uint16_t* __r
 
 cudaError_t launch_combine(const moe_layer_s* L, const uint16_t* y, const int32_t* inv, const float* w, int T,
                            uint16_t* out, int ldo, cudaStream_t st) {
-  combine_kernel<<<T, CB_THREADS, 0, st>>>(y, inv, w, T, L->K, L->H, out, ldo);
+  dim3 grid(T, (L->H + CB_THREADS * 8 - 1) / (CB_THREADS * 8));
+  combine_kernel<<<grid, CB_THREADS, 0, st>>>(y, inv, w, T, L->K, L->H, out, ldo);
   return cudaGetLastError();
 }
 

@@ -195,6 +195,18 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
 
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
+// (a0, a1) += (v0, v1) * f with one packed f32x2 FMA (round to nearest).
+__device__ __forceinline__ void ffma2(float& a0, float& a1, float v0, float v1, float f) {
+  asm("{\n\t.reg .b64 a, v, s, r;\n\t"
+      "mov.b64 a, {%0, %1};\n\t"
+      "mov.b64 v, {%2, %3};\n\t"
+      "mov.b64 s, {%4, %4};\n\t"
+      "fma.rn.f32x2 r, v, s, a;\n\t"
+      "mov.b64 {%0, %1}, r;\n\t}"
+      : "+f"(a0), "+f"(a1)
+      : "f"(v0), "f"(v1), "f"(f));
+}
+
 // ---------------------------------------------------------------- PDL
 
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }

@@ -52,7 +52,19 @@ constexpr int A_BYTES = BM * BK;           // 16 KB
 constexpr int BH_BYTES = 128 * BK;         // 16 KB per B half
 constexpr int STAGE_BYTES = A_BYTES + 2 * BH_BYTES;
 constexpr int EPI_WARPS = 8;
-constexpr int THREADS = 64 + EPI_WARPS * 32;
+// Three warpgroups: warpgroup 0 = TMA warp, MMA warp and two idle warps;
+// warpgroups 1 and 2 = the epilogue. setmaxnreg moves registers from the
+// first to the other two: the launch gets LAUNCH_REGS per thread (the
+// 384-thread, one-CTA-per-SM cap), the producer warpgroup keeps PRODUCER_REGS
+// and each epilogue thread gets EPILOGUE_REGS (128 FP32 accumulators plus
+// two 32-column TMEM loads in flight). The split adds up to the launch total.
+constexpr int THREADS = 384;
+constexpr int FIRST_EPI_WARP = 4;
+constexpr int LAUNCH_REGS = 168;
+constexpr int PRODUCER_REGS = 40;
+constexpr int EPILOGUE_REGS = 232;
+static_assert(128 * PRODUCER_REGS + 256 * EPILOGUE_REGS <= THREADS * LAUNCH_REGS, "register split exceeds launch");
+static_assert(THREADS == 32 * (FIRST_EPI_WARP + EPI_WARPS), "warp layout");
 constexpr int MCHUNK = 8;                  // row tiles per chunk of the tile order
 constexpr int MAX_GROUPS = 257;
 constexpr uint32_t TMEM_COLS = 512;
@@ -187,6 +199,11 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int total = s_prefix[p.ngroups];
   uint32_t issued = 0;
 
+  // The two warpgroup kinds run to the end of the kernel on separate paths
+  // (each with its own copy of the teardown), so that the register limits
+  // set by setmaxnreg hold on every instruction they execute.
+  if (warp < FIRST_EPI_WARP) {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(PRODUCER_REGS));
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -244,11 +261,25 @@ __global__ void __launch_bounds__(THREADS, 1)
       tc_commit(&done_bar);                 // all MMAs issued above have completed
       mbar_wait_drain(&done_bar, 0, p.status);
     }
+  }
+  // ---------------------------------------------------- teardown (warpgroup 0)
+  asm volatile("bar.sync 0;" ::: "memory");
+  if (warp == 0 && lane == 0) {
+    // copies issued but never consumed (only after an abort) must land first
+    for (uint32_t j = s_consumed; j < issued; ++j) mbar_wait_drain(&full_bar[j % STAGES], (j / STAGES) & 1u, p.status);
+  }
+  tc_fence_before();
+  asm volatile("bar.sync 0;" ::: "memory");
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(EPILOGUE_REGS));
     // ------------------------------------------------------------ epilogue
-    const int ew = warp - 2;
+    const int ew = warp - FIRST_EPI_WARP;
     const int q = warp & 3;          // TMEM lane quarter this warp may access
-    const int half = ew >> 2;        // column half of the tile
+    const int half = ew >> 2;        // column half of the tile (one per warpgroup)
     const int r_in = q * 32 + lane;  // row within the tile
     uint32_t tb = 0;
     uint32_t tile_iter = 0;
@@ -273,25 +304,52 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
       for (int j = 0; j < 128; ++j) acc[j] = 0.0f;
 
+      // Scales stay off the critical path: lane l holds the weight scales
+      // of K block (window + l), broadcast by a shuffle; the row's
+      // activation scales are prefetched four K blocks ahead.
+      float wr0 = 0.0f, wr1 = 0.0f;
+      const float* asp = p.as + row;
+      const size_t ast = size_t(p.rows);
+      float pf0 = 0.0f, pf1 = 0.0f, pf2 = 0.0f, pf3 = 0.0f;
+      if (valid) {
+        pf0 = __ldg(asp);
+        if (p.nkb > 1) pf1 = __ldg(asp + ast);
+        if (p.nkb > 2) pf2 = __ldg(asp + 2 * ast);
+        if (p.nkb > 3) pf3 = __ldg(asp + 3 * ast);
+      }
+
       for (int kb = 0; kb < p.nkb; ++kb) {
         const uint32_t buf = tb & 1u, tph = (tb >> 1) & 1u;
-        const float sa = valid ? __ldg(p.as + size_t(kb) * p.rows + row) : 0.0f;
-        const float f0 = __ldg(w0 + kb) * sa;
-        const float f1 = __ldg(w1 + kb) * sa;
+        if ((kb & 31) == 0) {
+          const int k = kb + lane;
+          wr0 = k < p.nkb ? __ldg(w0 + k) : 0.0f;
+          wr1 = k < p.nkb ? __ldg(w1 + k) : 0.0f;
+        }
+        const float sa = pf0;
+        pf0 = pf1;
+        pf1 = pf2;
+        pf2 = pf3;
+        pf3 = (valid && kb + 4 < p.nkb) ? __ldg(asp + size_t(kb + 4) * ast) : 0.0f;
+        const float f0 = __shfl_sync(0xFFFFFFFFu, wr0, kb & 31) * sa;
+        const float f1 = __shfl_sync(0xFFFFFFFFu, wr1, kb & 31) * sa;
         if (!mbar_wait(&tfull_bar[buf], tph, s_abort, p.status)) { ok = false; break; }
         tc_fence_after();
         if (warp_active) {
           const uint32_t tbase = tmem_base + (uint32_t(q * 32) << 16) + buf * BN;
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const uint32_t col = (MODE == MODE_GATEUP) ? uint32_t((c >> 1) * 128 + half * 64 + (c & 1) * 32)
+          for (int c = 0; c < 4; c += 2) {   // two 32-column chunks per TMEM round trip
+            const uint32_t col = (MODE == MODE_GATEUP) ? uint32_t((c >> 1) * 128 + half * 64)
                                                        : uint32_t(half * 128 + c * 32);
-            float v[32];
-            tmem_ld32(tbase + col, v);
+            float va[32], vb[32];
+            tmem_ld32(tbase + col, va);
+            tmem_ld32(tbase + col + 32, vb);
             tmem_ld_wait();
             const float f = (MODE == MODE_GATEUP && c >= 2) ? f1 : f0;
 #pragma unroll
-            for (int j = 0; j < 32; ++j) acc[c * 32 + j] = fmaf(v[j], f, acc[c * 32 + j]);
+            for (int j = 0; j < 32; j += 2) {
+              ffma2(acc[c * 32 + j], acc[c * 32 + j + 1], va[j], va[j + 1], f);
+              ffma2(acc[c * 32 + 32 + j], acc[c * 32 + 33 + j], vb[j], vb[j + 1], f);
+            }
           }
         }
         tc_fence_before();
@@ -319,12 +377,14 @@ __global__ void __launch_bounds__(THREADS, 1)
         // h = silu(G) * U for this thread's 64 channels, then the row's
         // 128-channel amax across the two column halves.
         float amax = 0.0f;
+        if (warp_active) {
 #pragma unroll
-        for (int j = 0; j < 64; ++j) {
-          const float g = acc[j];
-          const float hv = g / (1.0f + expf(-g)) * acc[64 + j];
-          acc[j] = hv;
-          amax = fmaxf(amax, fabsf(hv));
+          for (int j = 0; j < 64; ++j) {
+            const float g = acc[j];
+            const float hv = g / (1.0f + expf(-g)) * acc[64 + j];
+            acc[j] = hv;
+            amax = fmaxf(amax, fabsf(hv));
+          }
         }
         const uint32_t xb = tile_iter & 1u;
         s_amax[xb][half][r_in] = amax;
@@ -368,19 +428,11 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
       }
     }
-  }
 
-  // ------------------------------------------------------------ teardown
-  __syncthreads();
-  if (warp == 0 && lane == 0) {
-    // copies issued but never consumed (only after an abort) must land first
-    for (uint32_t j = s_consumed; j < issued; ++j) mbar_wait_drain(&full_bar[j % STAGES], (j / STAGES) & 1u, p.status);
-  }
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem_base, TMEM_COLS);
+    // ------------------------------------------------ teardown (epilogue side)
+    asm volatile("bar.sync 0;" ::: "memory");
+    tc_fence_before();
+    asm volatile("bar.sync 0;" ::: "memory");
   }
 }
 
@@ -389,8 +441,14 @@ cudaError_t launch_gemm(const moe_layer_s* L, const CUtensorMap& tmA, const CUte
                         const CUtensorMap& tmB1, const GemmArgs& a, cudaStream_t st) {
   static bool configured = false;  // per process; the attribute is per function
   if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<MODE, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         SMEM_DYN);
+    // setmaxnreg.inc waits until the registers it asks for are free; they
+    // come only from this CTA's launch allocation, so refuse to launch a
+    // build whose register count cannot fund the split.
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, grouped_gemm_kernel<MODE, EPI>);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs * THREADS < 128 * PRODUCER_REGS + 256 * EPILOGUE_REGS) return cudaErrorInvalidConfiguration;
+    e = cudaFuncSetAttribute(grouped_gemm_kernel<MODE, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_DYN);
     if (e != cudaSuccess) return e;
     configured = true;
   }

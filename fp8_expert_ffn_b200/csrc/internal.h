@@ -19,6 +19,8 @@ struct moe_layer_s {
   int device;
   int num_sms;
   uint32_t* status;  // device status word
+  uint16_t* router_split;  // [3][E][H] bf16 terms of router_w (library-owned)
+  CUtensorMap tm_router;   // over router_split, box 64 x 128 x 1
   CUtensorMap tm_gate;  // [E+1][F][ld_h] E4M3, box 128 x 128 x 1
   CUtensorMap tm_up;
   CUtensorMap tm_down;  // [E+1][H][ld_f] E4M3, box 128 x 128 x 1
@@ -70,5 +72,12 @@ cudaError_t launch_combine(const moe_layer_s* L, const uint16_t* y, const int32_
 // `ld` bytes, 128 x 128 boxes, 128-byte swizzle (3-D when depth > 1).
 bool encode_tmap_u8(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t rows, uint64_t depth,
                     uint64_t ld, uint64_t depth_stride);
+// Same for bf16 (box 64 x 128 elements = 128 bytes of K per row) or u8.
+bool encode_tmap(CUtensorMap* tm, bool bf16, const void* base, uint64_t inner, uint64_t rows, uint64_t depth,
+                 uint64_t ld_bytes, uint64_t depth_stride_bytes);
+
+// Router weight split into three bf16 terms (hi + mid + lo == w exactly for
+// normal-range fp32 w), [3][E][H]; written once at layer creation.
+cudaError_t launch_router_split(const float* w, int E, int H, uint16_t* out, cudaStream_t st);
 
 }  // namespace moe

@@ -96,15 +96,29 @@ __global__ void __launch_bounds__(256) permute_offsets_kernel(const int32_t* __r
   }
 }
 
-// One warp per token. Lane k < K owns slot k; lane K owns the shared row.
+constexpr int GATHER_GROUPS = 8;   // 128-channel groups per warp
+
+// One warp per (token, chunk of GATHER_GROUPS groups). Lane k < K owns slot
+// k; lane K owns the shared row. The chunk-0 warp writes inv and perm.
 __global__ void __launch_bounds__(256) permute_gather_kernel(
     const uint16_t* __restrict__ x, int T, int ldx, int H, const int32_t* __restrict__ idx, int K, int E, int W,
     const uint32_t* __restrict__ bitmap, const uint32_t* __restrict__ wprefix, const int32_t* __restrict__ offsets,
     int rows, int32_t* __restrict__ perm, int32_t* __restrict__ inv, uint8_t* __restrict__ xq,
     float* __restrict__ xs) {
   const int lane = threadIdx.x & 31;
-  const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int HB = H / 128;
+  const int nchunk = (HB + GATHER_GROUPS - 1) / GATHER_GROUPS;
+  const int wid = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int t = wid / nchunk, chunk = wid - t * nchunk;
   if (t >= T) return;
+  const int g0 = chunk * GATHER_GROUPS, g1 = min(HB, g0 + GATHER_GROUPS);
+  const uint16_t* xr = x + size_t(t) * ldx;
+  // issue the x loads of the whole chunk before anything waits on memory
+  uint2 raw[GATHER_GROUPS];
+#pragma unroll
+  for (int i = 0; i < GATHER_GROUPS; ++i)
+    raw[i] = (g0 + i < g1) ? *reinterpret_cast<const uint2*>(xr + (g0 + i) * 128 + lane * 4) : make_uint2(0, 0);
+
   int my_row = -1;
   if (lane < K) {
     const int e = idx[size_t(t) * K + lane];
@@ -114,23 +128,23 @@ __global__ void __launch_bounds__(256) permute_gather_kernel(
       const uint32_t word = bitmap[size_t(e) * W + (t >> 5)];
       my_row = offsets[e] + int(wprefix[size_t(e) * W + (t >> 5)]) + __popc(word & ((1u << (t & 31)) - 1u));
     }
-    inv[size_t(t) * K + lane] = my_row;
+    if (chunk == 0) inv[size_t(t) * K + lane] = my_row;
   } else if (lane == K) {
     my_row = offsets[E] + t;
   }
-  if (my_row >= 0) perm[my_row] = t;
+  if (chunk == 0 && my_row >= 0) perm[my_row] = t;
   // rows of this token, known to every lane
   int rowv[9];
 #pragma unroll
   for (int j = 0; j < 9; ++j) rowv[j] = __shfl_sync(0xFFFFFFFFu, my_row, j);
 
-  const uint16_t* xr = x + size_t(t) * ldx;
-  const int HB = H / 128;
-  for (int g = 0; g < HB; ++g) {
+#pragma unroll
+  for (int i = 0; i < GATHER_GROUPS; ++i) {
+    const int g = g0 + i;
+    if (g >= g1) break;
     // lane holds channels g*128 + lane*4 .. +3
-    const uint2 raw = *reinterpret_cast<const uint2*>(xr + g * 128 + lane * 4);
-    float v[4] = {bf16_bits_to_f32(uint16_t(raw.x & 0xFFFFu)), bf16_bits_to_f32(uint16_t(raw.x >> 16)),
-                  bf16_bits_to_f32(uint16_t(raw.y & 0xFFFFu)), bf16_bits_to_f32(uint16_t(raw.y >> 16))};
+    float v[4] = {bf16_bits_to_f32(uint16_t(raw[i].x & 0xFFFFu)), bf16_bits_to_f32(uint16_t(raw[i].x >> 16)),
+                  bf16_bits_to_f32(uint16_t(raw[i].y & 0xFFFFu)), bf16_bits_to_f32(uint16_t(raw[i].y >> 16))};
     float amax = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
@@ -168,8 +182,10 @@ cudaError_t launch_permute(const moe_layer_s* L, const uint16_t* x, int T, int l
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   permute_offsets_kernel<<<1, 256, 0, st>>>(s.counts, E, T, offsets);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  permute_gather_kernel<<<(T + 7) / 8, 256, 0, st>>>(x, T, ldx, L->H, idx, K, E, W, s.bitmap, s.wprefix, offsets,
-                                                     rows, perm, inv, xq, xs);
+  const int nchunk = (L->HB + GATHER_GROUPS - 1) / GATHER_GROUPS;
+  const long long warps = static_cast<long long>(T) * nchunk;
+  permute_gather_kernel<<<unsigned((warps + 7) / 8), 256, 0, st>>>(x, T, ldx, L->H, idx, K, E, W, s.bitmap,
+                                                                   s.wprefix, offsets, rows, perm, inv, xq, xs);
   return cudaGetLastError();
 }
 

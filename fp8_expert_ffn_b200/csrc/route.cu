@@ -1,5 +1,5 @@
-// Router: FP32 logits = x . Wr^T, then top-K per token with renormalised
-// softmax weights.
+// Router: FP32-accurate logits = x . Wr^T on the tensor cores, then top-K per
+// token with renormalised softmax weights.
 //
 // transformers docs page "Dots 3 Note Preview", Dots3NoteTextConfig:
 // n_routed_experts 256, num_experts_per_tok 8, n_group 1 / topk_group 1
@@ -7,11 +7,21 @@
 // FP32 (transformers PR #47844 states FP32 routing for the vision MoE router;
 // the same precision is taken for the text router).
 //
-// Kernel 1 (route_logits): CTA tile of 64 tokens x 64 experts over a range of
-// 128-channel K blocks (split-K when there are too few tiles to fill the
-// GPU); per-thread 4 x 4 register tile; each K block is summed on its own and
-// then added to the running sum (blocked summation keeps the FP32 error well
-// under the near-tie threshold). Partial sums go to partial[s][t][e].
+// FP32 accuracy from bf16 tensor cores: x is bf16 already, and every fp32
+// router weight splits exactly into three bf16 terms, w = hi + mid + lo
+// (8 significant bits each; the split is written once at layer creation). A
+// product of two bf16 values is exact in fp32, so x . Wr^T = sum over the
+// three terms of bf16 GEMMs, each with exact products. The tensor cores sum
+// the 3 x 64 products of one 64-channel K block into an fp32 TMEM partial;
+// epilogue warps add each partial into an fp32 register accumulator (blocked
+// summation, error far below the near-tie threshold of the routing).
+//
+// Kernel 1 (route_tc_kernel): CTA tile 128 tokens x 128 experts over a range of
+// 64-channel K blocks (split-K when there are fewer tiles than SMs); warp 0
+// TMA (x box 128 x 64 bf16 plus three 128 x 64 weight boxes per stage, 3
+// stages), warp 1 tcgen05.mma kind::f16 (M 128, N 128, K 16; 12 per stage)
+// into two 128-column TMEM buffers, warps 2-5 promote. Partial sums go to
+// partial[s][t][e].
 // Kernel 2 (route_topk): one warp per token sums the S partials in order,
 // selects the top K by logit with ties to the lower id (an order-preserving
 // 64-bit key), and writes the slots in ascending expert id with weights
@@ -24,83 +34,196 @@ namespace moe {
 
 namespace {
 
-constexpr int RT_T = 64;    // tokens per CTA tile
-constexpr int RT_E = 64;    // experts per CTA tile
-constexpr int RT_KC = 32;   // channels per shared-memory chunk
-constexpr int RT_THREADS = 256;
+constexpr int RM = 128;                  // tokens per tile
+constexpr int RN = 128;                  // experts per tile
+constexpr int RK = 64;                   // channels per K block (128 bytes of bf16)
+constexpr int R_STAGES = 3;
+constexpr int R_A_BYTES = RM * RK * 2;   // 16 KB
+constexpr int R_B_BYTES = RN * RK * 2;   // 16 KB per split term
+constexpr int R_STAGE_BYTES = R_A_BYTES + 3 * R_B_BYTES;
+constexpr int R_EPI_WARPS = 4;
+constexpr int R_THREADS = 64 + 32 * R_EPI_WARPS;
+constexpr int R_SMEM_DYN = R_STAGES * R_STAGE_BYTES + 1024;
+constexpr uint32_t R_TMEM_COLS = 256;
 
-__global__ void __launch_bounds__(RT_THREADS) route_logits_kernel(const uint16_t* __restrict__ x, int T, int ldx,
-                                                                  const float* __restrict__ wr, int E, int H,
-                                                                  int kb_per_split, float* __restrict__ partial) {
-  __shared__ __align__(16) float xs[RT_KC][RT_T];
-  __shared__ __align__(16) float ws[RT_KC][RT_E];
-  const int tid = threadIdx.x;
-  const int e0 = blockIdx.x * RT_E, t0 = blockIdx.y * RT_T, split = blockIdx.z;
-  const int HB = H / 128;
+// kind::f16 instruction descriptor: A = B = BF16, D = F32, both K-major.
+constexpr uint32_t idesc_bf16_f32(int M, int N) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
+}
+constexpr uint32_t R_IDESC = idesc_bf16_f32(RM, RN);
+
+__device__ __forceinline__ void mma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__global__ void __launch_bounds__(R_THREADS, 1)
+    route_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW, int T, int E,
+                    int kb_per_split, int nkb, float* __restrict__ partial, uint32_t* status) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t full_bar[R_STAGES];
+  __shared__ __align__(8) uint64_t empty_bar[R_STAGES];
+  __shared__ __align__(8) uint64_t tfull_bar[2];
+  __shared__ __align__(8) uint64_t tempty_bar[2];
+  __shared__ __align__(8) uint64_t done_bar;
+  __shared__ uint32_t tmem_base_s;
+  __shared__ int s_abort_store;
+  __shared__ uint32_t s_consumed;
+  volatile int* s_abort = &s_abort_store;
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int e0 = blockIdx.x * RN, t0 = blockIdx.y * RM, split = blockIdx.z;
   const int kb0 = split * kb_per_split;
-  const int kb1 = min(HB, kb0 + kb_per_split);
-  const int ty = tid / 16, tx = tid % 16;   // thread tile: tokens ty*4.., experts tx*4..
+  const int kb1 = min(nkb, kb0 + kb_per_split);
+  const int n = kb1 - kb0;
 
-  float acc[4][4] = {};
-  // loader mapping: 8 consecutive channels of one row per thread
-  const int lrow = tid / 4, lk = (tid % 4) * 8;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < R_STAGES; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull_bar[b], 1);
+      mbar_init(&tempty_bar[b], R_EPI_WARPS);
+    }
+    mbar_init(&done_bar, 1);
+    s_abort_store = 0;
+    s_consumed = 0;
+    fence_mbar_init();
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmX);
+    tma_prefetch_desc(&tmW);
+  }
+  if (warp == 1) tmem_alloc(&tmem_base_s, R_TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = tmem_base_s;
+  uint32_t issued = 0;
 
-  for (int kb = kb0; kb < kb1; ++kb) {
-    float part[4][4] = {};
-    for (int kc = 0; kc < 128; kc += RT_KC) {
-      const int k = kb * 128 + kc + lk;
-      {  // x chunk: token t0+lrow, channels k..k+7 (bf16)
-        const int t = t0 + lrow;
-        float v[8] = {};
-        if (t < T) {
-          uint4 raw = *reinterpret_cast<const uint4*>(x + size_t(t) * ldx + k);
-          const uint16_t* p = reinterpret_cast<const uint16_t*>(&raw);
+  if (warp == 0) {
+    if (lane == 0) {
+      uint32_t it = 0;
+      for (int kb = 0; kb < n; ++kb) {
+        const int s = it % R_STAGES;
+        const uint32_t ph = (it / R_STAGES) & 1u;
+        if (!mbar_wait(&empty_bar[s], ph ^ 1u, s_abort, status)) break;
+        uint8_t* a = smem + s * R_STAGE_BYTES;
+        mbar_arrive_expect_tx(&full_bar[s], R_STAGE_BYTES);
+        const int k = (kb0 + kb) * RK;
+        tma_load_2d(a, &tmX, &full_bar[s], k, t0);
 #pragma unroll
-          for (int j = 0; j < 8; ++j) v[j] = bf16_bits_to_f32(p[j]);
-        }
-#pragma unroll
-        for (int j = 0; j < 8; ++j) xs[lk + j][lrow] = v[j];
+        for (int j = 0; j < 3; ++j) tma_load_3d(a + R_A_BYTES + j * R_B_BYTES, &tmW, &full_bar[s], k, e0, j);
+        ++it;
       }
-      {  // W chunk: expert e0+lrow, channels k..k+7
-        const int e = e0 + lrow;
-        float v[8] = {};
-        if (e < E) {
-          const float4* p = reinterpret_cast<const float4*>(wr + size_t(e) * H + k);
-          float4 a = p[0], b = p[1];
-          v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-        }
-#pragma unroll
-        for (int j = 0; j < 8; ++j) ws[lk + j][lrow] = v[j];
-      }
-      __syncthreads();
-#pragma unroll 8
-      for (int kk = 0; kk < RT_KC; ++kk) {
-        float4 xv = *reinterpret_cast<const float4*>(&xs[kk][ty * 4]);
-        float4 wv = *reinterpret_cast<const float4*>(&ws[kk][tx * 4]);
-        const float xa[4] = {xv.x, xv.y, xv.z, xv.w};
-        const float wa[4] = {wv.x, wv.y, wv.z, wv.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-          for (int j = 0; j < 4; ++j) part[i][j] = fmaf(xa[i], wa[j], part[i][j]);
-      }
-      __syncthreads();
+      issued = it;
     }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      uint32_t it = 0;
+      for (int kb = 0; kb < n; ++kb) {
+        const int s = it % R_STAGES;
+        const uint32_t ph = (it / R_STAGES) & 1u;
+        const uint32_t buf = it & 1u, tph = (it >> 1) & 1u;
+        if (!mbar_wait(&tempty_bar[buf], tph ^ 1u, s_abort, status)) break;
+        if (!mbar_wait(&full_bar[s], ph, s_abort, status)) break;
+        tc_fence_after();
+        const uint32_t a_addr = smem_u32(smem + s * R_STAGE_BYTES);
+        const uint64_t ad = smem_desc_sw128(a_addr);
+        const uint32_t d = tmem_base + buf * RN;
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+        for (int j = 0; j < 3; ++j) {
+          const uint64_t bd = smem_desc_sw128(a_addr + R_A_BYTES + j * R_B_BYTES);
 #pragma unroll
-      for (int j = 0; j < 4; ++j) acc[i][j] += part[i][j];
-  }
+          for (int k = 0; k < RK / 16; ++k)   // 16 bf16 = 32 bytes = 2 in the 16-byte address field
+            mma_bf16(d, ad + uint64_t(2 * k), bd + uint64_t(2 * k), R_IDESC, (j | k) ? 1u : 0u);
+        }
+        tc_commit(&empty_bar[s]);
+        tc_commit(&tfull_bar[buf]);
+        ++it;
+      }
+      s_consumed = it;
+      tc_commit(&done_bar);
+      int never = 0;
+      mbar_wait(&done_bar, 0, &never, status);
+    }
+  } else {
+    const int q = warp & 3;
+    const int r_in = q * 32 + lane;
+    const int t = t0 + r_in;
+    float acc[RN];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int t = t0 + ty * 4 + i;
-    if (t >= T) continue;
+    for (int j = 0; j < RN; ++j) acc[j] = 0.0f;
+    bool ok = true;
+    for (int kb = 0; kb < n; ++kb) {
+      const uint32_t buf = kb & 1u, tph = (kb >> 1) & 1u;
+      if (!mbar_wait(&tfull_bar[buf], tph, s_abort, status)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t tbase = tmem_base + (uint32_t(q * 32) << 16) + buf * RN;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int e = e0 + tx * 4 + j;
-      if (e < E) partial[(size_t(split) * T + t) * E + e] = acc[i][j];
+      for (int c = 0; c < RN / 32; c += 2) {
+        float va[32], vb[32];
+        tmem_ld32(tbase + c * 32, va);
+        tmem_ld32(tbase + c * 32 + 32, vb);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          acc[c * 32 + j] += va[j];
+          acc[c * 32 + 32 + j] += vb[j];
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty_bar[buf]);
+    }
+    if (ok && t < T) {
+      float* dst = partial + (size_t(split) * T + t) * E + e0;
+      if (e0 + RN <= E && (E % 4) == 0) {
+#pragma unroll
+        for (int j = 0; j < RN; j += 4)
+          *reinterpret_cast<float4*>(dst + j) = make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
+      } else {
+#pragma unroll
+        for (int j = 0; j < RN; ++j)
+          if (e0 + j < E) dst[j] = acc[j];
+      }
     }
   }
+
+  __syncthreads();
+  if (warp == 0 && lane == 0) {
+    int never = 0;
+    for (uint32_t j = s_consumed; j < issued; ++j)
+      mbar_wait(&full_bar[j % R_STAGES], (j / R_STAGES) & 1u, &never, status);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, R_TMEM_COLS);
+  }
+}
+
+// hi = bf16(w), mid = bf16(w - hi), lo = bf16(w - hi - mid); both
+// differences are exact in fp32.
+__global__ void router_split_kernel(const float* __restrict__ w, size_t n, uint16_t* __restrict__ out) {
+  const size_t i = size_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  const float v = w[i];
+  const uint16_t hi = f32_to_bf16_bits(v);
+  const float r1 = v - bf16_bits_to_f32(hi);
+  const uint16_t mid = f32_to_bf16_bits(r1);
+  const float r2 = r1 - bf16_bits_to_f32(mid);
+  out[i] = hi;
+  out[n + i] = mid;
+  out[2 * n + i] = f32_to_bf16_bits(r2);
 }
 
 __device__ __forceinline__ uint32_t ordered_bits(float f) {
@@ -118,18 +241,28 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
   if (t >= T) return;
-  // expert e = lane + 32*j
+  // expert e = lane + 32*j; the S split-K partials are added in order s = 0..S-1
+  float l[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) l[j] = 0.0f;
+  const float* pt = partial + size_t(t) * E + lane;
+  const size_t ps = size_t(T) * E;
+  for (int s = 0; s < S; ++s) {
+    float v[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) v[j] = (lane + 32 * j < E) ? __ldg(pt + s * ps + 32 * j) : 0.0f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) l[j] += v[j];
+  }
   unsigned long long key[8];
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
     const int e = lane + 32 * j;
     key[j] = 0ull;
     if (e < E) {
-      float l = 0.0f;
-      for (int s = 0; s < S; ++s) l += partial[(size_t(s) * T + t) * E + e];
-      l += 0.0f;  // -0 -> +0 so that equal logits compare equal
-      if (logits_out) logits_out[size_t(t) * E + e] = l;
-      key[j] = (static_cast<unsigned long long>(ordered_bits(l)) << 32) | (0xFFFFFFFFu - uint32_t(e));
+      const float lj = l[j] + 0.0f;  // -0 -> +0 so that equal logits compare equal
+      if (logits_out) logits_out[size_t(t) * E + e] = lj;
+      key[j] = (static_cast<unsigned long long>(ordered_bits(lj)) << 32) | (0xFFFFFFFFu - uint32_t(e));
     }
   }
   int my_e = -1;
@@ -172,20 +305,35 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict
 }  // namespace
 
 int route_splits(const moe_layer_s* L, int T) {
-  const int tiles = ((T + RT_T - 1) / RT_T) * ((L->E + RT_E - 1) / RT_E);
-  int s = (2 * L->num_sms + tiles - 1) / tiles;
-  if (s < 1) s = 1;
-  if (s > L->HB) s = L->HB;
-  return s;
+  const int nkb = L->H / RK;
+  const int tiles = ((T + RM - 1) / RM) * ((L->E + RN - 1) / RN);
+  int s = (L->num_sms + tiles - 1) / tiles;
+  s = s > nkb / 4 ? nkb / 4 : s;          // at least 4 K blocks per split
+  return s < 1 ? 1 : s;
+}
+
+cudaError_t launch_router_split(const float* w, int E, int H, uint16_t* out, cudaStream_t st) {
+  const size_t n = size_t(E) * H;
+  router_split_kernel<<<unsigned((n + 255) / 256), 256, 0, st>>>(w, n, out);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_route(const moe_layer_s* L, const uint16_t* x, int T, int ldx, int32_t* idx, float* w,
                          float* logits, float* partial, cudaStream_t st) {
+  static bool configured = false;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(route_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, R_SMEM_DYN);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  const int nkb = L->H / RK;
   const int S = route_splits(L, T);
-  const int kb_per = (L->HB + S - 1) / S;
-  const int S_eff = (L->HB + kb_per - 1) / kb_per;
-  dim3 grid((L->E + RT_E - 1) / RT_E, (T + RT_T - 1) / RT_T, S_eff);
-  route_logits_kernel<<<grid, RT_THREADS, 0, st>>>(x, T, ldx, L->w.router_w, L->E, L->H, kb_per, partial);
+  const int kb_per = (nkb + S - 1) / S;
+  const int S_eff = (nkb + kb_per - 1) / kb_per;
+  CUtensorMap tmX;
+  if (!encode_tmap(&tmX, true, x, L->H, T, 1, uint64_t(ldx) * 2, 0)) return cudaErrorInvalidValue;
+  dim3 grid((L->E + RN - 1) / RN, (T + RM - 1) / RM, S_eff);
+  route_tc_kernel<<<grid, R_THREADS, R_SMEM_DYN, st>>>(tmX, L->tm_router, T, L->E, kb_per, nkb, partial, L->status);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   route_topk_kernel<<<(T + 7) / 8, 256, 0, st>>>(partial, S_eff, T, L->E, L->K, L->d.routed_scaling, idx, w,

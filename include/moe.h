@@ -27,8 +27,9 @@
  *
  * Conventions for every call:
  *   - all data pointers are DEVICE pointers owned by the caller; the library
- *     never allocates after moe_layer_create (which allocates one 4-byte
- *     device status word and nothing else);
+ *     never allocates after moe_layer_create (which allocates a 4-byte
+ *     device status word and the router weight's three-term bf16 split,
+ *     3*E*H*2 bytes, and nothing else);
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default);
  *     calls are asynchronous on that stream and never synchronise the host;
  *   - bf16 tensors are passed as uint16_t bit patterns;
@@ -112,8 +113,12 @@ typedef struct moe_layer_s* moe_layer_t;
 const char* moe_status_string(moe_status s);
 
 /* Validates desc/weights, queries the current device (must be sm_100),
- * encodes the weights' TMA descriptors once and allocates the 4-byte device
- * status word. On error *out is NULL. */
+ * encodes the weights' TMA descriptors once, allocates the 4-byte device
+ * status word and writes the router weight as three bf16 terms
+ * (hi + mid + lo == router_w exactly; the tensor-core router multiplies the
+ * bf16 input by each term). Synchronises the device once. On error *out is
+ * NULL. The router weight is read only here: a later change to router_w
+ * needs a new handle. */
 moe_status moe_layer_create(const moe_layer_desc* desc, const moe_weights* w, moe_layer_t* out);
 
 /* Frees the handle (not the caller's weights). NULL is accepted. */
