@@ -19,7 +19,9 @@ MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_MISALIGNED, MOE_ERR_UNSUPPORTED, MOE_ERR_WO
 
 ENTRY_POINTS = ("moe_status_string", "moe_layer_create", "moe_layer_destroy", "moe_workspace_size", "moe_route",
                 "moe_permute", "moe_expert_ffn", "moe_combine", "moe_layer_forward", "moe_get_device_status",
-                "moe_gate_up", "moe_down", "moe_test_grouped_gemm_f32")
+                "moe_gate_up", "moe_down", "moe_test_grouped_gemm_f32", "moe_permute_noalloc")
+
+MOE_NOALLOC_MAX_TOKENS = 4096   # include/moe.h
 
 
 class MoeError(RuntimeError):
@@ -69,6 +71,7 @@ def lib(build_if_missing: bool = True):
     L.moe_layer_forward.argtypes = [P, P, I, I, P, I, P, S, P]
     L.moe_get_device_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_uint32)]
     L.moe_gate_up.argtypes = [P, P, P, P, I, P, P, P]
+    L.moe_permute_noalloc.argtypes = [P, P, I, I, P, P, P, P, P, P, P]
     L.moe_down.argtypes = [P, P, P, P, I, P, P]
     L.moe_test_grouped_gemm_f32.argtypes = [P, I, P, P, P, I, P, P]
     for name in ENTRY_POINTS:
@@ -196,3 +199,11 @@ def moe_test_grouped_gemm_f32(layer, which, a, a_scales, offsets, T, out, stream
     _check("moe_test_grouped_gemm_f32",
            lib().moe_test_grouped_gemm_f32(layer.handle, which, _ptr(a), _ptr(a_scales), _ptr(offsets), T,
                                            _ptr(out), _stream(stream)))
+
+
+def moe_permute_noalloc(layer, x, T, ldx, topk_idx, offsets, perm, inv, xq, xs, stream=None):
+    """moe_permute without a workspace (scratch in a library-owned device
+    array; T <= MOE_NOALLOC_MAX_TOKENS; calls that overlap on the GPU race)."""
+    _check("moe_permute_noalloc",
+           lib().moe_permute_noalloc(layer.handle, _ptr(x), T, ldx, _ptr(topk_idx), _ptr(offsets), _ptr(perm),
+                                     _ptr(inv), _ptr(xq), _ptr(xs), _stream(stream)))

@@ -232,6 +232,19 @@ moe_status moe_permute(moe_layer_t L, const uint16_t* x, int T, int ldx, const i
       launch_permute(L, x, T, ldx, idx, offsets, perm, inv, xq, xs, sc, static_cast<cudaStream_t>(stream)));
 }
 
+moe_status moe_permute_noalloc(moe_layer_t L, const uint16_t* x, int T, int ldx, const int32_t* idx,
+                               int32_t* offsets, int32_t* perm, int32_t* inv, uint8_t* xq, float* xs, void* stream) {
+  if (!L || T < 0) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (T > kNoAllocMaxTokens || L->E > kNoAllocMaxExperts) return MOE_ERR_UNSUPPORTED;
+  moe_status s;
+  if ((s = check_x(L, x, ldx)) != MOE_OK) return s;
+  if (!idx || !offsets || !perm || !inv || !xq || !xs) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(xq)) return MOE_ERR_MISALIGNED;
+  return from_cuda(
+      launch_permute_noalloc(L, x, T, ldx, idx, offsets, perm, inv, xq, xs, static_cast<cudaStream_t>(stream)));
+}
+
 moe_status moe_gate_up(moe_layer_t L, const uint8_t* xq, const float* xs, const int32_t* offsets, int T,
                        uint8_t* h, float* hs, void* stream) {
   if (!L || T < 0 || T > kMaxT) return MOE_ERR_INVALID_ARG;

@@ -59,6 +59,12 @@ cudaError_t launch_route(const moe_layer_s* L, const uint16_t* x, int T, int ldx
 cudaError_t launch_permute(const moe_layer_s* L, const uint16_t* x, int T, int ldx, const int32_t* idx,
                            int32_t* offsets, int32_t* perm, int32_t* inv, uint8_t* xq, float* xs,
                            const Scratch& s, cudaStream_t st);
+// Limits of the allocation-free permutation (moe_permute_noalloc).
+constexpr int kNoAllocMaxTokens = MOE_NOALLOC_MAX_TOKENS;
+constexpr int kNoAllocMaxExperts = 256;
+cudaError_t launch_permute_noalloc(const moe_layer_s* L, const uint16_t* x, int T, int ldx, const int32_t* idx,
+                                   int32_t* offsets, int32_t* perm, int32_t* inv, uint8_t* xq, float* xs,
+                                   cudaStream_t st);
 cudaError_t launch_gate_up(const moe_layer_s* L, const uint8_t* xq, const float* xs, const int32_t* offsets, int T,
                            uint8_t* h, float* hs, cudaStream_t st);
 cudaError_t launch_down(const moe_layer_s* L, const uint8_t* h, const float* hs, const int32_t* offsets, int T,

@@ -18,6 +18,8 @@
 //   4. permute_gather   one warp per token: rows of its K slots and its
 //                       shared-expert row, inv/perm, then the 128-channel
 //                       groups of x quantised once and stored to all rows.
+#include <mutex>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -187,6 +189,59 @@ cudaError_t launch_permute(const moe_layer_s* L, const uint16_t* x, int T, int l
   permute_gather_kernel<<<unsigned((warps + 7) / 8), 256, 0, st>>>(x, T, ldx, L->H, idx, K, E, W, s.bitmap,
                                                                    s.wprefix, offsets, rows, perm, inv, xq, xs);
   return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant of the permutation: its scratch (the per-expert
+// token bitmap, the per-word prefix counts and the expert counts) lives in
+// one file-scope device array instead of a caller workspace, sized for
+// kNoAllocMaxTokens tokens and kNoAllocMaxExperts experts. Every GPU that
+// loads the library holds the array (about 257 KB) until the process exits.
+// All calls on a device share it and it keeps the last call's contents: the
+// bitmap is cleared at the start of every call (the prefixes and counts are
+// fully rewritten), and calls whose kernels overlap on the GPU race on it.
+namespace {
+
+constexpr int kNoAllocWords = kNoAllocMaxExperts * ((kNoAllocMaxTokens + 31) / 32);
+static __device__ __align__(256) uint32_t g_permute_scratch[2 * kNoAllocWords + kNoAllocMaxExperts];
+
+constexpr int kMaxDevices = 64;
+uint32_t* g_scratch_addr[kMaxDevices] = {};
+std::mutex g_scratch_mutex;
+
+// Device address of g_permute_scratch on the current device. In host code
+// the array's name is only a host-side stand-in, so the address is asked of
+// the runtime once per device (with that device current) and cached.
+cudaError_t noalloc_scratch(uint32_t** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (!g_scratch_addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_permute_scratch);
+    if (e != cudaSuccess) return e;
+    g_scratch_addr[dev] = static_cast<uint32_t*>(p);
+  }
+  *out = g_scratch_addr[dev];
+  return cudaSuccess;
+}
+
+}  // namespace
+
+cudaError_t launch_permute_noalloc(const moe_layer_s* L, const uint16_t* x, int T, int ldx, const int32_t* idx,
+                                   int32_t* offsets, int32_t* perm, int32_t* inv, uint8_t* xq, float* xs,
+                                   cudaStream_t st) {
+  uint32_t* base = nullptr;
+  cudaError_t e = noalloc_scratch(&base);
+  if (e != cudaSuccess) return e;
+  const int W = (T + 31) / 32;
+  Scratch s = {};
+  s.bitmap = base;
+  s.wprefix = base + size_t(L->E) * W;
+  s.counts = reinterpret_cast<int32_t*>(base + 2 * kNoAllocWords);
+  return launch_permute(L, x, T, ldx, idx, offsets, perm, inv, xq, xs, s, st);
 }
 
 }  // namespace moe

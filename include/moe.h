@@ -154,6 +154,29 @@ moe_status moe_permute(moe_layer_t layer, const uint16_t* x, int T, int ldx, con
                        int32_t* offsets, int32_t* perm, int32_t* inv, uint8_t* xq, float* xs, void* ws,
                        size_t ws_bytes, void* stream);
 
+/* moe_permute without a workspace, for callers that cannot allocate device
+ * memory: a serving runtime that has handed all free HBM to its own pools
+ * (KV cache, weights) and owns no spare buffer to lend, a caller that is
+ * capturing a stream into a CUDA graph in a mode where cudaMalloc is not
+ * permitted, or a latency-critical path where cudaMalloc's implicit device
+ * synchronisation is not acceptable. The pages describe no such call; it
+ * exists only for those callers.
+ *   Arguments and outputs are those of moe_permute (minus ws/ws_bytes).
+ *   T must be <= MOE_NOALLOC_MAX_TOKENS; larger T returns
+ *   MOE_ERR_UNSUPPORTED before anything is launched (use moe_permute).
+ *   The scratch is one library-owned device array per GPU (about 257 KB,
+ *   held until the process exits), found with cudaGetSymbolAddress on the
+ *   first call made on each device: make that first call before capturing
+ *   any stream. Every call on a device shares that array and it keeps the
+ *   last call's contents (each call clears what must start at zero), so
+ *   calls whose kernels overlap on the GPU (other streams, other host
+ *   threads) race on it and must be serialised by the caller.
+ *   Allocates nothing: no cudaMalloc, cudaFree or allocating library call. */
+#define MOE_NOALLOC_MAX_TOKENS 4096
+moe_status moe_permute_noalloc(moe_layer_t layer, const uint16_t* x, int T, int ldx, const int32_t* topk_idx,
+                               int32_t* offsets, int32_t* perm, int32_t* inv, uint8_t* xq, float* xs,
+                               void* stream);
+
 /* Grouped expert FFN over the permuted rows: for each group g and row r in
  * it, h = silu(xq Wg_g^T) * (xq Wu_g^T) with per-128-K-block scale promotion,
  * h quantised per 128 channels (E4M3, fp32 scale), y = h Wd_g^T in FP32,
