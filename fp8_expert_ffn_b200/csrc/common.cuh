@@ -195,6 +195,19 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
 
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
+// Special-function-unit approximations (PTX ex2.approx / rcp.approx, a few
+// ulp of fp32, subnormal results flushed to zero).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // (a0, a1) += (v0, v1) * f with one packed f32x2 FMA (round to nearest).
 __device__ __forceinline__ void ffma2(float& a0, float& a1, float v0, float v1, float f) {
   asm("{\n\t.reg .b64 a, v, s, r;\n\t"

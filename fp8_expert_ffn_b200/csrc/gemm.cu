@@ -344,6 +344,11 @@ __global__ void __launch_bounds__(THREADS, 1)
             tmem_ld32(tbase + col, va);
             tmem_ld32(tbase + col + 32, vb);
             tmem_ld_wait();
+            if (c == 2) {   // the buffer is in registers: hand it back before the last FMAs
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&tempty_bar[buf]);
+            }
             const float f = (MODE == MODE_GATEUP && c >= 2) ? f1 : f0;
 #pragma unroll
             for (int j = 0; j < 32; j += 2) {
@@ -351,10 +356,11 @@ __global__ void __launch_bounds__(THREADS, 1)
               ffma2(acc[c * 32 + 32 + j], acc[c * 32 + 33 + j], vb[j], vb[j + 1], f);
             }
           }
+        } else {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tempty_bar[buf]);
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&tempty_bar[buf]);
         ++tb;
       }
       if (!ok) break;
@@ -381,7 +387,10 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
           for (int j = 0; j < 64; ++j) {
             const float g = acc[j];
-            const float hv = g / (1.0f + expf(-g)) * acc[64 + j];
+            // silu(g) * u = g * u / (1 + 2^(-g log2 e)) with the approximate
+            // exponential and reciprocal of the special-function unit (a few
+            // ulp of fp32; h is re-quantised to 3 mantissa bits next)
+            const float hv = g * acc[64 + j] * rcp_approx(1.0f + ex2_approx(-1.4426950408889634f * g));
             acc[j] = hv;
             amax = fmaxf(amax, fabsf(hv));
           }
@@ -396,11 +405,15 @@ __global__ void __launch_bounds__(THREADS, 1)
           uint32_t pk[16];
           float s = 0.0f;
           if (amax > 0.0f) {
+            // same scale rule as the activations (s = amax/448, an IEEE
+            // divide); h/s is taken as h times the correctly rounded 1/s,
+            // within one fp32 ulp of the quotient
             s = __fdiv_rn(amax, 448.0f);
+            const float inv = __frcp_rn(s);
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
-              const uint32_t lo = e4m3x2(__fdiv_rn(acc[4 * j], s), __fdiv_rn(acc[4 * j + 1], s));
-              const uint32_t hi = e4m3x2(__fdiv_rn(acc[4 * j + 2], s), __fdiv_rn(acc[4 * j + 3], s));
+              const uint32_t lo = e4m3x2(acc[4 * j] * inv, acc[4 * j + 1] * inv);
+              const uint32_t hi = e4m3x2(acc[4 * j + 2] * inv, acc[4 * j + 3] * inv);
               pk[j] = lo | (hi << 16);
             }
           } else {
