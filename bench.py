@@ -46,6 +46,25 @@ def parse():
     return p.parse_args()
 
 
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "gemm_traffic.json")
+GEMM_SOURCE = os.path.join(ROOT, "fp8_expert_ffn_b200", "csrc", "gemm.cu")
+
+
+def measured_traffic(kernel: str, algorithmic_bytes: float):
+    """DRAM bytes per launch from the committed ncu record (ratio of measured
+    to algorithmic bytes on the profiling case), or None when the GEMM source
+    has changed since the counters were taken."""
+    import hashlib
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    rec = json.load(open(TRAFFIC_FILE))
+    sha = hashlib.sha256(open(GEMM_SOURCE, "rb").read()).hexdigest()
+    key = f"{kernel}_traffic_over_algorithmic"
+    if sha != rec.get("kernel_source_sha256") or key not in rec:
+        return None
+    return round(rec[key] * algorithmic_bytes)
+
+
 def peaks():
     if os.path.exists(PEAKS_FILE):
         d = json.load(open(PEAKS_FILE))
@@ -362,7 +381,7 @@ def run_ours(args):
     if hbm_bound:
         ach = work["bytes"][kern] / (kern_ms / 1e3) / 1e9
         roof = {"bound": "hbm", "kernel": kern, "achieved": round(ach, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
-                "frac": round(ach / pk["hbm_gbs"], 4), "traffic": None,
+                "frac": round(ach / pk["hbm_gbs"], 4), "traffic": measured_traffic(kern, work["bytes"][kern]),
                 "algorithmic_bytes_per_launch": work["bytes"][kern], "ms_per_launch": round(kern_ms, 5),
                 "peak_source": f"{pk['source']} hbm_gbs"}
     else:
