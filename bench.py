@@ -40,7 +40,7 @@ def parse():
     p.add_argument("--steps", type=int, default=200)
     p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    p.add_argument("--workload", default="decode", choices=["decode", "prefill", "zipf", "edge", "decode_e64"])
+    p.add_argument("--workload", default="decode", choices=["decode", "prefill", "zipf", "edge", "decode_e64", "vision", "dense"])
     p.add_argument("--no-secondary", action="store_true", help="skip the T=16384 Zipf measurement")
     p.add_argument("--no-cpu-baseline", action="store_true")
     return p.parse_args()
@@ -183,7 +183,7 @@ def algorithmic_work(layer, T, offsets):
     outputs once; FLOPs of the expert GEMMs only (2 * rows * N * K)."""
     sh = layer.shape
     H, F, E, K = sh.H, sh.F, sh.E, sh.K
-    rows = T * (K + 1)
+    rows = T * (K + sh.S)
     counts = np.diff(offsets)
     touched = int(np.count_nonzero(counts[:E])) + (1 if counts[E] > 0 else 0)
     gu_w = 2 * F * H + 2 * sh.FB * sh.HB * 4          # gate + up codes and scales of one expert
@@ -217,16 +217,16 @@ def load_layer(name, d, rank):
         host = None
     if d.world == 1:
         return wl, host, tu.upload_layer(host), x
-    shapes = {"w_gate": ((sh.E + 1, sh.F, sh.H), torch.uint8), "w_up": ((sh.E + 1, sh.F, sh.H), torch.uint8),
-              "w_down": ((sh.E + 1, sh.H, sh.ld_f), torch.uint8),
-              "s_gate": ((sh.E + 1, sh.FB, sh.HB), torch.float32), "s_up": ((sh.E + 1, sh.FB, sh.HB), torch.float32),
-              "s_down": ((sh.E + 1, sh.HB, sh.FB), torch.float32), "router_w": ((sh.E, sh.H), torch.float32)}
+    shapes = {"w_gate": ((sh.E + sh.S, sh.F, sh.H), torch.uint8), "w_up": ((sh.E + sh.S, sh.F, sh.H), torch.uint8),
+              "w_down": ((sh.E + sh.S, sh.H, sh.ld_f), torch.uint8),
+              "s_gate": ((sh.E + sh.S, sh.FB, sh.HB), torch.float32), "s_up": ((sh.E + sh.S, sh.FB, sh.HB), torch.float32),
+              "s_down": ((sh.E + sh.S, sh.HB, sh.FB), torch.float32), "router_w": ((sh.E, sh.H), torch.float32)}
     tens = {}
     for k, (shape, dt) in shapes.items():
         tens[k] = tu.to_device(getattr(host, k)) if rank == 0 else torch.empty(shape, dtype=dt, device="cuda")
         d.dist.broadcast(tens[k], 0)
     w = fx.LayerWeights(**tens)
-    dev = fx.MoeLayer(sh.H, sh.E, sh.K, sh.F, w, ld_h=sh.H, ld_f=sh.ld_f)
+    dev = fx.MoeLayer(sh.H, sh.E, sh.K, sh.F, w, ld_h=sh.H, ld_f=sh.ld_f, n_shared=sh.S)
     return wl, host, dev, x
 
 
@@ -242,7 +242,7 @@ class Stages:
         from fp8_expert_ffn_b200 import torch_utils as tu
         self.fx, self.dev, self.sh, self.T, self.x = fx, dev, sh, T, x
         K, E, H = sh.K, sh.E, sh.H
-        rows = T * (K + 1)
+        rows = T * (K + sh.S)
         c = "cuda"
         self.ws = tu.workspace(dev, T)
         self.idx = torch.empty((T, K), dtype=torch.int32, device=c)
@@ -397,7 +397,7 @@ def run_ours(args):
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 5), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "e4m3 (fp32 accumulate)", "data": "synthetic",
-        "config": {"workload": f"{wl.name}: {wl.note}", "T": T, "hidden": sh.H, "experts": f"{sh.E}+1",
+        "config": {"workload": f"{wl.name}: {wl.note}", "T": T, "hidden": sh.H, "experts": f"{sh.E}+{sh.S}",
                    "top_k": sh.K, "ffn": sh.F, "weights": "FP8 E4M3, 128x128 fp32 block scales, seeded synthetic",
                    "l2": "inputs larger than L2 (each step streams the touched experts' weights, GBs >> 126 MB)",
                    "parallelism": f"replicas x{world}", "touched_groups": work["touched_groups"]},

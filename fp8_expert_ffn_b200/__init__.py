@@ -123,10 +123,11 @@ class MoeLayer:
     """Owns a moe_layer_t; keeps the weight tensors alive while it exists."""
 
     def __init__(self, hidden, n_routed, top_k, ffn, weights: LayerWeights, ld_h=None, ld_f=None,
-                 routed_scaling=1.0):
+                 routed_scaling=1.0, n_shared=1):
         self.H, self.E, self.K, self.F = hidden, n_routed, top_k, ffn
         self.weights = weights
-        d = moe_layer_desc(hidden, n_routed, 1, top_k, ffn, ffn, 128, routed_scaling, 1)
+        self.S = n_shared
+        d = moe_layer_desc(hidden, n_routed, n_shared, top_k, ffn, ffn, 128, routed_scaling, 1)
         w = moe_weights(_ptr(weights.w_gate), _ptr(weights.w_up), _ptr(weights.w_down), _ptr(weights.s_gate),
                         _ptr(weights.s_up), _ptr(weights.s_down), _ptr(weights.router_w),
                         hidden if ld_h is None else ld_h, ffn if ld_f is None else ld_f)
@@ -146,7 +147,7 @@ class MoeLayer:
             pass
 
     def rows(self, T: int) -> int:
-        return T * (self.K + 1)
+        return T * (self.K + self.S)
 
 
 def moe_workspace_size(layer: MoeLayer, T: int) -> int:

@@ -38,14 +38,14 @@ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 }  // namespace
 
 bool encode_tmap(CUtensorMap* tm, bool bf16, const void* base, uint64_t inner, uint64_t rows, uint64_t depth,
-                 uint64_t ld_bytes, uint64_t depth_stride_bytes) {
+                 uint64_t ld_bytes, uint64_t depth_stride_bytes, bool force3d) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[3] = {inner, rows, depth};
   cuuint64_t strides[2] = {ld_bytes, depth_stride_bytes};
   cuuint32_t box[3] = {bf16 ? 64u : 128u, 128, 1};   // 128 bytes of K per box row
   cuuint32_t estr[3] = {1, 1, 1};
-  const cuuint32_t rank = depth > 1 ? 3 : 2;
+  const cuuint32_t rank = (depth > 1 || force3d) ? 3 : 2;
   CUresult r = fn(tm, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, rank,
                   const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -60,7 +60,7 @@ bool encode_tmap_u8(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t 
 Scratch carve(const moe_layer_s* L, int T, void* base) {
   Scratch s = {};
   const int K = L->K, E = L->E;
-  const size_t rows = size_t(T) * (K + 1);
+  const size_t rows = size_t(T) * (K + L->S);
   const size_t W = (size_t(T) + 31) / 32;
   char* b = static_cast<char*>(base);
   size_t off = 0;
@@ -136,8 +136,9 @@ moe_status moe_layer_create(const moe_layer_desc* d, const moe_weights* w, moe_l
   *out = nullptr;
   if (!d || !w) return MOE_ERR_INVALID_ARG;
   if (d->hidden <= 0 || d->n_routed <= 0 || d->top_k <= 0 || d->ffn <= 0) return MOE_ERR_INVALID_ARG;
-  if (d->hidden % 128 != 0 || d->hidden > 16384 || d->n_routed > 256 || d->n_shared != 1 || d->top_k > 8 ||
-      d->top_k > d->n_routed || d->ffn > 4096 || d->shared_ffn != d->ffn || d->block != 128 || d->norm_topk != 1)
+  if (d->hidden % 128 != 0 || d->hidden > 16384 || d->n_routed > 256 || d->n_shared < 0 || d->n_shared > 1 ||
+      d->top_k > 8 || d->top_k > d->n_routed || d->ffn > 16384 || (d->n_shared == 1 && d->shared_ffn != d->ffn) ||
+      d->block != 128 || d->norm_topk != 1)
     return MOE_ERR_UNSUPPORTED;
   if (!(d->routed_scaling == d->routed_scaling)) return MOE_ERR_INVALID_ARG;
   if (!w->w_gate || !w->w_up || !w->w_down || !w->s_gate || !w->s_up || !w->s_down || !w->router_w)
@@ -161,16 +162,18 @@ moe_status moe_layer_create(const moe_layer_desc* d, const moe_weights* w, moe_l
   L->H = d->hidden;
   L->E = d->n_routed;
   L->K = d->top_k;
+  L->S = d->n_shared;
   L->F = d->ffn;
   L->HB = d->hidden / 128;
   L->FB = (d->ffn + 127) / 128;
   L->ld_hh = L->FB * 128;
   L->device = dev;
   L->num_sms = prop.multiProcessorCount;
-  const uint64_t E1 = uint64_t(L->E) + 1;
-  if (!encode_tmap_u8(&L->tm_gate, w->w_gate, L->H, L->F, E1, w->ld_h, uint64_t(L->F) * w->ld_h) ||
-      !encode_tmap_u8(&L->tm_up, w->w_up, L->H, L->F, E1, w->ld_h, uint64_t(L->F) * w->ld_h) ||
-      !encode_tmap_u8(&L->tm_down, w->w_down, L->F, L->H, E1, w->ld_f, uint64_t(L->H) * w->ld_f)) {
+  // weight maps are always 3-D (expert index = z), even with a single expert
+  const uint64_t E1 = uint64_t(L->E) + L->S;
+  if (!encode_tmap(&L->tm_gate, false, w->w_gate, L->H, L->F, E1, w->ld_h, uint64_t(L->F) * w->ld_h, true) ||
+      !encode_tmap(&L->tm_up, false, w->w_up, L->H, L->F, E1, w->ld_h, uint64_t(L->F) * w->ld_h, true) ||
+      !encode_tmap(&L->tm_down, false, w->w_down, L->F, L->H, E1, w->ld_f, uint64_t(L->H) * w->ld_f, true)) {
     delete L;
     return MOE_ERR_CUDA;
   }

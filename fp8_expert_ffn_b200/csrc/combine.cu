@@ -20,7 +20,7 @@ constexpr int CB_THREADS = 128;
 // 8-channel (16-byte) piece and loads its K+1 rows at once.
 __global__ void __launch_bounds__(CB_THREADS) combine_kernel(const uint16_t* __restrict__ y,
                                                              const int32_t* __restrict__ inv,
-                                                             const float* __restrict__ w, int T, int K, int H,
+                                                             const float* __restrict__ w, int T, int K, int S, int H,
                                                              uint16_t* __restrict__ out, int ldo) {
   const int t = blockIdx.x;
   __shared__ int s_row[9];
@@ -39,7 +39,7 @@ __global__ void __launch_bounds__(CB_THREADS) combine_kernel(const uint16_t* __r
       const int r = k < K ? s_row[k] : -1;
       raws[k] = r >= 0 ? *reinterpret_cast<const uint4*>(y + size_t(r) * H + c) : make_uint4(0, 0, 0, 0);
     }
-    const uint4 raw_shared = *reinterpret_cast<const uint4*>(y + shared_row * H + c);
+    const uint4 raw_shared = S ? *reinterpret_cast<const uint4*>(y + shared_row * H + c) : make_uint4(0, 0, 0, 0);
     float acc[8] = {};
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
@@ -70,7 +70,7 @@ __global__ void __launch_bounds__(CB_THREADS) combine_kernel(const uint16_t* __r
 cudaError_t launch_combine(const moe_layer_s* L, const uint16_t* y, const int32_t* inv, const float* w, int T,
                            uint16_t* out, int ldo, cudaStream_t st) {
   dim3 grid(T, (L->H + CB_THREADS * 8 - 1) / (CB_THREADS * 8));
-  combine_kernel<<<grid, CB_THREADS, 0, st>>>(y, inv, w, T, L->K, L->H, out, ldo);
+  combine_kernel<<<grid, CB_THREADS, 0, st>>>(y, inv, w, T, L->K, L->S, L->H, out, ldo);
   return cudaGetLastError();
 }
 

@@ -511,7 +511,7 @@ static GemmArgs down_args(const moe_layer_s* L, const int32_t* offsets, int rows
 
 cudaError_t launch_gate_up(const moe_layer_s* L, const uint8_t* xq, const float* xs, const int32_t* offsets, int T,
                            uint8_t* h, float* hs, cudaStream_t st) {
-  const int rows = T * (L->K + 1);
+  const int rows = T * (L->K + L->S);
   CUtensorMap tmX;
   if (!encode_tmap_u8(&tmX, xq, L->H, rows, 1, L->H, 0)) return cudaErrorInvalidValue;
   GemmArgs a = gateup_args(L, offsets, rows, xs);
@@ -523,7 +523,7 @@ cudaError_t launch_gate_up(const moe_layer_s* L, const uint8_t* xq, const float*
 
 cudaError_t launch_down(const moe_layer_s* L, const uint8_t* h, const float* hs, const int32_t* offsets, int T,
                         uint16_t* y, cudaStream_t st) {
-  const int rows = T * (L->K + 1);
+  const int rows = T * (L->K + L->S);
   CUtensorMap tmH;
   if (!encode_tmap_u8(&tmH, h, L->F, rows, 1, L->ld_hh, 0)) return cudaErrorInvalidValue;
   GemmArgs a = down_args(L, offsets, rows, hs);
@@ -534,7 +534,7 @@ cudaError_t launch_down(const moe_layer_s* L, const uint8_t* h, const float* hs,
 
 cudaError_t launch_test_gemm_f32(const moe_layer_s* L, int which, const uint8_t* a_ptr, const float* as,
                                  const int32_t* offsets, int T, float* out, cudaStream_t st) {
-  const int rows = T * (L->K + 1);
+  const int rows = T * (L->K + L->S);
   CUtensorMap tmA;
   if (which == 0) {
     if (!encode_tmap_u8(&tmA, a_ptr, L->H, rows, 1, L->H, 0)) return cudaErrorInvalidValue;

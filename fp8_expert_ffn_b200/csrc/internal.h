@@ -13,6 +13,7 @@ struct moe_layer_s {
   moe_layer_desc d;
   moe_weights w;
   int H, E, K, F;
+  int S;         // shared experts (0 or 1); a token fills K + S rows
   int HB;        // H / 128
   int FB;        // ceil(F / 128)
   int ld_hh;     // row stride of the quantised SwiGLU output h: FB * 128
@@ -80,7 +81,7 @@ bool encode_tmap_u8(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t 
                     uint64_t ld, uint64_t depth_stride);
 // Same for bf16 (box 64 x 128 elements = 128 bytes of K per row) or u8.
 bool encode_tmap(CUtensorMap* tm, bool bf16, const void* base, uint64_t inner, uint64_t rows, uint64_t depth,
-                 uint64_t ld_bytes, uint64_t depth_stride_bytes);
+                 uint64_t ld_bytes, uint64_t depth_stride_bytes, bool force3d = false);
 
 // Router weight split into three bf16 terms (hi + mid + lo == w exactly for
 // normal-range fp32 w), [3][E][H]; written once at layer creation.

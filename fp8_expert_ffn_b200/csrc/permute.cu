@@ -77,7 +77,7 @@ __global__ void __launch_bounds__(256) permute_count_kernel(const uint32_t* __re
 
 // offsets[g] = sum of counts[0..g), offsets[E+1] = offsets[E] + T.
 __global__ void __launch_bounds__(256) permute_offsets_kernel(const int32_t* __restrict__ counts, int E, int T,
-                                                              int32_t* __restrict__ offsets) {
+                                                              int S, int32_t* __restrict__ offsets) {
   __shared__ int32_t warp_sums[8];
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   const int v = tid < E ? counts[tid] : 0;
@@ -94,7 +94,7 @@ __global__ void __launch_bounds__(256) permute_offsets_kernel(const int32_t* __r
   if (tid < E) offsets[tid] = base + incl - v;
   if (tid == E - 1) {
     offsets[E] = base + incl;
-    offsets[E + 1] = base + incl + T;
+    offsets[E + 1] = base + incl + T * S;
   }
 }
 
@@ -105,7 +105,7 @@ constexpr int GATHER_GROUPS = 8;   // 128-channel groups per warp
 __global__ void __launch_bounds__(256) permute_gather_kernel(
     const uint16_t* __restrict__ x, int T, int ldx, int H, const int32_t* __restrict__ idx, int K, int E, int W,
     const uint32_t* __restrict__ bitmap, const uint32_t* __restrict__ wprefix, const int32_t* __restrict__ offsets,
-    int rows, int32_t* __restrict__ perm, int32_t* __restrict__ inv, uint8_t* __restrict__ xq,
+    int S, int rows, int32_t* __restrict__ perm, int32_t* __restrict__ inv, uint8_t* __restrict__ xq,
     float* __restrict__ xs) {
   const int lane = threadIdx.x & 31;
   const int HB = H / 128;
@@ -131,7 +131,7 @@ __global__ void __launch_bounds__(256) permute_gather_kernel(
       my_row = offsets[e] + int(wprefix[size_t(e) * W + (t >> 5)]) + __popc(word & ((1u << (t & 31)) - 1u));
     }
     if (chunk == 0) inv[size_t(t) * K + lane] = my_row;
-  } else if (lane == K) {
+  } else if (lane == K && S) {
     my_row = offsets[E] + t;
   }
   if (chunk == 0 && my_row >= 0) perm[my_row] = t;
@@ -175,19 +175,20 @@ cudaError_t launch_permute(const moe_layer_s* L, const uint16_t* x, int T, int l
                            int32_t* offsets, int32_t* perm, int32_t* inv, uint8_t* xq, float* xs,
                            const Scratch& s, cudaStream_t st) {
   const int K = L->K, E = L->E, W = (T + 31) / 32;
-  const int rows = T * (K + 1);
+  const int S = L->S;
+  const int rows = T * (K + S);
   cudaError_t e = cudaMemsetAsync(s.bitmap, 0, sizeof(uint32_t) * size_t(E) * W, st);
   if (e != cudaSuccess) return e;
   permute_bitmap_kernel<<<(T * K + 255) / 256, 256, 0, st>>>(idx, T, K, E, W, s.bitmap, L->status);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   permute_count_kernel<<<E, 256, 0, st>>>(s.bitmap, W, s.wprefix, s.counts);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  permute_offsets_kernel<<<1, 256, 0, st>>>(s.counts, E, T, offsets);
+  permute_offsets_kernel<<<1, 256, 0, st>>>(s.counts, E, T, S, offsets);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   const int nchunk = (L->HB + GATHER_GROUPS - 1) / GATHER_GROUPS;
   const long long warps = static_cast<long long>(T) * nchunk;
   permute_gather_kernel<<<unsigned((warps + 7) / 8), 256, 0, st>>>(x, T, ldx, L->H, idx, K, E, W, s.bitmap,
-                                                                   s.wprefix, offsets, rows, perm, inv, xq, xs);
+                                                                   s.wprefix, offsets, S, rows, perm, inv, xq, xs);
   return cudaGetLastError();
 }
 

@@ -37,7 +37,7 @@ def upload_layer(host, device="cuda", routed_scaling=1.0, share_experts: MoeLaye
             s_up=to_device(host.s_up, device), s_down=to_device(host.s_down, device),
             router_w=to_device(host.router_w, device))
     return MoeLayer(sh.H, sh.E, sh.K, sh.F, w, ld_h=host.w_gate.shape[2], ld_f=host.w_down.shape[2],
-                    routed_scaling=routed_scaling)
+                    routed_scaling=routed_scaling, n_shared=getattr(sh, "S", 1))
 
 
 def workspace(layer: MoeLayer, T: int, device="cuda") -> torch.Tensor:

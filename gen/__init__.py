@@ -146,6 +146,7 @@ class LayerShape:
     K: int          # experts per token
     F: int          # expert FFN width (routed and shared)
     ld_f: int       # row stride (bytes) of the down-projection codes, >= F, multiple of 16
+    S: int = 1      # shared experts (0 or 1); the shared expert is index E
 
     @property
     def FB(self) -> int:
@@ -195,6 +196,15 @@ WORKLOADS = {
                      note="T=4099 (ragged)"),
     "edge_f1500": Workload("edge_f1500", 4099, DOTS3_F1500, x_seed=4, w_seed=2, outliers=8,
                            note="T=4099 on the FFN=1500 variant (partial 128x128 blocks)"),
+    # vision MoE of the ViT encoder (Dots3NoteVisionConfig: hidden_size 1536,
+    # num_local_experts 64, moe_intermediate_size 2112 = 16.5 x 128, no
+    # shared expert; top-k unstated, read as 2)
+    "vision": Workload("vision", 4096, LayerShape(H=1536, E=64, K=2, F=2112, ld_f=2112, S=0), x_seed=6, w_seed=4,
+                       note="T=4096 patch tokens, vision MoE: hidden 1536, 64 experts, top-2, FFN 2112, no shared"),
+    # the dense FFN layer of the language model (Dots3NoteTextConfig
+    # intermediate_size 13824 = 108 x 128) as a one-expert, top-1 layer
+    "dense": Workload("dense", 64, LayerShape(H=5120, E=1, K=1, F=13824, ld_f=13824, S=0), x_seed=7, w_seed=5,
+                      outliers=8, note="T=64, dense FP8 FFN 5120 -> 2 x 13824 -> 5120 (one expert, weight 1)"),
     # a smaller decode-shaped case (64 routed experts, 1.5 GB of weights) for
     # profiler captures that must stay a few GB on the device
     "decode_e64": Workload("decode_e64", 16, LayerShape(H=5120, E=64, K=8, F=1536, ld_f=1536), x_seed=5,
@@ -219,9 +229,10 @@ class Layer:
 def make_experts(shape: LayerShape, w_seed: int, nthreads: int = 0):
     """Expert checkpoint (gate, up, down codes and block scales) of one layer."""
     H, E, F = shape.H, shape.E, shape.F
-    wg, sg = fp8_blocks(w_seed, STREAM_GATE, E + 1, F, H, H, 1.0 / math.sqrt(H), nthreads)
-    wu, su = fp8_blocks(w_seed, STREAM_UP, E + 1, F, H, H, 1.0 / math.sqrt(H), nthreads)
-    wd, sd = fp8_blocks(w_seed, STREAM_DOWN, E + 1, H, F, shape.ld_f, 1.0 / math.sqrt(F), nthreads)
+    n = E + shape.S
+    wg, sg = fp8_blocks(w_seed, STREAM_GATE, n, F, H, H, 1.0 / math.sqrt(H), nthreads)
+    wu, su = fp8_blocks(w_seed, STREAM_UP, n, F, H, H, 1.0 / math.sqrt(H), nthreads)
+    wd, sd = fp8_blocks(w_seed, STREAM_DOWN, n, H, F, shape.ld_f, 1.0 / math.sqrt(F), nthreads)
     return wg, sg, wu, su, wd, sd
 
 

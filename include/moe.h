@@ -44,7 +44,9 @@
  *     layer's device status word, skip the offending work and are read back
  *     with moe_get_device_status.
  *
- * Row count: R = T*K routed rows plus T shared rows, rows = T*(K+1).
+ * Row count: R = T*K routed rows plus T*S shared rows (S = n_shared, 0 or 1),
+ * rows = T*(K+S). A layer with n_shared = 0 has no group-E rows; one with
+ * n_routed = 1, top_k = 1, n_shared = 0 is a dense FP8 FFN (weight 1).
  */
 #ifndef FP8_EXPERT_FFN_MOE_H
 #define FP8_EXPERT_FFN_MOE_H
@@ -71,29 +73,29 @@ typedef enum {
  * num_experts_per_tok, moe_intermediate_size, shared_experts_intermediate_size,
  * routed_scaling_factor, norm_topk_prob; block = the 128 x 128 weight block
  * edge of transformers PR #47844. This build requires: hidden % 128 == 0,
- * 128 <= hidden <= 16384, 1 <= n_routed <= 256, n_shared == 1,
- * 1 <= top_k <= min(8, n_routed), 1 <= ffn <= 4096, shared_ffn == ffn,
+ * 128 <= hidden <= 16384, 1 <= n_routed <= 256, n_shared 0 or 1,
+ * 1 <= top_k <= min(8, n_routed), 1 <= ffn <= 16384, shared_ffn == ffn when n_shared = 1,
  * block == 128, norm_topk == 1; otherwise MOE_ERR_UNSUPPORTED. */
 typedef struct {
   int hidden;           /* H */
   int n_routed;         /* E */
-  int n_shared;         /* must be 1 */
+  int n_shared;         /* S: 0 or 1 */
   int top_k;            /* K */
   int ffn;              /* F */
-  int shared_ffn;       /* must equal ffn */
+  int shared_ffn;       /* must equal ffn when n_shared = 1 */
   int block;            /* must be 128 */
   float routed_scaling; /* multiplies the renormalised routed weights */
   int norm_topk;        /* must be 1 */
 } moe_layer_desc;
 
 /* Caller-owned device weights; they must outlive the layer handle. Expert
- * index E is the shared expert. Codes are E4M3 bytes; scales are fp32
- * dequantisation multipliers, one per 128 x 128 block (edge blocks cover the
- * real rows/columns only):
- *   w_gate, w_up : [E+1][F][ld_h]   bytes, ld_h >= H, ld_h % 16 == 0
- *   s_gate, s_up : [E+1][ceil(F/128)][H/128]
- *   w_down       : [E+1][H][ld_f]   bytes, ld_f >= F, ld_f % 16 == 0
- *   s_down       : [E+1][H/128][ceil(F/128)]
+ * index E is the shared expert (present when n_shared = 1; S = n_shared).
+ * Codes are E4M3 bytes; scales are fp32 dequantisation multipliers, one per
+ * 128 x 128 block (edge blocks cover the real rows/columns only):
+ *   w_gate, w_up : [E+S][F][ld_h]   bytes, ld_h >= H, ld_h % 16 == 0
+ *   s_gate, s_up : [E+S][ceil(F/128)][H/128]
+ *   w_down       : [E+S][H][ld_f]   bytes, ld_f >= F, ld_f % 16 == 0
+ *   s_down       : [E+S][H/128][ceil(F/128)]
  *   router_w     : [E][H] fp32, row-major                                  */
 typedef struct {
   const uint8_t* w_gate;
@@ -141,7 +143,8 @@ moe_status moe_route(moe_layer_t layer, const uint16_t* x, int T, int ldx, int32
 
 /* Token permutation by expert with fused activation quantisation.
  * Counting sort of the T*K (token, slot) pairs by expert id, stable in token
- * order; group E (shared expert) holds rows [T*K, T*K+T) in token order.
+ * order; with n_shared = 1, group E (shared expert) holds rows [T*K, T*K+T)
+ * in token order (with n_shared = 0 it is empty).
  *   topk_idx  [T][K] int32 (in); ids outside [0,E) or repeated within a
  *             token set MOE_ERR_DEVICE and are skipped
  *   offsets   [E+2] int32 (out): group g is rows [offsets[g], offsets[g+1])
@@ -200,8 +203,8 @@ moe_status moe_gate_up(moe_layer_t layer, const uint8_t* xq, const float* xs, co
 moe_status moe_down(moe_layer_t layer, const uint8_t* h, const float* hs, const int32_t* offsets, int T,
                     uint16_t* y, void* stream);
 
-/* out[t] = bf16_RNE( sum_k topk_w[t,k] * y[inv[t,k]] + y[T*K + t] ), FP32
- * sum in slot order, shared row last.
+/* out[t] = bf16_RNE( sum_k topk_w[t,k] * y[inv[t,k]] + S * y[T*K + t] ), FP32
+ * sum in slot order, shared row (when n_shared = 1) last.
  *   out [T][ldo] bf16, ldo >= H                                            */
 moe_status moe_combine(moe_layer_t layer, const uint16_t* y, const int32_t* inv, const float* topk_w, int T,
                        uint16_t* out, int ldo, void* stream);
@@ -224,7 +227,7 @@ moe_status moe_get_device_status(moe_layer_t layer, void* stream, uint32_t* deta
  *              [256c+128, 256c+256)
  *   which = 1: down GEMM; a = h [rows][ceil(F/128)*128] (bytes beyond F are
  *              ignored), as = [ceil(F/128)][rows]; out [rows][H] fp32
- * offsets gives the groups as in moe_permute; rows = T*(K+1). */
+ * offsets gives the groups as in moe_permute; rows = T*(K+S). */
 moe_status moe_test_grouped_gemm_f32(moe_layer_t layer, int which, const uint8_t* a, const float* as,
                                      const int32_t* offsets, int T, float* out, void* stream);
 

@@ -176,23 +176,24 @@ class Perm:
     inv: np.ndarray      # int32 [T, K]; (token, slot) -> row
 
 
-def permute(idx: np.ndarray, E: int) -> Perm:
-    """Counting sort of (token, slot) pairs by expert, stable in token order."""
+def permute(idx: np.ndarray, E: int, S: int = 1) -> Perm:
+    """Counting sort of (token, slot) pairs by expert, stable in token order;
+    with S = 1 the shared expert's group E holds one row per token."""
     idx = np.asarray(idx)
     T, K = idx.shape
     R = T * K
     counts = np.bincount(idx.reshape(-1), minlength=E)[:E]
     offsets = np.zeros(E + 2, np.int64)
     offsets[1:E + 1] = np.cumsum(counts)
-    offsets[E + 1] = offsets[E] + T
+    offsets[E + 1] = offsets[E] + T * S
     flat = idx.reshape(-1)
     order = np.argsort(flat, kind="stable")     # (t, k) pairs grouped by expert, token order kept
     rows = np.empty(R, np.int64)
     rows[order] = np.arange(R)
     inv = rows.reshape(T, K)
-    perm = np.empty(R + T, np.int64)
+    perm = np.empty(R + T * S, np.int64)
     perm[rows] = np.arange(R) // K
-    perm[R:] = np.arange(T)
+    perm[R:] = np.arange(T * S) % max(T, 1)
     return Perm(offsets.astype(np.int32), perm.astype(np.int32), inv.astype(np.int32))
 
 
@@ -266,15 +267,15 @@ def expert_down_rows(hq, hs, offsets, layer, groups=None):
     return y
 
 
-def combine(y: np.ndarray, inv: np.ndarray, w: np.ndarray) -> np.ndarray:
-    """out[t] = sum_k w[t,k] * y[inv[t,k]] + y[R + t] (shared expert, weight 1)."""
+def combine(y: np.ndarray, inv: np.ndarray, w: np.ndarray, S: int = 1) -> np.ndarray:
+    """out[t] = sum_k w[t,k] * y[inv[t,k]] + y[R + t] (shared expert, weight 1, when S = 1)."""
     inv = np.asarray(inv)
     T, K = inv.shape
     R = T * K
     out = np.zeros((T, y.shape[1]), np.float64)
     for k in range(K):
         out += np.asarray(w, np.float64)[:, k:k + 1] * y[inv[:, k]]
-    return out + y[R:R + T]
+    return out + y[R:R + T] if S else out
 
 
 def quantize_tokens(x_bits: np.ndarray):
@@ -289,12 +290,12 @@ def gather_rows(tok_codes, tok_scales, perm):
 def layer_forward(x_bits: np.ndarray, layer) -> dict:
     """Whole layer: route -> permute -> quantise/gather -> expert FFNs -> combine."""
     sh = layer.shape
-    r = route(x_bits, layer.router_w, sh.K)
-    p = permute(r.idx, sh.E)
+    r = route(x_bits, layer.router_w, sh.K, getattr(layer, "routed_scaling", 1.0))
+    p = permute(r.idx, sh.E, sh.S)
     tq, ts = quantize_tokens(x_bits)
     xq, xs = gather_rows(tq, ts, p.perm)
     f = expert_ffn_rows(xq, xs, p.offsets, layer)
-    out = combine(f["y"], p.inv, r.w)
+    out = combine(f["y"], p.inv, r.w, sh.S)
     return {"route": r, "perm": p, "xq": xq, "xs": xs, **f, "out": out}
 
 
@@ -307,7 +308,7 @@ def token_outputs(x_bits: np.ndarray, layer, tokens, idx=None, w=None) -> np.nda
     tokens = np.asarray(tokens)
     xb = np.asarray(x_bits)[tokens]
     if idx is None:
-        r = route(xb, layer.router_w, sh.K)
+        r = route(xb, layer.router_w, sh.K, getattr(layer, "routed_scaling", 1.0))
         idx_s, w_s = r.idx, r.w
     else:
         idx_s, w_s = np.asarray(idx)[tokens], np.asarray(w, np.float64)[tokens]
@@ -319,8 +320,8 @@ def token_outputs(x_bits: np.ndarray, layer, tokens, idx=None, w=None) -> np.nda
     for i in range(n):
         for k in range(sh.K):
             users.setdefault(int(idx_s[i, k]), []).append((i, float(w_s[i, k])))
-    users.setdefault(sh.E, [])
-    users[sh.E] = [(i, 1.0) for i in range(n)]
+    if sh.S:
+        users[sh.E] = [(i, 1.0) for i in range(n)]
     def one(item):
         g, lst = item
         rows = np.array([i for i, _ in lst])
@@ -344,7 +345,7 @@ def layer_forward_bf16(x_bits: np.ndarray, layer, tokens=None, idx=None, w=None)
     tokens = np.arange(T) if tokens is None else np.asarray(tokens)
     xb = np.asarray(x_bits)[tokens]
     if idx is None:
-        r = route(xb, layer.router_w, sh.K)
+        r = route(xb, layer.router_w, sh.K, getattr(layer, "routed_scaling", 1.0))
         idx_s, w_s = r.idx, r.w
     else:
         idx_s, w_s = np.asarray(idx)[tokens], np.asarray(w, np.float64)[tokens]
@@ -354,7 +355,8 @@ def layer_forward_bf16(x_bits: np.ndarray, layer, tokens=None, idx=None, w=None)
     for i in range(len(tokens)):
         for k in range(sh.K):
             users.setdefault(int(idx_s[i, k]), []).append((i, float(w_s[i, k])))
-    users[sh.E] = [(i, 1.0) for i in range(len(tokens))]
+    if sh.S:
+        users[sh.E] = [(i, 1.0) for i in range(len(tokens))]
     def one(item):
         g, lst = item
         rows = np.array([i for i, _ in lst])

@@ -28,7 +28,7 @@ class Case:
         self.x_bits = x_bits
         self.dev = device_layer if device_layer is not None else tu.upload_layer(host_layer)
         T, K, E, H = self.T, sh.K, sh.E, sh.H
-        rows = T * (K + 1)
+        rows = T * (K + sh.S)
         self.rows = rows
         d = "cuda"
         self.x = tu.bf16_tensor(x_bits)
@@ -67,9 +67,9 @@ def bf16_f64(bits):
     return moe.bf16_to_f64(bits)
 
 
-def rows_of_tokens(inv: np.ndarray, T: int, K: int, tokens) -> np.ndarray:
+def rows_of_tokens(inv: np.ndarray, T: int, K: int, tokens, S: int = 1) -> np.ndarray:
     tokens = np.asarray(tokens)
-    return np.concatenate([inv[tokens].ravel(), T * K + tokens])
+    return np.concatenate([inv[tokens].ravel(), T * K + tokens]) if S else inv[tokens].ravel()
 
 
 def oracle_ffn_on_rows(layer, rows, xq, xs_rows_major, offsets):

@@ -45,8 +45,8 @@ def get_case(name):
 
 _device_layers = {}
 
-FULL = ["toy", "decode"]                    # every token / row checked
-SAMPLED = ["prefill", "zipf", "edge", "edge_f1500"]
+FULL = ["toy", "decode", "dense"]           # every token / row checked
+SAMPLED = ["prefill", "zipf", "edge", "edge_f1500", "vision"]
 ALL = FULL + SAMPLED
 
 
@@ -80,7 +80,7 @@ def test_route(name):
 def test_permute(name):
     wl, layer, c = get_case(name)
     sh, T = layer.shape, c.T
-    p = moe.permute(c.np("idx"), sh.E)
+    p = moe.permute(c.np("idx"), sh.E, sh.S)
     assert np.array_equal(c.np("offsets"), p.offsets)
     assert np.array_equal(c.np("perm"), p.perm)
     assert np.array_equal(c.np("inv"), p.inv)
@@ -100,7 +100,7 @@ def test_expert_ffn(name):
     wl, layer, c = get_case(name)
     sh, T = layer.shape, c.T
     toks = np.arange(T) if name in FULL else token_sample(T, 40)
-    rows = np.unique(gc.rows_of_tokens(c.np("inv"), T, sh.K, toks))
+    rows = np.unique(gc.rows_of_tokens(c.np("inv"), T, sh.K, toks, sh.S))
     off = c.np("offsets")
     xq = c.xq[torch.from_numpy(rows).cuda()].cpu().numpy()
     xs = c.np("xs")[:, rows].T.copy()
@@ -135,7 +135,7 @@ def test_combine(name):
     T = c.T
     toks = np.arange(T) if name in FULL else token_sample(T, 2048)
     y = moe.bf16_to_f64(tu.bf16_bits(c.y))
-    ref = moe.combine(y, c.np("inv"), c.np("w").astype(np.float64))[toks]
+    ref = moe.combine(y, c.np("inv"), c.np("w").astype(np.float64), layer.shape.S)[toks]
     out = moe.bf16_to_f64(c.np("out"))[toks]
     rms = np.sqrt(np.mean(ref ** 2))
     assert np.all(np.abs(out - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-5 * rms)
@@ -381,3 +381,30 @@ def test_forward_is_deterministic():
         fx.moe_layer_forward(c.dev, c.x, c.T, layer.shape.H, o, layer.shape.H, ws, ws.numel())
         outs.append(o)
     assert torch.equal(outs[0].view(torch.int16), outs[1].view(torch.int16))
+
+
+def test_routed_scaling_factor():
+    """routed_scaling_factor != 1 (Dots3NoteTextConfig field; the vision
+    router's router_scaling_factor plays the same part): the K weights sum to
+    the factor and the output follows the oracle with the same factor."""
+    wl, layer0, x = gen.workload_inputs("toy")
+    sh = layer0.shape
+    layer = gen.Layer(sh, layer0.router_w, layer0.w_gate, layer0.s_gate, layer0.w_up, layer0.s_up, layer0.w_down,
+                      layer0.s_down)
+    layer.routed_scaling = 2.5
+    dev = tu.upload_layer(layer, routed_scaling=2.5)
+    c = gc.Case(layer, x, dev)
+    assert np.allclose(c.np("w").sum(1), 2.5, atol=1e-5)
+    ref = moe.layer_forward(x, layer)
+    keep = ~ref["route"].near_tie
+    gc.assert_output_close(moe.bf16_to_f64(c.np("out"))[keep], ref["out"][keep], "routed_scaling 2.5")
+
+
+def test_dense_ffn_is_the_single_expert():
+    """The dense FFN workload (one expert, top-1, no shared expert): every
+    token is routed to expert 0 with weight exactly 1 and the output is that
+    expert's FFN rounded once to bf16 (combine of a single row)."""
+    wl, layer, c = get_case("dense")
+    assert not c.np("idx").any() and np.all(c.np("w") == 1.0)
+    assert np.array_equal(c.np("perm"), np.arange(c.T)) and np.array_equal(c.np("inv").ravel(), np.arange(c.T))
+    assert np.array_equal(tu.bf16_bits(c.y), c.np("out"))

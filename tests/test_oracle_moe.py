@@ -333,3 +333,34 @@ def test_bf16_checkpoint_cross_check(toy):
     b = moe.layer_forward_bf16(x, layer)
     rel = np.linalg.norm(a - b) / np.linalg.norm(b)
     assert 1e-4 < rel < 8e-2
+
+
+def test_no_shared_expert_and_single_expert_layer():
+    """S = 0: no shared rows; E = 1, K = 1: the layer is that expert's FFN."""
+    rng = np.random.default_rng(12)
+    idx = np.sort(np.array([rng.choice(8, 2, replace=False) for _ in range(10)]), axis=1)
+    p = moe.permute(idx, 8, S=0)
+    assert p.offsets[8] == p.offsets[9] == 20 and len(p.perm) == 20
+    y = rng.standard_normal((20, 3))
+    w = rng.uniform(size=(10, 2))
+    out = moe.combine(y, p.inv, w, S=0)
+    assert np.array_equal(out, sum(w[:, k:k + 1] * y[p.inv[:, k]] for k in range(2)))
+    sh = gen.LayerShape(H=256, E=1, K=1, F=200, ld_f=208, S=0)
+    layer = gen.make_layer(sh, 9)
+    assert layer.w_gate.shape[0] == 1
+    x = gen.make_x(5, 256, 2)
+    r = moe.layer_forward(x, layer)
+    assert np.all(r["route"].idx == 0) and np.all(r["route"].w == 1.0)
+    xf = moe.bf16_to_f64(x)
+    for t in range(5):
+        ref = textbook_ffn(xf[t], layer.w_gate[0], layer.s_gate[0], layer.w_up[0], layer.s_up[0],
+                           layer.w_down[0], layer.s_down[0], sh.F, sh.H)
+        assert np.allclose(r["out"][t], ref, rtol=1e-11, atol=1e-11 * np.abs(ref).max())
+
+
+def test_routed_scaling_in_oracle():
+    sh = gen.TOY
+    x = gen.make_x(6, sh.H, 1)
+    r1 = moe.route(x, gen.make_router(sh, 0), sh.K)
+    r2 = moe.route(x, gen.make_router(sh, 0), sh.K, routed_scaling=2.5)
+    assert np.array_equal(r1.idx, r2.idx) and np.allclose(r2.w, 2.5 * r1.w, rtol=1e-15)
