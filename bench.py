@@ -472,7 +472,7 @@ def run_reference(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": f"{wl.name}: {wl.note}", "T": wl.T, "hidden": wl.shape.H,
-                       "experts": f"{wl.shape.E}+1", "top_k": wl.shape.K, "ffn": wl.shape.F},
+                       "experts": f"{wl.shape.E}+{wl.shape.S}", "top_k": wl.shape.K, "ffn": wl.shape.F},
             "cpu_baseline": {"value": round(value, 4), "unit": "tokens/s", "kind": "oracle", "cores": moe.WORKERS,
                              "sample": f"{per_step} token per step through the whole layer (FP64 oracle)"},
             "e2e": {"value": round(value, 4), "unit": "tokens/s", "h2d_bytes_per_step": 0,
