@@ -40,7 +40,7 @@ def parse():
     p.add_argument("--steps", type=int, default=200)
     p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    p.add_argument("--workload", default="decode", choices=["decode", "prefill", "zipf", "edge", "decode_e64", "vision", "dense"])
+    p.add_argument("--workload", default="decode", choices=["decode", "prefill", "zipf", "edge", "decode_e64", "prefill_e32", "vision", "dense"])
     p.add_argument("--no-secondary", action="store_true", help="skip the T=16384 Zipf measurement")
     p.add_argument("--no-cpu-baseline", action="store_true")
     return p.parse_args()

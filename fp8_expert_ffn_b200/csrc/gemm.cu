@@ -69,7 +69,10 @@ constexpr int MCHUNK = 8;                  // row tiles per chunk of the tile or
 constexpr int MAX_GROUPS = 257;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t IDESC = idesc_e4m3_f32(BM, BN);
-constexpr int SMEM_DYN = STAGES * STAGE_BYTES + 1024;
+// down epilogue: each warp stages 32 rows x 64 bf16 columns (4 KB, the
+// 128-byte-swizzled box of one bulk tensor store) in shared memory
+constexpr int STG_WARP_BYTES = 32 * 128;
+constexpr int smem_dyn(int mode) { return STAGES * STAGE_BYTES + 1024 + (mode == 1 ? EPI_WARPS * STG_WARP_BYTES : 0); }
 
 enum { MODE_GATEUP = 0, MODE_DOWN = 1 };
 enum { EPI_FUSED = 0, EPI_F32 = 1 };
@@ -99,7 +102,8 @@ struct TileInfo {
   int g, nt, row0, nvalid;
 };
 
-__device__ __forceinline__ TileInfo decode_tile(int i, const int* s_prefix, const int* s_off, int ngroups, int ntn) {
+__device__ __forceinline__ TileInfo decode_tile(int i, const int* s_prefix, const int* __restrict__ off, int ngroups,
+                                                int ntn) {
   int lo = 0, hi = ngroups - 1;
   while (lo < hi) {  // last group whose prefix is <= i
     const int mid = (lo + hi + 1) >> 1;
@@ -108,7 +112,8 @@ __device__ __forceinline__ TileInfo decode_tile(int i, const int* s_prefix, cons
   TileInfo t;
   t.g = lo;
   const int local = i - s_prefix[lo];
-  const int n_g = s_off[lo + 1] - s_off[lo];
+  const int g0 = __ldg(off + lo);
+  const int n_g = __ldg(off + lo + 1) - g0;
   const int mt = (n_g + BM - 1) / BM;
   const int per_chunk = MCHUNK * ntn;
   const int chunk = local / per_chunk;
@@ -116,7 +121,7 @@ __device__ __forceinline__ TileInfo decode_tile(int i, const int* s_prefix, cons
   const int mc = min(MCHUNK, mt - chunk * MCHUNK);
   t.nt = within / mc;
   const int m = chunk * MCHUNK + (within - t.nt * mc);
-  t.row0 = s_off[lo] + m * BM;
+  t.row0 = g0 + m * BM;
   t.nvalid = min(BM, n_g - m * BM);
   return t;
 }
@@ -130,7 +135,8 @@ __device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity, 
 template <int MODE, int EPI>
 __global__ void __launch_bounds__(THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
-                        const __grid_constant__ CUtensorMap tmB1, const GemmArgs p) {
+                        const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmY,
+                        const GemmArgs p) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[STAGES];
   __shared__ __align__(8) uint64_t empty_bar[STAGES];
@@ -139,7 +145,6 @@ __global__ void __launch_bounds__(THREADS, 1)
   __shared__ __align__(8) uint64_t amax_bar[2];
   __shared__ __align__(8) uint64_t done_bar;
   __shared__ uint32_t tmem_base_s;
-  __shared__ int s_off[MAX_GROUPS + 1];
   __shared__ int s_prefix[MAX_GROUPS + 1];
   __shared__ float s_amax[2][2][BM];
   __shared__ int s_abort_store;
@@ -155,7 +160,6 @@ __global__ void __launch_bounds__(THREADS, 1)
     __shared__ int s_wsum[THREADS / 32];
     const int g = threadIdx.x;
     int v = 0;
-    if (g <= p.ngroups) s_off[g] = p.offsets[g];
     if (g < p.ngroups) v = ((p.offsets[g + 1] - p.offsets[g] + BM - 1) / BM) * p.ntn;
     int incl = v;
 #pragma unroll
@@ -210,7 +214,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       uint32_t it = 0;
       bool ok = true;
       for (int i = blockIdx.x; ok && i < total; i += gridDim.x) {
-        const TileInfo t = decode_tile(i, s_prefix, s_off, p.ngroups, p.ntn);
+        const TileInfo t = decode_tile(i, s_prefix, p.offsets, p.ngroups, p.ntn);
         for (int kb = 0; kb < p.nkb; ++kb) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1u;
@@ -285,7 +289,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     uint32_t tile_iter = 0;
     bool ok = true;
     for (int i = blockIdx.x; ok && i < total; i += gridDim.x, ++tile_iter) {
-      const TileInfo t = decode_tile(i, s_prefix, s_off, p.ngroups, p.ntn);
+      const TileInfo t = decode_tile(i, s_prefix, p.offsets, p.ngroups, p.ntn);
       const bool warp_active = q * 32 < t.nvalid;
       const bool valid = r_in < t.nvalid;
       const int row = t.row0 + r_in;
@@ -426,23 +430,46 @@ __global__ void __launch_bounds__(THREADS, 1)
             *reinterpret_cast<uint4*>(dst + 16 * v) = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
           if (half == 0) p.hs[size_t(t.nt) * p.rows + row] = s;
         }
-      } else {
-        if (valid && nb < p.nb_count) {
+      } else if (warp_active && nb < p.nb_count) {
+        if (q * 32 + 32 <= t.nvalid) {
+          // 32 full rows: bf16 into this warp's 128-byte-swizzled staging box
+          // (16-byte chunk c of row r at chunk c ^ (r % 8)), then one bulk
+          // tensor store per 64 columns; the copy runs while the warp moves on
+          uint8_t* stg = smem + STAGES * STAGE_BYTES + ew * STG_WARP_BYTES;
+          uint8_t* rowp = stg + lane * 128;
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            if (lane == 0) bulk_wait_read0();   // the previous store has read the box
+            __syncwarp();
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              const float* v = acc + 64 * j + 8 * c;
+              *reinterpret_cast<uint4*>(rowp + ((c ^ (lane & 7)) << 4)) =
+                  make_uint4(bf16x2_rn(v[0], v[1]), bf16x2_rn(v[2], v[3]), bf16x2_rn(v[4], v[5]), bf16x2_rn(v[6], v[7]));
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&tmY, stg, nb * 128 + 64 * j, t.row0 + q * 32);
+              bulk_commit();
+            }
+          }
+        } else if (valid) {
+          // the group's last rows (a partial warp): direct stores, so that no
+          // row of the next group is written
           uint16_t* dst = p.y + size_t(row) * p.ld_y + nb * 128;
 #pragma unroll
           for (int v = 0; v < 16; ++v) {
-            uint32_t o[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-              o[j] = uint32_t(f32_to_bf16_bits(acc[8 * v + 2 * j])) |
-                     (uint32_t(f32_to_bf16_bits(acc[8 * v + 2 * j + 1])) << 16);
-            *reinterpret_cast<uint4*>(dst + 8 * v) = make_uint4(o[0], o[1], o[2], o[3]);
+            const float* a8 = acc + 8 * v;
+            *reinterpret_cast<uint4*>(dst + 8 * v) =
+                make_uint4(bf16x2_rn(a8[0], a8[1]), bf16x2_rn(a8[2], a8[3]), bf16x2_rn(a8[4], a8[5]), bf16x2_rn(a8[6], a8[7]));
           }
         }
       }
     }
 
     // ------------------------------------------------ teardown (epilogue side)
+    if (MODE == MODE_DOWN && lane == 0) bulk_wait0();   // stores complete before the CTA exits
     asm volatile("bar.sync 0;" ::: "memory");
     tc_fence_before();
     asm volatile("bar.sync 0;" ::: "memory");
@@ -451,7 +478,8 @@ __global__ void __launch_bounds__(THREADS, 1)
 
 template <int MODE, int EPI>
 cudaError_t launch_gemm(const moe_layer_s* L, const CUtensorMap& tmA, const CUtensorMap& tmB0,
-                        const CUtensorMap& tmB1, const GemmArgs& a, cudaStream_t st) {
+                        const CUtensorMap& tmB1, const CUtensorMap& tmY, const GemmArgs& a, cudaStream_t st) {
+  constexpr int SMEM_DYN = smem_dyn(MODE);
   static bool configured = false;  // per process; the attribute is per function
   if (!configured) {
     // setmaxnreg.inc waits until the registers it asks for are free; they
@@ -469,7 +497,7 @@ cudaError_t launch_gemm(const moe_layer_s* L, const CUtensorMap& tmA, const CUte
   const long long bound = (static_cast<long long>(a.rows) / BM + a.ngroups) * a.ntn;
   const int grid = int(bound < L->num_sms ? bound : L->num_sms);
   if (grid <= 0) return cudaSuccess;
-  grouped_gemm_kernel<MODE, EPI><<<grid, THREADS, SMEM_DYN, st>>>(tmA, tmB0, tmB1, a);
+  grouped_gemm_kernel<MODE, EPI><<<grid, THREADS, SMEM_DYN, st>>>(tmA, tmB0, tmB1, tmY, a);
   return cudaGetLastError();
 }
 
@@ -518,7 +546,7 @@ cudaError_t launch_gate_up(const moe_layer_s* L, const uint8_t* xq, const float*
   a.h = h;
   a.hs = hs;
   a.ld_h = L->ld_hh;
-  return launch_gemm<MODE_GATEUP, EPI_FUSED>(L, tmX, L->tm_gate, L->tm_up, a, st);
+  return launch_gemm<MODE_GATEUP, EPI_FUSED>(L, tmX, L->tm_gate, L->tm_up, tmX, a, st);
 }
 
 cudaError_t launch_down(const moe_layer_s* L, const uint8_t* h, const float* hs, const int32_t* offsets, int T,
@@ -526,10 +554,12 @@ cudaError_t launch_down(const moe_layer_s* L, const uint8_t* h, const float* hs,
   const int rows = T * (L->K + L->S);
   CUtensorMap tmH;
   if (!encode_tmap_u8(&tmH, h, L->F, rows, 1, L->ld_hh, 0)) return cudaErrorInvalidValue;
+  CUtensorMap tmY;
+  if (!encode_tmap_store_bf16(&tmY, y, L->H, rows, size_t(L->H) * 2)) return cudaErrorInvalidValue;
   GemmArgs a = down_args(L, offsets, rows, hs);
   a.y = y;
   a.ld_y = L->H;
-  return launch_gemm<MODE_DOWN, EPI_FUSED>(L, tmH, L->tm_down, L->tm_down, a, st);
+  return launch_gemm<MODE_DOWN, EPI_FUSED>(L, tmH, L->tm_down, L->tm_down, tmY, a, st);
 }
 
 cudaError_t launch_test_gemm_f32(const moe_layer_s* L, int which, const uint8_t* a_ptr, const float* as,
@@ -541,13 +571,13 @@ cudaError_t launch_test_gemm_f32(const moe_layer_s* L, int which, const uint8_t*
     GemmArgs a = gateup_args(L, offsets, rows, as);
     a.out = out;
     a.ld_out = 2 * L->FB * 128;
-    return launch_gemm<MODE_GATEUP, EPI_F32>(L, tmA, L->tm_gate, L->tm_up, a, st);
+    return launch_gemm<MODE_GATEUP, EPI_F32>(L, tmA, L->tm_gate, L->tm_up, tmA, a, st);
   }
   if (!encode_tmap_u8(&tmA, a_ptr, L->F, rows, 1, L->ld_hh, 0)) return cudaErrorInvalidValue;
   GemmArgs a = down_args(L, offsets, rows, as);
   a.out = out;
   a.ld_out = L->H;
-  return launch_gemm<MODE_DOWN, EPI_F32>(L, tmA, L->tm_down, L->tm_down, a, st);
+  return launch_gemm<MODE_DOWN, EPI_F32>(L, tmA, L->tm_down, L->tm_down, tmA, a, st);
 }
 
 }  // namespace moe

@@ -209,6 +209,12 @@ WORKLOADS = {
     # profiler captures that must stay a few GB on the device
     "decode_e64": Workload("decode_e64", 16, LayerShape(H=5120, E=64, K=8, F=1536, ld_f=1536), x_seed=5,
                            w_seed=3, outliers=8, note="T=16, 64+1 experts, hidden 5120, FFN 1536 (profiling case)"),
+    # a prefill-shaped case with several row tiles per expert (about 1000
+    # rows each, like the busier experts of the long prefill) whose weights
+    # and activations stay near 1 GB, for full profiler captures
+    "prefill_e32": Workload("prefill_e32", 4096, LayerShape(H=5120, E=32, K=8, F=1536, ld_f=1536), x_seed=8,
+                            w_seed=6, outliers=8,
+                            note="T=4096, 32+1 experts, hidden 5120, FFN 1536 (profiling case)"),
 }
 
 
