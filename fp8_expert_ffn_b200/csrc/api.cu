@@ -52,15 +52,16 @@ bool encode_tmap(CUtensorMap* tm, bool bf16, const void* base, uint64_t inner, u
   return r == CUDA_SUCCESS;
 }
 
-bool encode_tmap_store_bf16(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t rows, uint64_t ld_bytes) {
+bool encode_tmap_store(CUtensorMap* tm, bool bf16, const void* base, uint64_t inner, uint64_t rows, uint64_t ld_bytes) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {inner, rows};
   cuuint64_t strides[1] = {ld_bytes};
   cuuint32_t box[2] = {64, 32};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+  CUresult r = fn(tm, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
+                  const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  bf16 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }

@@ -69,10 +69,11 @@ constexpr int MCHUNK = 8;                  // row tiles per chunk of the tile or
 constexpr int MAX_GROUPS = 257;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t IDESC = idesc_e4m3_f32(BM, BN);
-// down epilogue: each warp stages 32 rows x 64 bf16 columns (4 KB, the
-// 128-byte-swizzled box of one bulk tensor store) in shared memory
-constexpr int STG_WARP_BYTES = 32 * 128;
-constexpr int smem_dyn(int mode) { return STAGES * STAGE_BYTES + 1024 + (mode == 1 ? EPI_WARPS * STG_WARP_BYTES : 0); }
+// Output staging, one box of a bulk tensor store per epilogue warp: down,
+// 32 rows x 64 bf16 columns (4 KB, 128-byte swizzle); gate/up, 32 rows x the
+// warp's 64 h channels (2 KB, 64-byte swizzle).
+constexpr int stg_warp_bytes(int mode) { return mode == 1 ? 32 * 128 : 32 * 64; }
+constexpr int smem_dyn(int mode) { return STAGES * STAGE_BYTES + 1024 + EPI_WARPS * stg_warp_bytes(mode); }
 
 enum { MODE_GATEUP = 0, MODE_DOWN = 1 };
 enum { EPI_FUSED = 0, EPI_F32 = 1 };
@@ -142,7 +143,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   __shared__ __align__(8) uint64_t empty_bar[STAGES];
   __shared__ __align__(8) uint64_t tfull_bar[2];
   __shared__ __align__(8) uint64_t tempty_bar[2];
-  __shared__ __align__(8) uint64_t amax_bar[2];
+  __shared__ __align__(8) uint64_t amax_bar[2][4];   // [tile parity][TMEM lane quarter]
   __shared__ __align__(8) uint64_t done_bar;
   __shared__ uint32_t tmem_base_s;
   __shared__ int s_prefix[MAX_GROUPS + 1];
@@ -182,7 +183,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull_bar[b], 1);
       mbar_init(&tempty_bar[b], EPI_WARPS);
-      mbar_init(&amax_bar[b], EPI_WARPS);
+      for (int qq = 0; qq < 4; ++qq) mbar_init(&amax_bar[b][qq], 2);   // the two warps sharing those rows
     }
     mbar_init(&done_bar, 1);
     s_abort_store = 0;
@@ -402,8 +403,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         const uint32_t xb = tile_iter & 1u;
         s_amax[xb][half][r_in] = amax;
         __syncwarp();
-        if (lane == 0) mbar_arrive(&amax_bar[xb]);
-        if (!mbar_wait(&amax_bar[xb], (tile_iter >> 1) & 1u, s_abort, p.status)) { ok = false; break; }
+        if (lane == 0) mbar_arrive(&amax_bar[xb][q]);
+        if (!mbar_wait(&amax_bar[xb][q], (tile_iter >> 1) & 1u, s_abort, p.status)) { ok = false; break; }
         amax = fmaxf(amax, s_amax[xb][half ^ 1][r_in]);
         if (valid) {
           uint32_t pk[16];
@@ -424,10 +425,31 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
             for (int j = 0; j < 16; ++j) pk[j] = 0u;
           }
-          uint8_t* dst = p.h + size_t(row) * p.ld_h + t.nt * 128 + half * 64;
+          if (q * 32 + 32 <= t.nvalid) {
+            // 32 full rows: this warp's 64 channels into its 64-byte-swizzled
+            // box (16-byte chunk c of row r at chunk c ^ ((r / 2) % 4)), then
+            // one asynchronous bulk tensor store
+            uint8_t* stg = smem + STAGES * STAGE_BYTES + ew * stg_warp_bytes(MODE);
+            if (lane == 0) bulk_wait_read0();   // the previous store has read the box
+            __syncwarp();
 #pragma unroll
-          for (int v = 0; v < 4; ++v)
-            *reinterpret_cast<uint4*>(dst + 16 * v) = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+            for (int v = 0; v < 4; ++v)
+              *reinterpret_cast<uint4*>(stg + lane * 64 + ((v ^ ((lane >> 1) & 3)) << 4)) =
+                  make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&tmY, stg, t.nt * 128 + half * 64, t.row0 + q * 32);
+              bulk_commit();
+            }
+          } else {
+            // the group's last rows (a partial warp): direct stores, so that
+            // no row of the next group is written
+            uint8_t* dst = p.h + size_t(row) * p.ld_h + t.nt * 128 + half * 64;
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+              *reinterpret_cast<uint4*>(dst + 16 * v) = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+          }
           if (half == 0) p.hs[size_t(t.nt) * p.rows + row] = s;
         }
       } else if (warp_active && nb < p.nb_count) {
@@ -435,7 +457,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           // 32 full rows: bf16 into this warp's 128-byte-swizzled staging box
           // (16-byte chunk c of row r at chunk c ^ (r % 8)), then one bulk
           // tensor store per 64 columns; the copy runs while the warp moves on
-          uint8_t* stg = smem + STAGES * STAGE_BYTES + ew * STG_WARP_BYTES;
+          uint8_t* stg = smem + STAGES * STAGE_BYTES + ew * stg_warp_bytes(MODE);
           uint8_t* rowp = stg + lane * 128;
 #pragma unroll
           for (int j = 0; j < 2; ++j) {
@@ -469,7 +491,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
 
     // ------------------------------------------------ teardown (epilogue side)
-    if (MODE == MODE_DOWN && lane == 0) bulk_wait0();   // stores complete before the CTA exits
+    if (lane == 0) bulk_wait0();   // bulk stores complete before the CTA exits
     asm volatile("bar.sync 0;" ::: "memory");
     tc_fence_before();
     asm volatile("bar.sync 0;" ::: "memory");
@@ -540,13 +562,14 @@ static GemmArgs down_args(const moe_layer_s* L, const int32_t* offsets, int rows
 cudaError_t launch_gate_up(const moe_layer_s* L, const uint8_t* xq, const float* xs, const int32_t* offsets, int T,
                            uint8_t* h, float* hs, cudaStream_t st) {
   const int rows = T * (L->K + L->S);
-  CUtensorMap tmX;
+  CUtensorMap tmX, tmHst;
   if (!encode_tmap_u8(&tmX, xq, L->H, rows, 1, L->H, 0)) return cudaErrorInvalidValue;
+  if (!encode_tmap_store(&tmHst, false, h, L->ld_hh, rows, L->ld_hh)) return cudaErrorInvalidValue;
   GemmArgs a = gateup_args(L, offsets, rows, xs);
   a.h = h;
   a.hs = hs;
   a.ld_h = L->ld_hh;
-  return launch_gemm<MODE_GATEUP, EPI_FUSED>(L, tmX, L->tm_gate, L->tm_up, tmX, a, st);
+  return launch_gemm<MODE_GATEUP, EPI_FUSED>(L, tmX, L->tm_gate, L->tm_up, tmHst, a, st);
 }
 
 cudaError_t launch_down(const moe_layer_s* L, const uint8_t* h, const float* hs, const int32_t* offsets, int T,
@@ -555,7 +578,7 @@ cudaError_t launch_down(const moe_layer_s* L, const uint8_t* h, const float* hs,
   CUtensorMap tmH;
   if (!encode_tmap_u8(&tmH, h, L->F, rows, 1, L->ld_hh, 0)) return cudaErrorInvalidValue;
   CUtensorMap tmY;
-  if (!encode_tmap_store_bf16(&tmY, y, L->H, rows, size_t(L->H) * 2)) return cudaErrorInvalidValue;
+  if (!encode_tmap_store(&tmY, true, y, L->H, rows, size_t(L->H) * 2)) return cudaErrorInvalidValue;
   GemmArgs a = down_args(L, offsets, rows, hs);
   a.y = y;
   a.ld_y = L->H;

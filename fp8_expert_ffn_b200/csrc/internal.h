@@ -77,9 +77,10 @@ cudaError_t launch_combine(const moe_layer_s* L, const uint16_t* y, const int32_
 
 // TMA descriptor for a row-major byte matrix [rows][inner] with row stride
 // `ld` bytes, 128 x 128 boxes, 128-byte swizzle (3-D when depth > 1).
-// Store map of a bf16 [rows][inner] matrix: boxes of 64 columns x 32 rows,
-// 128-byte swizzle (the layout the down epilogue stages).
-bool encode_tmap_store_bf16(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t rows, uint64_t ld_bytes);
+// Store map of a [rows][inner] matrix for the GEMM epilogues: bf16, boxes of
+// 64 columns x 32 rows with 128-byte swizzle (the down GEMM's y); u8, boxes
+// of 64 columns x 32 rows with 64-byte swizzle (the gate/up GEMM's h).
+bool encode_tmap_store(CUtensorMap* tm, bool bf16, const void* base, uint64_t inner, uint64_t rows, uint64_t ld_bytes);
 bool encode_tmap_u8(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t rows, uint64_t depth,
                     uint64_t ld, uint64_t depth_stride);
 // Same for bf16 (box 64 x 128 elements = 128 bytes of K per row) or u8.
