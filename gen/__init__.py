@@ -186,6 +186,10 @@ ZIPF_CHANNEL = 0   # x[:, 0] = 1 carries the bias through the router GEMM
 WORKLOADS = {
     "toy": Workload("toy", 32, TOY, x_seed=0, w_seed=0,
                     note="T=32, hidden 512, 16+1 experts, top-4, FFN 256"),
+    # the toy layer at a batch with several row tiles per group (about 600
+    # rows each), checked on every token
+    "toy_t2048": Workload("toy_t2048", 2048, TOY, x_seed=9, w_seed=0,
+                          note="T=2048, hidden 512, 16+1 experts, top-4, FFN 256"),
     "decode": Workload("decode", 64, DOTS3, x_seed=1, w_seed=1, outliers=8,
                        note="T=64, dots3-note MoE layer, balanced router"),
     "prefill": Workload("prefill", 4096, DOTS3, x_seed=2, w_seed=1, outliers=8,

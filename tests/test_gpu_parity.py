@@ -45,7 +45,7 @@ def get_case(name):
 
 _device_layers = {}
 
-FULL = ["toy", "decode", "dense"]           # every token / row checked
+FULL = ["toy", "toy_t2048", "decode", "dense"]   # every token / row checked
 SAMPLED = ["prefill", "zipf", "edge", "edge_f1500", "vision"]
 ALL = FULL + SAMPLED
 
@@ -204,13 +204,15 @@ def _group_offsets(sh, T, rng):
     return off.astype(np.int32)
 
 
+# T = 60: groups of up to two row tiles; T = 1000: groups of several row
+# tiles (chunks of the tile order, partial last tiles)
+@pytest.mark.parametrize("T", [60, 1000])
 @pytest.mark.parametrize("which", [0, 1])
-def test_grouped_gemm_exact_integers(which):
+def test_grouped_gemm_exact_integers(which, T):
     layer, vals = _integer_layer()
     sh = layer.shape
     dev = tu.upload_layer(layer)
     rng = np.random.default_rng(3 + which)
-    T = 60
     rows = T * (sh.K + 1)
     off = _group_offsets(sh, T, rng)
     Kdim = sh.H if which == 0 else sh.FB * 128
@@ -239,8 +241,9 @@ def test_grouped_gemm_exact_integers(which):
             assert np.array_equal(got[r0:r1], A[r0:r1, :sh.F] @ Wd.T)
 
 
+@pytest.mark.parametrize("T", [60, 1000])
 @pytest.mark.parametrize("which", [0, 1])
-def test_grouped_gemm_promotion_random_scales(which):
+def test_grouped_gemm_promotion_random_scales(which, T):
     """Non-uniform scales: a transposed or shifted scale index would show."""
     wl, layer0, _ = gen.workload_inputs("toy")
     sh = layer0.shape
@@ -249,7 +252,6 @@ def test_grouped_gemm_promotion_random_scales(which):
                       .astype(np.float32), layer0.w_up, layer0.s_up, layer0.w_down,
                       layer0.s_down * rng.uniform(0.25, 4, layer0.s_down.shape).astype(np.float32))
     dev = tu.upload_layer(layer)
-    T = 60
     rows = T * (sh.K + 1)
     off = _group_offsets(sh, T, rng)
     Kdim = sh.H if which == 0 else sh.FB * 128
