@@ -19,6 +19,15 @@ Steps and the readings taken where the pages are silent:
            weights are p renormalised to sum 1, times routed_scaling_factor
            (1.0). Slots are listed in ascending expert id. A token is flagged
            as a near-tie when p_(K) - p_(K+1) < 1e-6.
+           Router variants the config schema allows (n_group, topk_group,
+           norm_topk_prob, and the selection bias of routers balanced by a
+           bias instead of an auxiliary loss): the selection score is
+           p + bias; with n_group > 1 the experts form n_group contiguous
+           groups, each scored by its best member, and only the topk_group
+           best groups (ties to the lower group) are eligible; the weights
+           come from the unbiased p of the selected experts, renormalised
+           only if norm_topk_prob. The near-tie gap is then taken on the
+           selection score, and on the group scores when groups apply.
   permute  counting sort of the (token, slot) pairs by expert, stable in
            token order; offsets has E+2 entries, the shared expert is group E
            and holds one row per token, in token order.
@@ -141,28 +150,58 @@ def softmax(logits: np.ndarray) -> np.ndarray:
     return e / e.sum(axis=1, keepdims=True)
 
 
-def select_topk(probs: np.ndarray, K: int, routed_scaling: float = 1.0):
-    """Top-K by probability, ties to the lower expert id; slots in ascending id."""
+def select_topk(probs: np.ndarray, K: int, routed_scaling: float = 1.0, n_group: int = 1, topk_group: int = 1,
+                bias=None, norm_topk: bool = True):
+    """Top-K by selection score s = p + bias among the eligible experts, ties
+    to the lower expert id; slots in ascending id. Dots3NoteTextConfig:
+    n_group partitions the routed experts for selection and topk_group is
+    the number of groups a token may draw from (1 and 1: ungrouped)."""
     T, E = probs.shape
     ids = np.arange(E)
+    b = np.zeros(E) if bias is None else np.asarray(bias, np.float64)
+    gsize = E // n_group
     idx = np.empty((T, K), np.int32)
     w = np.empty((T, K), np.float64)
     gap = np.empty(T, np.float64)
     for t in range(T):
-        order = np.lexsort((ids, -probs[t]))    # primary: p descending; secondary: id ascending
+        s = probs[t] + b
+        ggap = np.inf
+        if n_group > 1:
+            gscore = s.reshape(n_group, gsize).max(axis=1)          # a group's best member
+            gorder = np.lexsort((np.arange(n_group), -gscore))
+            keep = gorder[:topk_group]
+            if topk_group < n_group:
+                ggap = gscore[gorder[topk_group - 1]] - gscore[gorder[topk_group]]
+            cand = np.sort(np.concatenate([ids[g * gsize:(g + 1) * gsize] for g in keep]))
+        else:
+            cand = ids
+        order = cand[np.lexsort((cand, -s[cand]))]   # primary: s descending; secondary: id ascending
         sel = np.sort(order[:K])
         idx[t] = sel
         ps = probs[t, sel]
-        w[t] = ps / ps.sum() * routed_scaling
-        gap[t] = probs[t, order[K - 1]] - probs[t, order[K]] if K < E else np.inf
+        w[t] = (ps / ps.sum() if norm_topk else ps) * routed_scaling
+        egap = s[order[K - 1]] - s[order[K]] if K < len(cand) else np.inf
+        gap[t] = min(egap, ggap)
     return idx, w, gap
 
 
-def route(x_bits: np.ndarray, router_w: np.ndarray, K: int, routed_scaling: float = 1.0) -> Route:
+def route(x_bits: np.ndarray, router_w: np.ndarray, K: int, routed_scaling: float = 1.0, n_group: int = 1,
+          topk_group: int = 1, bias=None, norm_topk: bool = True) -> Route:
     logits = router_logits(x_bits, router_w)
     probs = softmax(logits)
-    idx, w, gap = select_topk(probs, K, routed_scaling)
+    idx, w, gap = select_topk(probs, K, routed_scaling, n_group, topk_group, bias, norm_topk)
     return Route(logits, probs, idx, w, gap, gap < NEAR_TIE)
+
+
+def router_options(layer) -> dict:
+    """The layer's router settings (defaults: the text model's)."""
+    return {"routed_scaling": getattr(layer, "routed_scaling", 1.0), "n_group": getattr(layer, "n_group", 1),
+            "topk_group": getattr(layer, "topk_group", 1), "bias": getattr(layer, "router_bias", None),
+            "norm_topk": getattr(layer, "norm_topk", True)}
+
+
+def route_layer(x_bits: np.ndarray, layer) -> Route:
+    return route(x_bits, layer.router_w, layer.shape.K, **router_options(layer))
 
 
 # ---------------------------------------------------------------------------
@@ -290,7 +329,7 @@ def gather_rows(tok_codes, tok_scales, perm):
 def layer_forward(x_bits: np.ndarray, layer) -> dict:
     """Whole layer: route -> permute -> quantise/gather -> expert FFNs -> combine."""
     sh = layer.shape
-    r = route(x_bits, layer.router_w, sh.K, getattr(layer, "routed_scaling", 1.0))
+    r = route_layer(x_bits, layer)
     p = permute(r.idx, sh.E, sh.S)
     tq, ts = quantize_tokens(x_bits)
     xq, xs = gather_rows(tq, ts, p.perm)
@@ -308,7 +347,7 @@ def token_outputs(x_bits: np.ndarray, layer, tokens, idx=None, w=None) -> np.nda
     tokens = np.asarray(tokens)
     xb = np.asarray(x_bits)[tokens]
     if idx is None:
-        r = route(xb, layer.router_w, sh.K, getattr(layer, "routed_scaling", 1.0))
+        r = route_layer(xb, layer)
         idx_s, w_s = r.idx, r.w
     else:
         idx_s, w_s = np.asarray(idx)[tokens], np.asarray(w, np.float64)[tokens]
@@ -345,7 +384,7 @@ def layer_forward_bf16(x_bits: np.ndarray, layer, tokens=None, idx=None, w=None)
     tokens = np.arange(T) if tokens is None else np.asarray(tokens)
     xb = np.asarray(x_bits)[tokens]
     if idx is None:
-        r = route(xb, layer.router_w, sh.K, getattr(layer, "routed_scaling", 1.0))
+        r = route_layer(xb, layer)
         idx_s, w_s = r.idx, r.w
     else:
         idx_s, w_s = np.asarray(idx)[tokens], np.asarray(w, np.float64)[tokens]

@@ -364,3 +364,101 @@ def test_routed_scaling_in_oracle():
     r1 = moe.route(x, gen.make_router(sh, 0), sh.K)
     r2 = moe.route(x, gen.make_router(sh, 0), sh.K, routed_scaling=2.5)
     assert np.array_equal(r1.idx, r2.idx) and np.allclose(r2.w, 2.5 * r1.w, rtol=1e-15)
+
+
+# ----------------------------------------------------------------------------- router variants
+
+def test_group_limited_hand_example():
+    """8 experts in 4 groups of 2, two groups eligible, top-3 (worked by hand):
+    group maxima 0.30, 0.20, 0.03, 0.25 keep groups 0 and 3, so expert 2
+    (0.20, group 1) loses to expert 6 (0.04); ungrouped the top-3 is 0, 2, 7."""
+    p = np.array([[0.30, 0.01, 0.20, 0.15, 0.02, 0.03, 0.04, 0.25]])
+    idx, w, gap = moe.select_topk(p, 3, n_group=4, topk_group=2)
+    assert idx.tolist() == [[0, 6, 7]]
+    np.testing.assert_allclose(w[0], np.array([0.30, 0.04, 0.25]) / 0.59, rtol=1e-15)
+    assert gap[0] == pytest.approx(min(0.04 - 0.01, 0.25 - 0.20))
+    idx0, _, _ = moe.select_topk(p, 3)
+    assert idx0.tolist() == [[0, 2, 7]]
+
+
+def test_group_limited_reduces_to_ungrouped():
+    rng = np.random.default_rng(21)
+    p = rng.dirichlet(np.ones(16), size=64)
+    ref = moe.select_topk(p, 4)
+    # every group eligible
+    got = moe.select_topk(p, 4, n_group=4, topk_group=4)
+    assert np.array_equal(got[0], ref[0]) and np.allclose(got[1], ref[1])
+    # one expert per group, K groups eligible: the K best experts
+    got = moe.select_topk(p, 4, n_group=16, topk_group=4)
+    assert np.array_equal(got[0], ref[0]) and np.allclose(got[1], ref[1])
+
+
+def test_group_limited_properties():
+    """Checked on the output only: at most topk_group groups are used, every
+    dropped group's best member is no better than every kept group's, and no
+    eligible expert left out beats a selected one."""
+    rng = np.random.default_rng(22)
+    E, G, TG, K = 64, 8, 3, 6
+    p = rng.dirichlet(np.ones(E) * 0.3, size=200)
+    idx, w, _ = moe.select_topk(p, K, n_group=G, topk_group=TG)
+    gs = E // G
+    for t in range(len(p)):
+        used = set(int(e) // gs for e in idx[t])
+        assert len(used) <= TG
+        gmax = p[t].reshape(G, gs).max(axis=1)
+        # the kept groups: the used ones plus (if fewer) the next best
+        kept = sorted(range(G), key=lambda g: (-gmax[g], g))[:TG]
+        assert used <= set(kept)
+        for g in set(range(G)) - set(kept):
+            assert gmax[g] <= min(gmax[k] for k in kept)
+        elig = [e for e in range(E) if e // gs in kept]
+        left = [e for e in elig if e not in idx[t]]
+        assert max(p[t, left]) <= min(p[t, idx[t]])
+        assert w[t].sum() == pytest.approx(1.0)
+
+
+def test_selection_bias_selects_but_does_not_weight():
+    rng = np.random.default_rng(23)
+    E, K = 32, 4
+    logits = rng.normal(0, 1, (50, E))
+    p = np.exp(logits - logits.max(1, keepdims=True))
+    p /= p.sum(1, keepdims=True)
+    ref = moe.select_topk(p, K)
+    # a constant bias changes nothing
+    got = moe.select_topk(p, K, bias=np.full(E, 0.7))
+    assert np.array_equal(got[0], ref[0]) and np.allclose(got[1], ref[1], rtol=1e-14)
+    # a large negative bias removes an expert, a large positive one forces one in
+    b = np.zeros(E)
+    b[5] = -1000.0
+    b[9] = 1000.0
+    idx, w, _ = moe.select_topk(p, K, bias=b)
+    assert (idx != 5).all() and (idx == 9).any(axis=1).all()
+    for t in range(len(p)):
+        # the weights are the unbiased probabilities of the selected experts,
+        # renormalised (softmax of their logits)
+        sel = idx[t]
+        ex = np.exp(logits[t, sel] - logits[t, sel].max())
+        np.testing.assert_allclose(w[t], ex / ex.sum(), rtol=1e-12)
+
+
+def test_norm_topk_off_keeps_the_softmax_weights():
+    import scipy.special
+    rng = np.random.default_rng(24)
+    sh = gen.TOY
+    x = gen.make_x(9, sh.H, 2)
+    router = gen.make_router(sh, 0)
+    r = moe.route(x, router, sh.K, routed_scaling=2.0, norm_topk=False)
+    full = scipy.special.softmax(moe.bf16_to_f64(x) @ router.astype(np.float64).T, axis=1)
+    np.testing.assert_allclose(r.w, 2.0 * np.take_along_axis(full, r.idx.astype(np.int64), 1), rtol=1e-12)
+    assert (r.w.sum(1) < 2.0).all()
+    r1 = moe.route(x, router, sh.K)
+    assert np.array_equal(r.idx, r1.idx)
+
+
+def test_route_layer_reads_the_layer_options():
+    sh = gen.TOY
+    x = gen.make_x(10, sh.H, 1)
+    wl, layer, _ = gen.workload_inputs("toy")
+    a = moe.route_layer(x, layer)
+    b = moe.route(x, layer.router_w, sh.K)
+    assert np.array_equal(a.idx, b.idx) and np.array_equal(a.w, b.w)
