@@ -33,13 +33,15 @@ class MoeError(RuntimeError):
 class moe_layer_desc(ctypes.Structure):
     _fields_ = [("hidden", ctypes.c_int), ("n_routed", ctypes.c_int), ("n_shared", ctypes.c_int),
                 ("top_k", ctypes.c_int), ("ffn", ctypes.c_int), ("shared_ffn", ctypes.c_int),
-                ("block", ctypes.c_int), ("routed_scaling", ctypes.c_float), ("norm_topk", ctypes.c_int)]
+                ("block", ctypes.c_int), ("routed_scaling", ctypes.c_float), ("norm_topk", ctypes.c_int),
+                ("n_group", ctypes.c_int), ("topk_group", ctypes.c_int)]
 
 
 class moe_weights(ctypes.Structure):
     _fields_ = [("w_gate", ctypes.c_void_p), ("w_up", ctypes.c_void_p), ("w_down", ctypes.c_void_p),
                 ("s_gate", ctypes.c_void_p), ("s_up", ctypes.c_void_p), ("s_down", ctypes.c_void_p),
-                ("router_w", ctypes.c_void_p), ("ld_h", ctypes.c_int), ("ld_f", ctypes.c_int)]
+                ("router_w", ctypes.c_void_p), ("ld_h", ctypes.c_int), ("ld_f", ctypes.c_int),
+                ("router_bias", ctypes.c_void_p)]
 
 
 _lib = None
@@ -123,14 +125,16 @@ class MoeLayer:
     """Owns a moe_layer_t; keeps the weight tensors alive while it exists."""
 
     def __init__(self, hidden, n_routed, top_k, ffn, weights: LayerWeights, ld_h=None, ld_f=None,
-                 routed_scaling=1.0, n_shared=1):
+                 routed_scaling=1.0, n_shared=1, n_group=1, topk_group=1, norm_topk=True, router_bias=None):
+        """router_bias: device fp32 [E] selection-only bias (copied at creation) or None."""
         self.H, self.E, self.K, self.F = hidden, n_routed, top_k, ffn
         self.weights = weights
         self.S = n_shared
-        d = moe_layer_desc(hidden, n_routed, n_shared, top_k, ffn, ffn, 128, routed_scaling, 1)
+        d = moe_layer_desc(hidden, n_routed, n_shared, top_k, ffn, ffn, 128, routed_scaling, int(bool(norm_topk)),
+                           n_group, topk_group)
         w = moe_weights(_ptr(weights.w_gate), _ptr(weights.w_up), _ptr(weights.w_down), _ptr(weights.s_gate),
                         _ptr(weights.s_up), _ptr(weights.s_down), _ptr(weights.router_w),
-                        hidden if ld_h is None else ld_h, ffn if ld_f is None else ld_f)
+                        hidden if ld_h is None else ld_h, ffn if ld_f is None else ld_f, _ptr(router_bias))
         h = ctypes.c_void_p()
         _check("moe_layer_create", lib().moe_layer_create(ctypes.byref(d), ctypes.byref(w), ctypes.byref(h)))
         self.handle = h.value

@@ -152,7 +152,10 @@ moe_status moe_layer_create(const moe_layer_desc* d, const moe_weights* w, moe_l
   if (d->hidden <= 0 || d->n_routed <= 0 || d->top_k <= 0 || d->ffn <= 0) return MOE_ERR_INVALID_ARG;
   if (d->hidden % 128 != 0 || d->hidden > 16384 || d->n_routed > 256 || d->n_shared < 0 || d->n_shared > 1 ||
       d->top_k > 8 || d->top_k > d->n_routed || d->ffn > 16384 || (d->n_shared == 1 && d->shared_ffn != d->ffn) ||
-      d->block != 128 || d->norm_topk != 1)
+      d->block != 128 || (d->norm_topk != 0 && d->norm_topk != 1))
+    return MOE_ERR_UNSUPPORTED;
+  if (d->n_group < 1 || d->n_group > 32 || d->n_routed % d->n_group != 0 || d->topk_group < 1 ||
+      d->topk_group > d->n_group || d->top_k > d->topk_group * (d->n_routed / d->n_group))
     return MOE_ERR_UNSUPPORTED;
   if (!(d->routed_scaling == d->routed_scaling)) return MOE_ERR_INVALID_ARG;
   if (!w->w_gate || !w->w_up || !w->w_down || !w->s_gate || !w->s_up || !w->s_down || !w->router_w)
@@ -162,6 +165,7 @@ moe_status moe_layer_create(const moe_layer_desc* d, const moe_weights* w, moe_l
   const void* ptrs[] = {w->w_gate, w->w_up, w->w_down, w->s_gate, w->s_up, w->s_down, w->router_w};
   for (const void* p : ptrs)
     if (!aligned16(p)) return MOE_ERR_MISALIGNED;
+  if (w->router_bias && !aligned16(w->router_bias)) return MOE_ERR_MISALIGNED;
 
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
@@ -195,6 +199,11 @@ moe_status moe_layer_create(const moe_layer_desc* d, const moe_weights* w, moe_l
   bool ok = cudaMalloc(&L->status, sizeof(uint32_t)) == cudaSuccess;
   ok = ok && cudaMalloc(&L->router_split, split_bytes) == cudaSuccess;
   ok = ok && cudaMemset(L->status, 0, sizeof(uint32_t)) == cudaSuccess;
+  if (w->router_bias) {
+    ok = ok && cudaMalloc(&L->router_bias, sizeof(float) * L->E) == cudaSuccess;
+    ok = ok && cudaMemcpy(L->router_bias, w->router_bias, sizeof(float) * L->E, cudaMemcpyDeviceToDevice) ==
+                   cudaSuccess;
+  }
   ok = ok && launch_router_split(w->router_w, L->E, L->H, L->router_split, nullptr) == cudaSuccess;
   ok = ok && cudaDeviceSynchronize() == cudaSuccess;
   ok = ok && encode_tmap(&L->tm_router, true, L->router_split, L->H, L->E, 3, uint64_t(L->H) * 2,
@@ -202,6 +211,7 @@ moe_status moe_layer_create(const moe_layer_desc* d, const moe_weights* w, moe_l
   if (!ok) {
     cudaFree(L->status);
     cudaFree(L->router_split);
+    cudaFree(L->router_bias);
     delete L;
     return MOE_ERR_CUDA;
   }
@@ -213,6 +223,10 @@ moe_status moe_layer_destroy(moe_layer_t L) {
   if (!L) return MOE_OK;
   cudaError_t e = cudaFree(L->status);
   cudaError_t e2 = cudaFree(L->router_split);
+  if (L->router_bias) {
+    const cudaError_t e3 = cudaFree(L->router_bias);
+    if (e2 == cudaSuccess) e2 = e3;
+  }
   delete L;
   return from_cuda(e != cudaSuccess ? e : e2);
 }

@@ -21,6 +21,7 @@ struct moe_layer_s {
   int num_sms;
   uint32_t* status;  // device status word
   uint16_t* router_split;  // [3][E][H] bf16 terms of router_w (library-owned)
+  float* router_bias;      // [E] selection-only bias (library-owned copy) or null
   CUtensorMap tm_router;   // over router_split, box 64 x 128 x 1
   CUtensorMap tm_gate;  // [E+1][F][ld_h] E4M3, box 128 x 128 x 1
   CUtensorMap tm_up;

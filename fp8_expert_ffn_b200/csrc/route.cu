@@ -27,6 +27,10 @@
 // 64-bit key), and writes the slots in ascending expert id with weights
 // softmax(selected logits) * routed_scaling, which equals the softmax over
 // all experts renormalised over the selection.
+// Router variants of the config schema: with a selection-only bias the key
+// is p + bias (p the softmax over all experts); with n_group > 1 only the
+// topk_group groups whose best member scores highest (ties to the lower
+// group) are eligible; with norm_topk_prob off the weights are p itself.
 #include "common.cuh"
 #include "internal.h"
 
@@ -230,39 +234,122 @@ __device__ __forceinline__ uint32_t ordered_bits(float f) {
   uint32_t u = __float_as_uint(f);
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
-__device__ __forceinline__ float from_ordered_bits(uint32_t o) {
-  uint32_t u = (o & 0x80000000u) ? (o & 0x7FFFFFFFu) : ~o;
-  return __uint_as_float(u);
+
+struct TopkArgs {
+  const float* partial;  // [S][T][E] split-K partial logits
+  int S, T, E, K;
+  float scaling;         // routed_scaling_factor
+  int norm;              // norm_topk_prob
+  int n_group, topk_group;
+  const float* bias;     // [E] selection-only bias or null
+  int32_t* idx;
+  float* w;
+  float* logits_out;     // [T][E] or null
+};
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, off));
+  return v;
 }
 
-__global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict__ partial, int S, int T, int E,
-                                                         int K, float scaling, int32_t* __restrict__ idx,
-                                                         float* __restrict__ w, float* __restrict__ logits_out) {
-  const int lane = threadIdx.x & 31;
-  const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
-  if (t >= T) return;
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, off);
+  return v;
+}
+
+__device__ __forceinline__ unsigned long long warp_max_u64(unsigned long long v) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    const unsigned long long o = __shfl_xor_sync(0xFFFFFFFFu, v, off);
+    v = o > v ? o : v;
+  }
+  return v;
+}
+
+__global__ void __launch_bounds__(256) route_topk_kernel(const TopkArgs a) {
+  __shared__ unsigned long long s_key[8][256];   // per warp: the selection keys, for group scores
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int t = blockIdx.x * 8 + wid;
+  if (t >= a.T) return;
+  const int E = a.E, K = a.K;
   // expert e = lane + 32*j; the S split-K partials are added in order s = 0..S-1
   float l[8];
 #pragma unroll
   for (int j = 0; j < 8; ++j) l[j] = 0.0f;
-  const float* pt = partial + size_t(t) * E + lane;
-  const size_t ps = size_t(T) * E;
-  for (int s = 0; s < S; ++s) {
+  const float* pt = a.partial + size_t(t) * E + lane;
+  const size_t ps = size_t(a.T) * E;
+  for (int s = 0; s < a.S; ++s) {
     float v[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) v[j] = (lane + 32 * j < E) ? __ldg(pt + s * ps + 32 * j) : 0.0f;
 #pragma unroll
     for (int j = 0; j < 8; ++j) l[j] += v[j];
   }
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    l[j] += 0.0f;  // -0 -> +0 so that equal logits compare equal
+    if (a.logits_out && lane + 32 * j < E) a.logits_out[size_t(t) * E + lane + 32 * j] = l[j];
+  }
+  // softmax over all E experts, needed for a selection bias (s = p + b) and
+  // for weights that are not renormalised
+  const bool full_p = a.bias != nullptr || !a.norm;
+  float lmax_all = 0.0f, sum_all = 1.0f;
+  float ex[8];
+  if (full_p) {
+    float m = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (lane + 32 * j < E) m = fmaxf(m, l[j]);
+    lmax_all = warp_max(m);
+    float sl = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      ex[j] = (lane + 32 * j < E) ? expf(l[j] - lmax_all) : 0.0f;
+      sl += ex[j];
+    }
+    sum_all = warp_sum(sl);
+  }
+  // selection keys: order-preserving bits of the score, inverted id as tie-break
   unsigned long long key[8];
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
     const int e = lane + 32 * j;
     key[j] = 0ull;
     if (e < E) {
-      const float lj = l[j] + 0.0f;  // -0 -> +0 so that equal logits compare equal
-      if (logits_out) logits_out[size_t(t) * E + e] = lj;
-      key[j] = (static_cast<unsigned long long>(ordered_bits(lj)) << 32) | (0xFFFFFFFFu - uint32_t(e));
+      const float sc = a.bias ? ex[j] / sum_all + __ldg(a.bias + e) : l[j];
+      key[j] = (static_cast<unsigned long long>(ordered_bits(sc)) << 32) | (0xFFFFFFFFu - uint32_t(e));
+    }
+  }
+  if (a.n_group > 1) {
+    // group g = experts [g*gs, (g+1)*gs), scored by its best member; the
+    // topk_group best groups (ties to the lower group) stay eligible
+    const int gs = E / a.n_group;
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (lane + 32 * j < E) s_key[wid][lane + 32 * j] = key[j];
+    __syncwarp();
+    unsigned long long gk = 0ull;
+    if (lane < a.n_group) {
+      uint32_t best = 0u;
+      for (int e = lane * gs; e < (lane + 1) * gs; ++e) {
+        const uint32_t sb = uint32_t(s_key[wid][e] >> 32);
+        best = sb > best ? sb : best;
+      }
+      gk = (static_cast<unsigned long long>(best) << 32) | (0xFFFFFFFFu - uint32_t(lane));
+    }
+    uint32_t keep = 0u;
+    for (int r = 0; r < a.topk_group; ++r) {
+      const unsigned long long b = warp_max_u64(gk);
+      const int g = int(0xFFFFFFFFu - uint32_t(b & 0xFFFFFFFFull));
+      keep |= 1u << g;
+      if (lane == g) gk = 0ull;
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int e = lane + 32 * j;
+      if (e < E && !((keep >> (e / gs)) & 1u)) key[j] = 0ull;
     }
   }
   int my_e = -1;
@@ -271,25 +358,33 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict
     unsigned long long best = 0ull;
 #pragma unroll
     for (int j = 0; j < 8; ++j) best = key[j] > best ? key[j] : best;
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      unsigned long long o = __shfl_xor_sync(0xFFFFFFFFu, best, off);
-      best = o > best ? o : best;
-    }
+    best = warp_max_u64(best);
     const int e = int(0xFFFFFFFFu - uint32_t(best & 0xFFFFFFFFull));
+    float le = 0.0f;   // the winner's logit, from the lane that holds it
 #pragma unroll
     for (int j = 0; j < 8; ++j)
-      if (lane + 32 * j == e) key[j] = 0ull;      // remove the winner
+      if (lane + 32 * j == e) {
+        key[j] = 0ull;  // remove the winner
+        le = l[j];
+      }
+    le = __shfl_sync(0xFFFFFFFFu, le, e & 31);
     if (lane == r) {
       my_e = e;
-      my_l = from_ordered_bits(uint32_t(best >> 32));
+      my_l = le;
     }
   }
-  // weights: softmax over the selected logits; the first pick is the max.
-  const float lmax = __shfl_sync(0xFFFFFFFFu, my_l, 0);
-  const float ex = (lane < K) ? expf(my_l - lmax) : 0.0f;
-  float sum = 0.0f;
-  for (int r = 0; r < K; ++r) sum += __shfl_sync(0xFFFFFFFFu, ex, r);
+  // weights from the unbiased probabilities: renormalised, the softmax over
+  // the selected logits; otherwise the softmax over all experts
+  float wv;
+  if (a.norm) {
+    const float lmax = warp_max(lane < K ? my_l : -INFINITY);
+    const float es = (lane < K) ? expf(my_l - lmax) : 0.0f;
+    float sum = 0.0f;
+    for (int r = 0; r < K; ++r) sum += __shfl_sync(0xFFFFFFFFu, es, r);
+    wv = es / sum;
+  } else {
+    wv = expf(my_l - lmax_all) / sum_all;
+  }
   // slot position = rank of the expert id among the selected ids
   int pos = 0;
   for (int r = 0; r < K; ++r) {
@@ -297,8 +392,8 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict
     pos += (er < my_e) ? 1 : 0;
   }
   if (lane < K) {
-    idx[size_t(t) * K + pos] = my_e;
-    w[size_t(t) * K + pos] = (ex / sum) * scaling;
+    a.idx[size_t(t) * K + pos] = my_e;
+    a.w[size_t(t) * K + pos] = wv * a.scaling;
   }
 }
 
@@ -336,8 +431,21 @@ cudaError_t launch_route(const moe_layer_s* L, const uint16_t* x, int T, int ldx
   route_tc_kernel<<<grid, R_THREADS, R_SMEM_DYN, st>>>(tmX, L->tm_router, T, L->E, kb_per, nkb, partial, L->status);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  route_topk_kernel<<<(T + 7) / 8, 256, 0, st>>>(partial, S_eff, T, L->E, L->K, L->d.routed_scaling, idx, w,
-                                                  logits);
+  TopkArgs ta;
+  ta.partial = partial;
+  ta.S = S_eff;
+  ta.T = T;
+  ta.E = L->E;
+  ta.K = L->K;
+  ta.scaling = L->d.routed_scaling;
+  ta.norm = L->d.norm_topk;
+  ta.n_group = L->d.n_group;
+  ta.topk_group = L->d.topk_group;
+  ta.bias = L->router_bias;
+  ta.idx = idx;
+  ta.w = w;
+  ta.logits_out = logits;
+  route_topk_kernel<<<(T + 7) / 8, 256, 0, st>>>(ta);
   return cudaGetLastError();
 }
 

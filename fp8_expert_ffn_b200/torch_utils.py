@@ -21,10 +21,12 @@ def bf16_bits(t: torch.Tensor) -> np.ndarray:
     return t.detach().contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
 
 
-def upload_layer(host, device="cuda", routed_scaling=1.0, share_experts: MoeLayer = None) -> MoeLayer:
+def upload_layer(host, device="cuda", routed_scaling=None, share_experts: MoeLayer = None) -> MoeLayer:
     """host: an object with shape (H, E, K, F, ld_f) and the numpy weight arrays
-    router_w, w_gate, s_gate, w_up, s_up, w_down, s_down. With share_experts,
-    the expert tensors of that layer are reused and only the router is copied."""
+    router_w, w_gate, s_gate, w_up, s_up, w_down, s_down; optional router
+    settings routed_scaling, n_group, topk_group, norm_topk and router_bias
+    (numpy [E]) are read from it when present. With share_experts, the expert
+    tensors of that layer are reused and only the router is copied."""
     sh = host.shape
     if share_experts is not None:
         src = share_experts.weights
@@ -36,8 +38,14 @@ def upload_layer(host, device="cuda", routed_scaling=1.0, share_experts: MoeLaye
             w_down=to_device(host.w_down, device), s_gate=to_device(host.s_gate, device),
             s_up=to_device(host.s_up, device), s_down=to_device(host.s_down, device),
             router_w=to_device(host.router_w, device))
+    if routed_scaling is None:
+        routed_scaling = getattr(host, "routed_scaling", 1.0)
+    bias = getattr(host, "router_bias", None)
+    bias_dev = None if bias is None else to_device(np.asarray(bias, np.float32), device)
     return MoeLayer(sh.H, sh.E, sh.K, sh.F, w, ld_h=host.w_gate.shape[2], ld_f=host.w_down.shape[2],
-                    routed_scaling=routed_scaling, n_shared=getattr(sh, "S", 1))
+                    routed_scaling=routed_scaling, n_shared=getattr(sh, "S", 1),
+                    n_group=getattr(host, "n_group", 1), topk_group=getattr(host, "topk_group", 1),
+                    norm_topk=getattr(host, "norm_topk", True), router_bias=bias_dev)
 
 
 def workspace(layer: MoeLayer, T: int, device="cuda") -> torch.Tensor:

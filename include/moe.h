@@ -14,7 +14,9 @@
  *   - router logits are FP32; top-K by logit (equivalently by softmax
  *     probability), ties to the lower expert id; the K weights are the
  *     softmax over the K selected logits (= softmax over all E experts
- *     renormalised over the selection), times routed_scaling;
+ *     renormalised over the selection), times routed_scaling; the router
+ *     variants of the config schema (n_group / topk_group, norm_topk_prob
+ *     off, a selection-only bias) are described at moe_route;
  *   - the K slots of a token are listed in ascending expert id;
  *   - E4M3 is the OCP "FN" flavour (max 448, no infinities); quantisation
  *     is s = fp32(amax)/448 (IEEE fp32 divide), q = E4M3_RNE_satfinite(v/s)
@@ -71,11 +73,13 @@ typedef enum {
 /* Layer description; mirrors Dots3NoteTextConfig (transformers docs page
  * "Dots 3 Note Preview"): hidden_size, n_routed_experts, n_shared_experts,
  * num_experts_per_tok, moe_intermediate_size, shared_experts_intermediate_size,
- * routed_scaling_factor, norm_topk_prob; block = the 128 x 128 weight block
- * edge of transformers PR #47844. This build requires: hidden % 128 == 0,
- * 128 <= hidden <= 16384, 1 <= n_routed <= 256, n_shared 0 or 1,
- * 1 <= top_k <= min(8, n_routed), 1 <= ffn <= 16384, shared_ffn == ffn when n_shared = 1,
- * block == 128, norm_topk == 1; otherwise MOE_ERR_UNSUPPORTED. */
+ * routed_scaling_factor, norm_topk_prob, n_group, topk_group; block = the
+ * 128 x 128 weight block edge of transformers PR #47844. This build requires:
+ * hidden % 128 == 0, 128 <= hidden <= 16384, 1 <= n_routed <= 256, n_shared
+ * 0 or 1, 1 <= top_k <= min(8, n_routed), 1 <= ffn <= 16384, shared_ffn ==
+ * ffn when n_shared = 1, block == 128, norm_topk 0 or 1, 1 <= n_group <= 32
+ * with n_routed % n_group == 0, 1 <= topk_group <= n_group and top_k <=
+ * topk_group * n_routed / n_group; otherwise MOE_ERR_UNSUPPORTED. */
 typedef struct {
   int hidden;           /* H */
   int n_routed;         /* E */
@@ -84,8 +88,10 @@ typedef struct {
   int ffn;              /* F */
   int shared_ffn;       /* must equal ffn when n_shared = 1 */
   int block;            /* must be 128 */
-  float routed_scaling; /* multiplies the renormalised routed weights */
-  int norm_topk;        /* must be 1 */
+  float routed_scaling; /* multiplies the routed weights */
+  int norm_topk;        /* 1: the K weights are renormalised to sum 1 */
+  int n_group;          /* experts e of group e / (E / n_group); 1 = ungrouped */
+  int topk_group;       /* groups a token may draw its K experts from */
 } moe_layer_desc;
 
 /* Caller-owned device weights; they must outlive the layer handle. Expert
@@ -96,7 +102,10 @@ typedef struct {
  *   s_gate, s_up : [E+S][ceil(F/128)][H/128]
  *   w_down       : [E+S][H][ld_f]   bytes, ld_f >= F, ld_f % 16 == 0
  *   s_down       : [E+S][H/128][ceil(F/128)]
- *   router_w     : [E][H] fp32, row-major                                  */
+ *   router_w     : [E][H] fp32, row-major
+ *   router_bias  : [E] fp32 or NULL; selection-only bias of routers balanced
+ *                  by a bias instead of an auxiliary loss (added to the
+ *                  softmax probabilities to choose experts, not to weigh them) */
 typedef struct {
   const uint8_t* w_gate;
   const uint8_t* w_up;
@@ -107,6 +116,7 @@ typedef struct {
   const float* router_w;
   int ld_h;
   int ld_f;
+  const float* router_bias;
 } moe_weights;
 
 typedef struct moe_layer_s* moe_layer_t;
@@ -118,9 +128,9 @@ const char* moe_status_string(moe_status s);
  * encodes the weights' TMA descriptors once, allocates the 4-byte device
  * status word and writes the router weight as three bf16 terms
  * (hi + mid + lo == router_w exactly; the tensor-core router multiplies the
- * bf16 input by each term). Synchronises the device once. On error *out is
- * NULL. The router weight is read only here: a later change to router_w
- * needs a new handle. */
+ * bf16 input by each term) and copies router_bias when given. Synchronises
+ * the device once. On error *out is NULL. The router weight and bias are
+ * read only here: a later change to either needs a new handle. */
 moe_status moe_layer_create(const moe_layer_desc* desc, const moe_weights* w, moe_layer_t* out);
 
 /* Frees the handle (not the caller's weights). NULL is accepted. */
@@ -130,9 +140,14 @@ moe_status moe_layer_destroy(moe_layer_t layer);
  * covers the scratch of moe_permute and moe_expert_ffn. 0 on bad input. */
 size_t moe_workspace_size(moe_layer_t layer, int T);
 
-/* Router: logits = x . router_w^T in FP32, top-K experts per token (ties to
- * the lower id, slots in ascending id), weights = softmax over the K selected
- * logits times routed_scaling.
+/* Router: logits = x . router_w^T in FP32, p = softmax over the E experts,
+ * selection score s = p + router_bias (s orders like the logits when there
+ * is no bias); with n_group > 1 only the topk_group groups with the best
+ * member s (ties to the lower group) are eligible; top-K eligible experts by
+ * s (ties to the lower id, slots in ascending id); weights = the selected p
+ * (renormalised to sum 1 when norm_topk) times routed_scaling. Dots3NoteTextConfig
+ * n_group / topk_group / norm_topk_prob / routed_scaling_factor; the pages
+ * give no group-scoring rule, a group is scored by its best member.
  *   x             [T][ldx] bf16, ldx >= H
  *   topk_idx      [T][K] int32 (out)
  *   topk_w        [T][K] fp32  (out)

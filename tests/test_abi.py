@@ -46,13 +46,13 @@ def test_status_strings():
 
 def _desc(**kw):
     d = dict(hidden=5120, n_routed=256, n_shared=1, top_k=8, ffn=1536, shared_ffn=1536, block=128,
-             routed_scaling=1.0, norm_topk=1)
+             routed_scaling=1.0, norm_topk=1, n_group=1, topk_group=1)
     d.update(kw)
     return fx.moe_layer_desc(**d)
 
 
-def _weights(ptr=4096, ld_h=5120, ld_f=1536):
-    return fx.moe_weights(ptr, ptr, ptr, ptr, ptr, ptr, ptr, ld_h, ld_f)
+def _weights(ptr=4096, ld_h=5120, ld_f=1536, bias=None):
+    return fx.moe_weights(ptr, ptr, ptr, ptr, ptr, ptr, ptr, ld_h, ld_f, bias)
 
 
 def _create(desc, w):
@@ -69,7 +69,13 @@ def _create(desc, w):
     (dict(n_routed=300), fx.MOE_ERR_UNSUPPORTED),
     (dict(shared_ffn=1024), fx.MOE_ERR_UNSUPPORTED),
     (dict(block=64), fx.MOE_ERR_UNSUPPORTED),
-    (dict(norm_topk=0), fx.MOE_ERR_UNSUPPORTED),
+    (dict(norm_topk=2), fx.MOE_ERR_UNSUPPORTED),
+    (dict(n_group=0), fx.MOE_ERR_UNSUPPORTED),
+    (dict(n_group=3), fx.MOE_ERR_UNSUPPORTED),            # 256 experts do not split in 3
+    (dict(n_group=64), fx.MOE_ERR_UNSUPPORTED),           # more than 32 groups
+    (dict(n_group=8, topk_group=9), fx.MOE_ERR_UNSUPPORTED),
+    (dict(n_group=8, topk_group=0), fx.MOE_ERR_UNSUPPORTED),
+    (dict(n_routed=16, top_k=8, n_group=8, topk_group=3), fx.MOE_ERR_UNSUPPORTED),  # 3 groups of 2 < 8
     (dict(top_k=0), fx.MOE_ERR_INVALID_ARG),
     (dict(ffn=0, shared_ffn=0), fx.MOE_ERR_INVALID_ARG),
 ])
@@ -83,6 +89,7 @@ def test_create_rejects_bad_weights():
     assert _create(_desc(), None)[0] == fx.MOE_ERR_INVALID_ARG
     assert _create(_desc(), _weights(ptr=0))[0] == fx.MOE_ERR_INVALID_ARG
     assert _create(_desc(), _weights(ptr=4097))[0] == fx.MOE_ERR_MISALIGNED
+    assert _create(_desc(), _weights(bias=4100))[0] == fx.MOE_ERR_MISALIGNED
     assert _create(_desc(), _weights(ld_h=5128))[0] == fx.MOE_ERR_MISALIGNED
     assert _create(_desc(), _weights(ld_h=4096))[0] == fx.MOE_ERR_INVALID_ARG
     assert _create(_desc(), _weights(ld_f=1500))[0] == fx.MOE_ERR_INVALID_ARG

@@ -410,3 +410,72 @@ def test_dense_ffn_is_the_single_expert():
     assert not c.np("idx").any() and np.all(c.np("w") == 1.0)
     assert np.array_equal(c.np("perm"), np.arange(c.T)) and np.array_equal(c.np("inv").ravel(), np.arange(c.T))
     assert np.array_equal(tu.bf16_bits(c.y), c.np("out"))
+
+
+# ----------------------------------------------------------------------------- router variants
+
+def _variant_layer(layer0, **opts):
+    layer = gen.Layer(layer0.shape, layer0.router_w, layer0.w_gate, layer0.s_gate, layer0.w_up, layer0.s_up,
+                      layer0.w_down, layer0.s_down)
+    for k, v in opts.items():
+        setattr(layer, k, v)
+    return layer
+
+
+_VARIANTS = {
+    "groups": dict(n_group=4, topk_group=2),
+    "bias": dict(router_bias="random"),
+    "no_norm": dict(norm_topk=False, routed_scaling=1.5),
+    "all": dict(n_group=8, topk_group=3, router_bias="random", norm_topk=False, routed_scaling=2.0),
+}
+
+
+def _opts(name, E):
+    opts = dict(_VARIANTS[name])
+    if opts.get("router_bias") == "random":
+        # of the order of the probabilities (1/E), so that it changes choices
+        opts["router_bias"] = np.random.default_rng(31).normal(0, 1.0 / E, E).astype(np.float32)
+    return opts
+
+
+@pytest.mark.parametrize("variant", list(_VARIANTS))
+def test_router_variants_toy(variant):
+    """Group-limited selection, a selection-only bias and norm_topk_prob off
+    (Dots3NoteTextConfig n_group / topk_group / norm_topk_prob): routing
+    bit-exact apart from flagged near-ties, and the whole layer within the
+    output tolerance, on the toy layer at T = 512."""
+    wl, layer0, _ = gen.workload_inputs("toy")
+    sh = layer0.shape
+    layer = _variant_layer(layer0, **_opts(variant, sh.E))
+    x = gen.make_x(512, sh.H, 40 + len(variant))
+    c = gc.Case(layer, x, tu.upload_layer(layer))
+    ref = moe.layer_forward(x, layer)
+    r = ref["route"]
+    keep = ~r.near_tie
+    assert keep.mean() > 0.95
+    assert np.array_equal(c.np("idx")[keep], r.idx[keep])
+    assert np.allclose(c.np("w")[keep], r.w[keep], rtol=2e-5, atol=1e-6)
+    if variant == "bias":   # the bias changed the choice of some tokens
+        assert (moe.route(x, layer.router_w, sh.K).idx != r.idx).any()
+    gc.assert_output_close(moe.bf16_to_f64(c.np("out"))[keep], ref["out"][keep], f"router variant {variant}")
+
+
+def test_router_variants_full_router():
+    """The 256-expert router with 8 groups (4 eligible) and a bias: routing
+    and weights against the oracle on the decode batch."""
+    wl, layer0, c0 = get_case("decode")
+    sh = layer0.shape
+    layer = _variant_layer(layer0, n_group=8, topk_group=4, **{"router_bias": _opts("bias", sh.E)["router_bias"]})
+    dev = tu.upload_layer(layer, share_experts=c0.dev)
+    T = c0.T
+    idx = torch.empty((T, sh.K), dtype=torch.int32, device="cuda")
+    w = torch.empty((T, sh.K), dtype=torch.float32, device="cuda")
+    ws = tu.workspace(dev, T)
+    fx.moe_route(dev, c0.x, T, sh.H, idx, w, None, ws, ws.numel())
+    r = moe.route_layer(c0.x_bits, layer)
+    keep = ~r.near_tie
+    got = idx.cpu().numpy()
+    assert np.array_equal(got[keep], r.idx[keep])
+    assert np.allclose(w.cpu().numpy()[keep], r.w[keep], rtol=2e-5, atol=1e-6)
+    gs = sh.E // 8
+    assert all(len(set(int(e) // gs for e in row)) <= 4 for row in got)
