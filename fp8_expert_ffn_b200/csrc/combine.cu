@@ -22,6 +22,8 @@ __global__ void __launch_bounds__(CB_THREADS) combine_kernel(const uint16_t* __r
                                                              const int32_t* __restrict__ inv,
                                                              const float* __restrict__ w, int T, int K, int S, int H,
                                                              uint16_t* __restrict__ out, int ldo) {
+  pdl_wait();
+  pdl_launch_dependents();
   const int t = blockIdx.x;
   __shared__ int s_row[9];
   __shared__ float s_w[9];
@@ -70,8 +72,7 @@ __global__ void __launch_bounds__(CB_THREADS) combine_kernel(const uint16_t* __r
 cudaError_t launch_combine(const moe_layer_s* L, const uint16_t* y, const int32_t* inv, const float* w, int T,
                            uint16_t* out, int ldo, cudaStream_t st) {
   dim3 grid(T, (L->H + CB_THREADS * 8 - 1) / (CB_THREADS * 8));
-  combine_kernel<<<grid, CB_THREADS, 0, st>>>(y, inv, w, T, L->K, L->S, L->H, out, ldo);
-  return cudaGetLastError();
+  return launch_pdl(combine_kernel, grid, dim3(CB_THREADS), 0, st, y, inv, w, T, L->K, L->S, L->H, out, ldo);
 }
 
 }  // namespace moe

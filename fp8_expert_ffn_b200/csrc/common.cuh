@@ -245,6 +245,10 @@ __device__ __forceinline__ void ffma2(float& a0, float& a1, float v0, float v1, 
 }
 
 // ---------------------------------------------------------------- PDL
+// pdl_wait: returns once the kernels before this one on the stream have
+// completed and their writes are visible (a no-op without programmatic
+// dependent launch). pdl_launch_dependents: lets the next kernel's CTAs be
+// scheduled once every CTA of this grid has issued it or exited.
 
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_launch_dependents() {

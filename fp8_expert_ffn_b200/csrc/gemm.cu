@@ -155,26 +155,6 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // Group offsets and the exclusive prefix of the tile counts (every CTA
-  // derives the same tile list from the device-side offsets).
-  {
-    __shared__ int s_wsum[THREADS / 32];
-    const int g = threadIdx.x;
-    int v = 0;
-    if (g < p.ngroups) v = ((p.offsets[g + 1] - p.offsets[g] + BM - 1) / BM) * p.ntn;
-    int incl = v;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int o = __shfl_up_sync(0xFFFFFFFFu, incl, off);
-      if ((threadIdx.x & 31) >= off) incl += o;
-    }
-    if ((threadIdx.x & 31) == 31) s_wsum[threadIdx.x >> 5] = incl;
-    __syncthreads();
-    int base = 0;
-    for (int j = 0; j < (threadIdx.x >> 5); ++j) base += s_wsum[j];
-    if (g < p.ngroups) s_prefix[g] = base + incl - v;
-    if (g == p.ngroups - 1) s_prefix[p.ngroups] = base + incl;
-  }
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full_bar[s], 1);
@@ -197,6 +177,31 @@ __global__ void __launch_bounds__(THREADS, 1)
     tma_prefetch_desc(&tmB1);
   }
   if (warp == 1) tmem_alloc(&tmem_base_s, TMEM_COLS);
+  // the set-up above overlaps the previous kernel; its outputs (offsets, the
+  // A operand) and this kernel's outputs are touched only below
+  pdl_wait();
+  pdl_launch_dependents();
+
+  // Group offsets and the exclusive prefix of the tile counts (every CTA
+  // derives the same tile list from the device-side offsets).
+  {
+    __shared__ int s_wsum[THREADS / 32];
+    const int g = threadIdx.x;
+    int v = 0;
+    if (g < p.ngroups) v = ((p.offsets[g + 1] - p.offsets[g] + BM - 1) / BM) * p.ntn;
+    int incl = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int o = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+      if ((threadIdx.x & 31) >= off) incl += o;
+    }
+    if ((threadIdx.x & 31) == 31) s_wsum[threadIdx.x >> 5] = incl;
+    __syncthreads();
+    int base = 0;
+    for (int j = 0; j < (threadIdx.x >> 5); ++j) base += s_wsum[j];
+    if (g < p.ngroups) s_prefix[g] = base + incl - v;
+    if (g == p.ngroups - 1) s_prefix[p.ngroups] = base + incl;
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -519,8 +524,7 @@ cudaError_t launch_gemm(const moe_layer_s* L, const CUtensorMap& tmA, const CUte
   const long long bound = (static_cast<long long>(a.rows) / BM + a.ngroups) * a.ntn;
   const int grid = int(bound < L->num_sms ? bound : L->num_sms);
   if (grid <= 0) return cudaSuccess;
-  grouped_gemm_kernel<MODE, EPI><<<grid, THREADS, SMEM_DYN, st>>>(tmA, tmB0, tmB1, tmY, a);
-  return cudaGetLastError();
+  return launch_pdl(grouped_gemm_kernel<MODE, EPI>, dim3(grid), dim3(THREADS), SMEM_DYN, st, tmA, tmB0, tmB1, tmY, a);
 }
 
 }  // namespace

@@ -81,6 +81,26 @@ cudaError_t launch_combine(const moe_layer_s* L, const uint16_t* y, const int32_
 // Store map of a [rows][inner] matrix for the GEMM epilogues: bf16, boxes of
 // 64 columns x 32 rows with 128-byte swizzle (the down GEMM's y); u8, boxes
 // of 64 columns x 32 rows with 64-byte swizzle (the gate/up GEMM's h).
+// Launch with programmatic dependent launch allowed: the kernel's CTAs may
+// start while the previous kernel on the stream is finishing. Every kernel of
+// the library calls pdl_wait() before it touches memory that an earlier
+// kernel writes or reads, and pdl_launch_dependents() right after, so each
+// kernel's set-up overlaps the tail of the one before.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args... args) {
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 bool encode_tmap_store(CUtensorMap* tm, bool bf16, const void* base, uint64_t inner, uint64_t rows, uint64_t ld_bytes);
 bool encode_tmap_u8(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t rows, uint64_t depth,
                     uint64_t ld, uint64_t depth_stride);

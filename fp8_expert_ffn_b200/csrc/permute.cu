@@ -27,8 +27,19 @@ namespace moe {
 
 namespace {
 
+// Zeroes the token bitmap (n words) that the bitmap kernel ORs into.
+__global__ void __launch_bounds__(256) permute_clear_kernel(uint32_t* __restrict__ bitmap, size_t n) {
+  pdl_wait();
+  pdl_launch_dependents();
+  const size_t i = (size_t(blockIdx.x) * blockDim.x + threadIdx.x) * 4;
+  if (i + 4 <= n) *reinterpret_cast<uint4*>(bitmap + i) = make_uint4(0u, 0u, 0u, 0u);
+  else for (size_t k = i; k < n; ++k) bitmap[k] = 0u;
+}
+
 __global__ void permute_bitmap_kernel(const int32_t* __restrict__ idx, int T, int K, int E, int W,
                                       uint32_t* __restrict__ bitmap, uint32_t* status) {
+  pdl_wait();
+  pdl_launch_dependents();
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= T * K) return;
   const int t = i / K;
@@ -47,6 +58,8 @@ __global__ void permute_bitmap_kernel(const int32_t* __restrict__ idx, int T, in
 __global__ void __launch_bounds__(256) permute_count_kernel(const uint32_t* __restrict__ bitmap, int W,
                                                             uint32_t* __restrict__ wprefix,
                                                             int32_t* __restrict__ counts) {
+  pdl_wait();
+  pdl_launch_dependents();
   __shared__ uint32_t warp_sums[8];
   const int e = blockIdx.x, tid = threadIdx.x;
   const uint32_t* row = bitmap + size_t(e) * W;
@@ -78,6 +91,8 @@ __global__ void __launch_bounds__(256) permute_count_kernel(const uint32_t* __re
 // offsets[g] = sum of counts[0..g), offsets[E+1] = offsets[E] + T.
 __global__ void __launch_bounds__(256) permute_offsets_kernel(const int32_t* __restrict__ counts, int E, int T,
                                                               int S, int32_t* __restrict__ offsets) {
+  pdl_wait();
+  pdl_launch_dependents();
   __shared__ int32_t warp_sums[8];
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   const int v = tid < E ? counts[tid] : 0;
@@ -107,6 +122,8 @@ __global__ void __launch_bounds__(256) permute_gather_kernel(
     const uint32_t* __restrict__ bitmap, const uint32_t* __restrict__ wprefix, const int32_t* __restrict__ offsets,
     int S, int rows, int32_t* __restrict__ perm, int32_t* __restrict__ inv, uint8_t* __restrict__ xq,
     float* __restrict__ xs) {
+  pdl_wait();
+  pdl_launch_dependents();
   const int lane = threadIdx.x & 31;
   const int HB = H / 128;
   const int nchunk = (HB + GATHER_GROUPS - 1) / GATHER_GROUPS;
@@ -177,19 +194,24 @@ cudaError_t launch_permute(const moe_layer_s* L, const uint16_t* x, int T, int l
   const int K = L->K, E = L->E, W = (T + 31) / 32;
   const int S = L->S;
   const int rows = T * (K + S);
-  cudaError_t e = cudaMemsetAsync(s.bitmap, 0, sizeof(uint32_t) * size_t(E) * W, st);
+  const size_t nwords = size_t(E) * W;
+  cudaError_t e = launch_pdl(permute_clear_kernel, dim3(unsigned((nwords + 1023) / 1024)), dim3(256), 0, st,
+                             s.bitmap, nwords);
   if (e != cudaSuccess) return e;
-  permute_bitmap_kernel<<<(T * K + 255) / 256, 256, 0, st>>>(idx, T, K, E, W, s.bitmap, L->status);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  permute_count_kernel<<<E, 256, 0, st>>>(s.bitmap, W, s.wprefix, s.counts);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  permute_offsets_kernel<<<1, 256, 0, st>>>(s.counts, E, T, S, offsets);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  e = launch_pdl(permute_bitmap_kernel, dim3((T * K + 255) / 256), dim3(256), 0, st, idx, T, K, E, W, s.bitmap,
+                 L->status);
+  if (e != cudaSuccess) return e;
+  e = launch_pdl(permute_count_kernel, dim3(E), dim3(256), 0, st, static_cast<const uint32_t*>(s.bitmap), W,
+                 s.wprefix, s.counts);
+  if (e != cudaSuccess) return e;
+  e = launch_pdl(permute_offsets_kernel, dim3(1), dim3(256), 0, st, static_cast<const int32_t*>(s.counts), E, T, S,
+                 offsets);
+  if (e != cudaSuccess) return e;
   const int nchunk = (L->HB + GATHER_GROUPS - 1) / GATHER_GROUPS;
   const long long warps = static_cast<long long>(T) * nchunk;
-  permute_gather_kernel<<<unsigned((warps + 7) / 8), 256, 0, st>>>(x, T, ldx, L->H, idx, K, E, W, s.bitmap,
-                                                                   s.wprefix, offsets, S, rows, perm, inv, xq, xs);
-  return cudaGetLastError();
+  return launch_pdl(permute_gather_kernel, dim3(unsigned((warps + 7) / 8)), dim3(256), 0, st, x, T, ldx, L->H, idx,
+                    K, E, W, static_cast<const uint32_t*>(s.bitmap), static_cast<const uint32_t*>(s.wprefix),
+                    static_cast<const int32_t*>(offsets), S, rows, perm, inv, xq, xs);
 }
 
 // ---------------------------------------------------------------------------

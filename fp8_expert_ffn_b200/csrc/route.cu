@@ -109,6 +109,8 @@ __global__ void __launch_bounds__(R_THREADS, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  pdl_wait();   // set-up above overlaps the previous kernel; x and the partials are touched below
+  pdl_launch_dependents();
   const uint32_t tmem_base = tmem_base_s;
   uint32_t issued = 0;
 
@@ -269,6 +271,8 @@ __device__ __forceinline__ unsigned long long warp_max_u64(unsigned long long v)
 }
 
 __global__ void __launch_bounds__(256) route_topk_kernel(const TopkArgs a) {
+  pdl_wait();
+  pdl_launch_dependents();
   __shared__ unsigned long long s_key[8][256];   // per warp: the selection keys, for group scores
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   const int t = blockIdx.x * 8 + wid;
@@ -428,8 +432,8 @@ cudaError_t launch_route(const moe_layer_s* L, const uint16_t* x, int T, int ldx
   CUtensorMap tmX;
   if (!encode_tmap(&tmX, true, x, L->H, T, 1, uint64_t(ldx) * 2, 0)) return cudaErrorInvalidValue;
   dim3 grid((L->E + RN - 1) / RN, (T + RM - 1) / RM, S_eff);
-  route_tc_kernel<<<grid, R_THREADS, R_SMEM_DYN, st>>>(tmX, L->tm_router, T, L->E, kb_per, nkb, partial, L->status);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(route_tc_kernel, grid, dim3(R_THREADS), R_SMEM_DYN, st, tmX, L->tm_router, T, L->E,
+                             kb_per, nkb, partial, L->status);
   if (e != cudaSuccess) return e;
   TopkArgs ta;
   ta.partial = partial;
@@ -445,8 +449,7 @@ cudaError_t launch_route(const moe_layer_s* L, const uint16_t* x, int T, int ldx
   ta.idx = idx;
   ta.w = w;
   ta.logits_out = logits;
-  route_topk_kernel<<<(T + 7) / 8, 256, 0, st>>>(ta);
-  return cudaGetLastError();
+  return launch_pdl(route_topk_kernel, dim3((T + 7) / 8), dim3(256), 0, st, ta);
 }
 
 }  // namespace moe
