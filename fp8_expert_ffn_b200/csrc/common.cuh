@@ -244,6 +244,11 @@ __device__ __forceinline__ void ffma2(float& a0, float& a1, float v0, float v1, 
       : "f"(v0), "f"(v1), "f"(f));
 }
 
+// Pulls the line holding *p into this SM's L1 (no register result).
+__device__ __forceinline__ void prefetch_l1(const void* p) {
+  asm volatile("prefetch.global.L1 [%0];" ::"l"(p));
+}
+
 // ---------------------------------------------------------------- PDL
 // pdl_wait: returns once the kernels before this one on the stream have
 // completed and their writes are visible (a no-op without programmatic

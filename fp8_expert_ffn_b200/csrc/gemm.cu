@@ -145,6 +145,9 @@ __global__ void __launch_bounds__(THREADS, 1)
   __shared__ __align__(8) uint64_t tempty_bar[2];
   __shared__ __align__(8) uint64_t amax_bar[2][4];   // [tile parity][TMEM lane quarter]
   __shared__ __align__(8) uint64_t done_bar;
+  __shared__ __align__(8) uint64_t tinfo_full[2];    // tile list handed from warp 2 to the epilogue
+  __shared__ __align__(8) uint64_t tinfo_empty[2];
+  __shared__ int4 s_tinfo[2];
   __shared__ uint32_t tmem_base_s;
   __shared__ int s_prefix[MAX_GROUPS + 1];
   __shared__ float s_amax[2][2][BM];
@@ -166,6 +169,10 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int qq = 0; qq < 4; ++qq) mbar_init(&amax_bar[b][qq], 2);   // the two warps sharing those rows
     }
     mbar_init(&done_bar, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tinfo_full[b], 1);
+      mbar_init(&tinfo_empty[b], EPI_WARPS);
+    }
     s_abort_store = 0;
     s_consumed = 0;
     fence_mbar_init();
@@ -271,6 +278,34 @@ __global__ void __launch_bounds__(THREADS, 1)
       tc_commit(&done_bar);                 // all MMAs issued above have completed
       mbar_wait_drain(&done_bar, 0, p.status);
     }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ tile list
+    // Decodes this CTA's tiles one ahead of the epilogue into a two-slot
+    // ring and pulls each tile's first activation scales and its weight
+    // scales into L1, so a tile starts without global-memory latency.
+    uint32_t k = 0;
+    for (int i = blockIdx.x; i < total; i += gridDim.x, ++k) {
+      const uint32_t b = k & 1u, ph = (k >> 1) & 1u;
+      bool go = true;
+      if (lane == 0) go = mbar_wait(&tinfo_empty[b], ph ^ 1u, s_abort, p.status);
+      if (!__shfl_sync(0xFFFFFFFFu, go ? 1 : 0, 0)) break;
+      const TileInfo t = decode_tile(i, s_prefix, p.offsets, p.ngroups, p.ntn);
+      if (lane == 0) {
+        s_tinfo[b] = make_int4(t.g, t.nt, t.row0, t.nvalid);
+        mbar_arrive(&tinfo_full[b]);   // release: the slot's contents precede the arrival
+      }
+      for (int r = lane; r < t.nvalid; r += 32)
+        for (int kk = 0; kk < 4 && kk < p.nkb; ++kk) prefetch_l1(p.as + size_t(kk) * p.rows + t.row0 + r);
+      for (int kk = lane; kk < p.nkb; kk += 32) {
+        if (MODE == MODE_GATEUP) {
+          prefetch_l1(p.ws0 + (size_t(t.g) * p.ws_nb + t.nt) * p.ws_kb + kk);
+          prefetch_l1(p.ws1 + (size_t(t.g) * p.ws_nb + t.nt) * p.ws_kb + kk);
+        } else {
+          for (int hh = 0; hh < 2; ++hh)
+            prefetch_l1(p.ws0 + (size_t(t.g) * p.ws_nb + min(2 * t.nt + hh, p.ws_nb - 1)) * p.ws_kb + kk);
+        }
+      }
+    }
   }
   // ---------------------------------------------------- teardown (warpgroup 0)
   asm volatile("bar.sync 0;" ::: "memory");
@@ -295,7 +330,18 @@ __global__ void __launch_bounds__(THREADS, 1)
     uint32_t tile_iter = 0;
     bool ok = true;
     for (int i = blockIdx.x; ok && i < total; i += gridDim.x, ++tile_iter) {
-      const TileInfo t = decode_tile(i, s_prefix, p.offsets, p.ngroups, p.ntn);
+      TileInfo t;
+      {  // the tile, decoded ahead by warp 2
+        const uint32_t b = tile_iter & 1u;
+        if (!mbar_wait(&tinfo_full[b], (tile_iter >> 1) & 1u, s_abort, p.status)) break;
+        const int4 v = s_tinfo[b];
+        t.g = v.x;
+        t.nt = v.y;
+        t.row0 = v.z;
+        t.nvalid = v.w;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tinfo_empty[b]);
+      }
       const bool warp_active = q * 32 < t.nvalid;
       const bool valid = r_in < t.nvalid;
       const int row = t.row0 + r_in;
