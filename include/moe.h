@@ -34,6 +34,8 @@
  *     3*E*H*2 bytes, and nothing else);
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default);
  *     calls are asynchronous on that stream and never synchronise the host;
+ *     the kernels are chained with programmatic dependent launch (each one's
+ *     set-up overlaps the previous kernel's tail; stream order is kept);
  *   - bf16 tensors are passed as uint16_t bit patterns;
  *   - row strides (ld*) are in elements; every byte stride must be a
  *     multiple of 16 and every base pointer 16-byte aligned, else

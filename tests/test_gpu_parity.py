@@ -479,3 +479,21 @@ def test_router_variants_full_router():
     assert np.allclose(w.cpu().numpy()[keep], r.w[keep], rtol=2e-5, atol=1e-6)
     gs = sh.E // 8
     assert all(len(set(int(e) // gs for e in row)) <= 4 for row in got)
+
+
+# ----------------------------------------------------------------------------- degenerate batches
+
+@pytest.mark.parametrize("T", [1, 2])
+def test_single_token_batches(T):
+    """T = 1 and 2 on the full layer (one row per touched group, K+1 groups
+    per token): routing bit-exact and every output value within tolerance."""
+    wl, layer, c0 = get_case("decode")
+    x = c0.x_bits[:T]
+    c = gc.Case(layer, x, c0.dev)
+    r = moe.route(x, layer.router_w, layer.shape.K)
+    keep = ~r.near_tie
+    assert np.array_equal(c.np("idx")[keep], r.idx[keep])
+    off = c.np("offsets")
+    assert off[-1] == T * (layer.shape.K + 1) and (np.diff(off) >= 0).all()
+    ref = moe.token_outputs(x, layer, np.arange(T)[keep])
+    gc.assert_output_close(moe.bf16_to_f64(c.np("out"))[keep], ref, f"T={T}")
