@@ -198,6 +198,7 @@ moe_status moe_layer_create(const moe_layer_desc* d, const moe_weights* w, moe_l
   const size_t split_bytes = 3 * size_t(L->E) * L->H * sizeof(uint16_t);
   bool ok = cudaMalloc(&L->status, sizeof(uint32_t)) == cudaSuccess;
   ok = ok && cudaMalloc(&L->router_split, split_bytes) == cudaSuccess;
+  ok = ok && cudaMalloc(&L->splitk, sizeof(float) * size_t(kSplitMax) * kSplitRows * L->H) == cudaSuccess;
   ok = ok && cudaMemset(L->status, 0, sizeof(uint32_t)) == cudaSuccess;
   if (w->router_bias) {
     ok = ok && cudaMalloc(&L->router_bias, sizeof(float) * L->E) == cudaSuccess;
@@ -212,6 +213,7 @@ moe_status moe_layer_create(const moe_layer_desc* d, const moe_weights* w, moe_l
     cudaFree(L->status);
     cudaFree(L->router_split);
     cudaFree(L->router_bias);
+    cudaFree(L->splitk);
     delete L;
     return MOE_ERR_CUDA;
   }
@@ -223,6 +225,8 @@ moe_status moe_layer_destroy(moe_layer_t L) {
   if (!L) return MOE_OK;
   cudaError_t e = cudaFree(L->status);
   cudaError_t e2 = cudaFree(L->router_split);
+  const cudaError_t e4 = cudaFree(L->splitk);
+  if (e2 == cudaSuccess) e2 = e4;
   if (L->router_bias) {
     const cudaError_t e3 = cudaFree(L->router_bias);
     if (e2 == cudaSuccess) e2 = e3;

@@ -76,7 +76,11 @@ constexpr int stg_warp_bytes(int mode) { return mode == 1 ? 32 * 128 : 32 * 64; 
 constexpr int smem_dyn(int mode) { return STAGES * STAGE_BYTES + 1024 + EPI_WARPS * stg_warp_bytes(mode); }
 
 enum { MODE_GATEUP = 0, MODE_DOWN = 1 };
-enum { EPI_FUSED = 0, EPI_F32 = 1 };
+// EPI_SPLIT (down GEMM only): the tile's K blocks are split over ksplit
+// CTAs, each writes its promoted FP32 partial, and a second kernel sums the
+// partials in split order and rounds to bf16 (batches with fewer output
+// tiles than SMs, e.g. the dense FFN at decode sizes).
+enum { EPI_FUSED = 0, EPI_F32 = 1, EPI_SPLIT = 2 };
 
 struct GemmArgs {
   const int32_t* offsets;  // [ngroups + 1] row offsets of the groups
@@ -96,15 +100,27 @@ struct GemmArgs {
   int ld_y;
   float* out;              // test: promoted accumulators [rows][ld_out]
   int ld_out;
+  int ksplit;              // K splits per output tile (1 unless EPI_SPLIT)
+  float* part;             // EPI_SPLIT: partials [ksplit][rows][ld_y] fp32
   uint32_t* status;
 };
 
 struct TileInfo {
   int g, nt, row0, nvalid;
+  int kb0, kb1, sp;        // K blocks [kb0, kb1) of split sp
 };
 
+// K blocks of split sp of ksplit (contiguous, sizes differ by at most one).
+__device__ __forceinline__ void split_range(int sp, int ksplit, int nkb, int& kb0, int& kb1) {
+  kb0 = sp * nkb / ksplit;
+  kb1 = (sp + 1) * nkb / ksplit;
+}
+
+// Tile i of the list: output tile i / ksplit, split i % ksplit.
 __device__ __forceinline__ TileInfo decode_tile(int i, const int* s_prefix, const int* __restrict__ off, int ngroups,
-                                                int ntn) {
+                                                int ntn, int ksplit, int nkb) {
+  const int sp = i % ksplit;
+  i /= ksplit;
   int lo = 0, hi = ngroups - 1;
   while (lo < hi) {  // last group whose prefix is <= i
     const int mid = (lo + hi + 1) >> 1;
@@ -124,6 +140,8 @@ __device__ __forceinline__ TileInfo decode_tile(int i, const int* s_prefix, cons
   const int m = chunk * MCHUNK + (within - t.nt * mc);
   t.row0 = g0 + m * BM;
   t.nvalid = min(BM, n_g - m * BM);
+  t.sp = sp;
+  split_range(sp, ksplit, nkb, t.kb0, t.kb1);
   return t;
 }
 
@@ -147,7 +165,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   __shared__ __align__(8) uint64_t done_bar;
   __shared__ __align__(8) uint64_t tinfo_full[2];    // tile list handed from warp 2 to the epilogue
   __shared__ __align__(8) uint64_t tinfo_empty[2];
-  __shared__ int4 s_tinfo[2];
+  __shared__ int4 s_tinfo[2][2];
   __shared__ uint32_t tmem_base_s;
   __shared__ int s_prefix[MAX_GROUPS + 1];
   __shared__ float s_amax[2][2][BM];
@@ -213,7 +231,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = tmem_base_s;
-  const int total = s_prefix[p.ngroups];
+  const int total = s_prefix[p.ngroups] * p.ksplit;
   uint32_t issued = 0;
 
   // The two warpgroup kinds run to the end of the kernel on separate paths
@@ -227,8 +245,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       uint32_t it = 0;
       bool ok = true;
       for (int i = blockIdx.x; ok && i < total; i += gridDim.x) {
-        const TileInfo t = decode_tile(i, s_prefix, p.offsets, p.ngroups, p.ntn);
-        for (int kb = 0; kb < p.nkb; ++kb) {
+        const TileInfo t = decode_tile(i, s_prefix, p.offsets, p.ngroups, p.ntn, p.ksplit, p.nkb);
+        for (int kb = t.kb0; kb < t.kb1; ++kb) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1u;
           if (!mbar_wait(&empty_bar[s], ph ^ 1u, s_abort, p.status)) { ok = false; break; }
@@ -254,7 +272,9 @@ __global__ void __launch_bounds__(THREADS, 1)
       uint32_t it = 0, tb = 0;
       bool ok = true;
       for (int i = blockIdx.x; ok && i < total; i += gridDim.x) {
-        for (int kb = 0; kb < p.nkb; ++kb) {
+        int kb0, kb1;
+        split_range(i % p.ksplit, p.ksplit, p.nkb, kb0, kb1);
+        for (int kb = kb0; kb < kb1; ++kb) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1u;
           const uint32_t buf = tb & 1u, tph = (tb >> 1) & 1u;
@@ -289,14 +309,15 @@ __global__ void __launch_bounds__(THREADS, 1)
       bool go = true;
       if (lane == 0) go = mbar_wait(&tinfo_empty[b], ph ^ 1u, s_abort, p.status);
       if (!__shfl_sync(0xFFFFFFFFu, go ? 1 : 0, 0)) break;
-      const TileInfo t = decode_tile(i, s_prefix, p.offsets, p.ngroups, p.ntn);
+      const TileInfo t = decode_tile(i, s_prefix, p.offsets, p.ngroups, p.ntn, p.ksplit, p.nkb);
       if (lane == 0) {
-        s_tinfo[b] = make_int4(t.g, t.nt, t.row0, t.nvalid);
+        s_tinfo[b][0] = make_int4(t.g, t.nt, t.row0, t.nvalid);
+        s_tinfo[b][1] = make_int4(t.kb0, t.kb1, t.sp, 0);
         mbar_arrive(&tinfo_full[b]);   // release: the slot's contents precede the arrival
       }
       for (int r = lane; r < t.nvalid; r += 32)
-        for (int kk = 0; kk < 4 && kk < p.nkb; ++kk) prefetch_l1(p.as + size_t(kk) * p.rows + t.row0 + r);
-      for (int kk = lane; kk < p.nkb; kk += 32) {
+        for (int kk = t.kb0; kk < t.kb0 + 4 && kk < t.kb1; ++kk) prefetch_l1(p.as + size_t(kk) * p.rows + t.row0 + r);
+      for (int kk = t.kb0 + lane; kk < t.kb1; kk += 32) {
         if (MODE == MODE_GATEUP) {
           prefetch_l1(p.ws0 + (size_t(t.g) * p.ws_nb + t.nt) * p.ws_kb + kk);
           prefetch_l1(p.ws1 + (size_t(t.g) * p.ws_nb + t.nt) * p.ws_kb + kk);
@@ -334,11 +355,14 @@ __global__ void __launch_bounds__(THREADS, 1)
       {  // the tile, decoded ahead by warp 2
         const uint32_t b = tile_iter & 1u;
         if (!mbar_wait(&tinfo_full[b], (tile_iter >> 1) & 1u, s_abort, p.status)) break;
-        const int4 v = s_tinfo[b];
+        const int4 v = s_tinfo[b][0], u = s_tinfo[b][1];
         t.g = v.x;
         t.nt = v.y;
         t.row0 = v.z;
         t.nvalid = v.w;
+        t.kb0 = u.x;
+        t.kb1 = u.y;
+        t.sp = u.z;
         __syncwarp();
         if (lane == 0) mbar_arrive(&tinfo_empty[b]);
       }
@@ -363,31 +387,33 @@ __global__ void __launch_bounds__(THREADS, 1)
       // Scales stay off the critical path: lane l holds the weight scales
       // of K block (window + l), broadcast by a shuffle; the row's
       // activation scales are prefetched four K blocks ahead.
+      // (kr counts the tile's K blocks from its split's first, t.kb0)
       float wr0 = 0.0f, wr1 = 0.0f;
-      const float* asp = p.as + row;
       const size_t ast = size_t(p.rows);
+      const float* asp = p.as + size_t(t.kb0) * ast + row;
+      const int nk = t.kb1 - t.kb0;
       float pf0 = 0.0f, pf1 = 0.0f, pf2 = 0.0f, pf3 = 0.0f;
       if (valid) {
         pf0 = __ldg(asp);
-        if (p.nkb > 1) pf1 = __ldg(asp + ast);
-        if (p.nkb > 2) pf2 = __ldg(asp + 2 * ast);
-        if (p.nkb > 3) pf3 = __ldg(asp + 3 * ast);
+        if (nk > 1) pf1 = __ldg(asp + ast);
+        if (nk > 2) pf2 = __ldg(asp + 2 * ast);
+        if (nk > 3) pf3 = __ldg(asp + 3 * ast);
       }
 
-      for (int kb = 0; kb < p.nkb; ++kb) {
+      for (int kr = 0; kr < nk; ++kr) {
         const uint32_t buf = tb & 1u, tph = (tb >> 1) & 1u;
-        if ((kb & 31) == 0) {
-          const int k = kb + lane;
-          wr0 = k < p.nkb ? __ldg(w0 + k) : 0.0f;
-          wr1 = k < p.nkb ? __ldg(w1 + k) : 0.0f;
+        if ((kr & 31) == 0) {
+          const int k = t.kb0 + kr + lane;
+          wr0 = k < t.kb1 ? __ldg(w0 + k) : 0.0f;
+          wr1 = k < t.kb1 ? __ldg(w1 + k) : 0.0f;
         }
         const float sa = pf0;
         pf0 = pf1;
         pf1 = pf2;
         pf2 = pf3;
-        pf3 = (valid && kb + 4 < p.nkb) ? __ldg(asp + size_t(kb + 4) * ast) : 0.0f;
-        const float f0 = __shfl_sync(0xFFFFFFFFu, wr0, kb & 31) * sa;
-        const float f1 = __shfl_sync(0xFFFFFFFFu, wr1, kb & 31) * sa;
+        pf3 = (valid && kr + 4 < nk) ? __ldg(asp + size_t(kr + 4) * ast) : 0.0f;
+        const float f0 = __shfl_sync(0xFFFFFFFFu, wr0, kr & 31) * sa;
+        const float f1 = __shfl_sync(0xFFFFFFFFu, wr1, kr & 31) * sa;
         if (!mbar_wait(&tfull_bar[buf], tph, s_abort, p.status)) { ok = false; break; }
         tc_fence_after();
         if (warp_active) {
@@ -421,7 +447,15 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       if (!ok) break;
 
-      if (EPI == EPI_F32) {
+      if (EPI == EPI_SPLIT) {
+        // this split's promoted FP32 partial; the reduce kernel adds the splits
+        if (valid && nb < p.nb_count) {
+          float* dst = p.part + (size_t(t.sp) * p.rows + row) * p.ld_y + nb * 128;
+#pragma unroll
+          for (int v = 0; v < 32; ++v)
+            *reinterpret_cast<float4*>(dst + 4 * v) = make_float4(acc[4 * v], acc[4 * v + 1], acc[4 * v + 2], acc[4 * v + 3]);
+        }
+      } else if (EPI == EPI_F32) {
         if (valid) {
           float* dst = p.out + size_t(row) * p.ld_out;
           if (MODE == MODE_GATEUP) {
@@ -567,10 +601,36 @@ cudaError_t launch_gemm(const moe_layer_s* L, const CUtensorMap& tmA, const CUte
     configured = true;
   }
   // upper bound on the number of tiles: every group may add one partial row tile
-  const long long bound = (static_cast<long long>(a.rows) / BM + a.ngroups) * a.ntn;
+  const long long bound = (static_cast<long long>(a.rows) / BM + a.ngroups) * a.ntn * a.ksplit;
   const int grid = int(bound < L->num_sms ? bound : L->num_sms);
   if (grid <= 0) return cudaSuccess;
   return launch_pdl(grouped_gemm_kernel<MODE, EPI>, dim3(grid), dim3(THREADS), SMEM_DYN, st, tmA, tmB0, tmB1, tmY, a);
+}
+
+// y = bf16(sum over the splits s = 0..ks-1 of part[s]), 8 columns per thread.
+__global__ void __launch_bounds__(256) splitk_reduce_kernel(const float* __restrict__ part, int ks, size_t n,
+                                                            uint16_t* __restrict__ y) {
+  pdl_wait();
+  pdl_launch_dependents();
+  const size_t i = (size_t(blockIdx.x) * blockDim.x + threadIdx.x) * 8;
+  if (i >= n) return;
+  float v[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) v[j] = 0.0f;
+  for (int s = 0; s < ks; ++s) {
+    const float4 a = __ldg(reinterpret_cast<const float4*>(part + s * n + i));
+    const float4 b = __ldg(reinterpret_cast<const float4*>(part + s * n + i + 4));
+    v[0] += a.x;
+    v[1] += a.y;
+    v[2] += a.z;
+    v[3] += a.w;
+    v[4] += b.x;
+    v[5] += b.y;
+    v[6] += b.z;
+    v[7] += b.w;
+  }
+  *reinterpret_cast<uint4*>(y + i) =
+      make_uint4(bf16x2_rn(v[0], v[1]), bf16x2_rn(v[2], v[3]), bf16x2_rn(v[4], v[5]), bf16x2_rn(v[6], v[7]));
 }
 
 }  // namespace
@@ -588,6 +648,7 @@ static GemmArgs gateup_args(const moe_layer_s* L, const int32_t* offsets, int ro
   a.ws_nb = L->FB;
   a.ws_kb = L->HB;
   a.nb_count = L->FB;
+  a.ksplit = 1;
   a.status = L->status;
   return a;
 }
@@ -605,6 +666,7 @@ static GemmArgs down_args(const moe_layer_s* L, const int32_t* offsets, int rows
   a.ws_nb = L->HB;
   a.ws_kb = L->FB;
   a.nb_count = L->HB;
+  a.ksplit = 1;
   a.status = L->status;
   return a;
 }
@@ -632,7 +694,23 @@ cudaError_t launch_down(const moe_layer_s* L, const uint8_t* h, const float* hs,
   GemmArgs a = down_args(L, offsets, rows, hs);
   a.y = y;
   a.ld_y = L->H;
-  return launch_gemm<MODE_DOWN, EPI_FUSED>(L, tmH, L->tm_down, L->tm_down, tmY, a, st);
+  // Few output tiles for the SMs (a layer with one or two groups at small
+  // batches): split the K blocks and reduce the partials in a second kernel.
+  const long long tiles = (static_cast<long long>(rows) / BM + L->E + L->S) * a.ntn;   // groups with rows
+  int ks = 1;
+  if (L->splitk && rows <= kSplitRows && tiles * 2 <= L->num_sms) {
+    ks = int(L->num_sms / tiles);
+    ks = ks < kSplitMax ? ks : kSplitMax;
+    ks = ks < a.nkb / 4 ? ks : a.nkb / 4;   // at least 4 K blocks per split
+  }
+  if (ks < 2) return launch_gemm<MODE_DOWN, EPI_FUSED>(L, tmH, L->tm_down, L->tm_down, tmY, a, st);
+  a.ksplit = ks;
+  a.part = L->splitk;
+  cudaError_t e = launch_gemm<MODE_DOWN, EPI_SPLIT>(L, tmH, L->tm_down, L->tm_down, tmY, a, st);
+  if (e != cudaSuccess) return e;
+  const size_t n = size_t(rows) * L->H;
+  return launch_pdl(splitk_reduce_kernel, dim3(unsigned((n / 8 + 255) / 256)), dim3(256), 0, st,
+                    static_cast<const float*>(L->splitk), ks, n, y);
 }
 
 cudaError_t launch_test_gemm_f32(const moe_layer_s* L, int which, const uint8_t* a_ptr, const float* as,

@@ -22,6 +22,7 @@ struct moe_layer_s {
   uint32_t* status;  // device status word
   uint16_t* router_split;  // [3][E][H] bf16 terms of router_w (library-owned)
   float* router_bias;      // [E] selection-only bias (library-owned copy) or null
+  float* splitk;           // [kSplitMax][kSplitRows][H] fp32 partials of the split down GEMM
   CUtensorMap tm_router;   // over router_split, box 64 x 128 x 1
   CUtensorMap tm_gate;  // [E+1][F][ld_h] E4M3, box 128 x 128 x 1
   CUtensorMap tm_up;
@@ -64,6 +65,10 @@ cudaError_t launch_permute(const moe_layer_s* L, const uint16_t* x, int T, int l
 // Limits of the allocation-free permutation (moe_permute_noalloc).
 constexpr int kNoAllocMaxTokens = MOE_NOALLOC_MAX_TOKENS;
 constexpr int kNoAllocMaxExperts = 256;
+// Split-K of the down GEMM (batches with fewer output tiles than half the
+// SMs): at most kSplitMax splits over at most kSplitRows rows.
+constexpr int kSplitMax = 8;
+constexpr int kSplitRows = 256;
 cudaError_t launch_permute_noalloc(const moe_layer_s* L, const uint16_t* x, int T, int ldx, const int32_t* idx,
                                    int32_t* offsets, int32_t* perm, int32_t* inv, uint8_t* xq, float* xs,
                                    cudaStream_t st);

@@ -130,9 +130,14 @@ const char* moe_status_string(moe_status s);
  * encodes the weights' TMA descriptors once, allocates the 4-byte device
  * status word and writes the router weight as three bf16 terms
  * (hi + mid + lo == router_w exactly; the tensor-core router multiplies the
- * bf16 input by each term) and copies router_bias when given. Synchronises
- * the device once. On error *out is NULL. The router weight and bias are
- * read only here: a later change to either needs a new handle. */
+ * bf16 input by each term) and copies router_bias when given. It also
+ * allocates 8 x 256 x H fp32 of split-K partials (8 MB per 1024 of H): when a
+ * batch gives the down GEMM fewer output tiles than half the SMs (a layer
+ * with one or two groups at up to 256 rows), its K blocks are split over
+ * CTAs and a second kernel adds the partials in a fixed order, so calls on
+ * one handle must not overlap on the GPU. Synchronises the device once. On
+ * error *out is NULL. The router weight and bias are read only here: a later
+ * change to either needs a new handle. */
 moe_status moe_layer_create(const moe_layer_desc* desc, const moe_weights* w, moe_layer_t* out);
 
 /* Frees the handle (not the caller's weights). NULL is accepted. */

@@ -497,3 +497,32 @@ def test_single_token_batches(T):
     assert off[-1] == T * (layer.shape.K + 1) and (np.diff(off) >= 0).all()
     ref = moe.token_outputs(x, layer, np.arange(T)[keep])
     gc.assert_output_close(moe.bf16_to_f64(c.np("out"))[keep], ref, f"T={T}")
+
+
+# ----------------------------------------------------------------------------- split-K down GEMM
+
+def test_split_k_down_exact_integers():
+    """A one-group layer at a small batch has fewer down-GEMM output tiles than
+    SMs, so the down GEMM splits its K blocks over CTAs and a second kernel
+    adds the FP32 partials. With integer codes and unit scales every partial
+    and the total are exact, so y must be bf16(A Wd^T) bit for bit."""
+    sh = gen.LayerShape(H=512, E=1, K=1, F=2048, ld_f=2048, S=0)
+    rng = np.random.default_rng(41)
+    vals = np.array([0x00, 0x38, 0x40, 0x44, 0x48, 0xB8, 0xC0, 0xC4, 0xC8], np.uint8)
+    pick = lambda shape: vals[rng.integers(0, 9, shape)]
+    layer = gen.Layer(sh, gen.make_router(sh, 0), pick((1, sh.F, sh.H)), np.ones((1, sh.FB, sh.HB), np.float32),
+                      pick((1, sh.F, sh.H)), np.ones((1, sh.FB, sh.HB), np.float32),
+                      pick((1, sh.H, sh.ld_f)), np.ones((1, sh.HB, sh.FB), np.float32))
+    dev = tu.upload_layer(layer)
+    T = 64
+    hq = pick((T, sh.FB * 128))
+    hs = np.ones((sh.FB, T), np.float32)
+    off = np.array([0, T, T], np.int32)
+    y = torch.full((T, sh.H), float("nan"), dtype=torch.bfloat16, device="cuda")
+    fx.moe_down(dev, tu.to_device(hq), tu.to_device(hs), tu.to_device(off), T, y)
+    code, bits = fx.moe_get_device_status(dev)
+    assert code == fx.MOE_OK, f"{bits:#x}"
+    ints = moe.e4m3.decode(np.arange(256, dtype=np.uint8))
+    exact = ints[hq].astype(np.int64) @ ints[layer.w_down[0]].astype(np.int64).T
+    want = tu.bf16_bits(torch.tensor(exact.astype(np.float32)).to(torch.bfloat16))
+    assert np.array_equal(tu.bf16_bits(y), want)
