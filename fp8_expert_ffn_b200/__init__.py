@@ -19,7 +19,8 @@ MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_MISALIGNED, MOE_ERR_UNSUPPORTED, MOE_ERR_WO
 
 ENTRY_POINTS = ("moe_status_string", "moe_layer_create", "moe_layer_destroy", "moe_workspace_size", "moe_route",
                 "moe_permute", "moe_expert_ffn", "moe_combine", "moe_layer_forward", "moe_get_device_status",
-                "moe_gate_up", "moe_down", "moe_test_grouped_gemm_f32", "moe_permute_noalloc")
+                "moe_gate_up", "moe_down", "moe_test_grouped_gemm_f32", "moe_permute_noalloc",
+                "moe_kernels_per_forward")
 
 MOE_NOALLOC_MAX_TOKENS = 4096   # include/moe.h
 
@@ -76,6 +77,7 @@ def lib(build_if_missing: bool = True):
     L.moe_permute_noalloc.argtypes = [P, P, I, I, P, P, P, P, P, P, P]
     L.moe_down.argtypes = [P, P, P, P, I, P, P]
     L.moe_test_grouped_gemm_f32.argtypes = [P, I, P, P, P, I, P, P]
+    L.moe_kernels_per_forward.argtypes = [P, I]
     for name in ENTRY_POINTS:
         if name not in ("moe_status_string", "moe_workspace_size"):
             getattr(L, name).restype = I
@@ -152,6 +154,10 @@ class MoeLayer:
 
     def rows(self, T: int) -> int:
         return T * (self.K + self.S)
+
+
+def moe_kernels_per_forward(layer: MoeLayer, T: int) -> int:
+    return int(lib().moe_kernels_per_forward(layer.handle, T))
 
 
 def moe_workspace_size(layer: MoeLayer, T: int) -> int:

@@ -341,6 +341,12 @@ moe_status moe_layer_forward(moe_layer_t L, const uint16_t* x, int T, int ldx, u
   return from_cuda(e);
 }
 
+int moe_kernels_per_forward(moe_layer_t L, int T) {
+  if (!L || T <= 0 || T > kMaxT) return 0;
+  const int rows = T * (L->K + L->S);
+  return 2 + 5 + 1 + 1 + (down_ksplit(L, rows) > 1 ? 1 : 0) + 1;
+}
+
 moe_status moe_get_device_status(moe_layer_t L, void* stream, uint32_t* detail) {
   if (!L) return MOE_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);

@@ -635,6 +635,18 @@ __global__ void __launch_bounds__(256) splitk_reduce_kernel(const float* __restr
 
 }  // namespace
 
+// K splits of the down GEMM for `rows` rows: more than one only when the
+// batch has fewer output tiles than half the SMs (a layer with one or two
+// groups at small batches), at least 4 K blocks per split.
+int down_ksplit(const moe_layer_s* L, int rows) {
+  const int ntn = (L->HB + 1) / 2;
+  const long long tiles = (static_cast<long long>(rows) / BM + L->E + L->S) * ntn;   // groups with rows
+  if (!L->splitk || rows > kSplitRows || tiles * 2 > L->num_sms) return 1;
+  int ks = int(L->num_sms / tiles);
+  ks = ks < kSplitMax ? ks : kSplitMax;
+  return ks < L->FB / 4 ? ks : L->FB / 4;
+}
+
 static GemmArgs gateup_args(const moe_layer_s* L, const int32_t* offsets, int rows, const float* xs) {
   GemmArgs a = {};
   a.offsets = offsets;
@@ -694,15 +706,7 @@ cudaError_t launch_down(const moe_layer_s* L, const uint8_t* h, const float* hs,
   GemmArgs a = down_args(L, offsets, rows, hs);
   a.y = y;
   a.ld_y = L->H;
-  // Few output tiles for the SMs (a layer with one or two groups at small
-  // batches): split the K blocks and reduce the partials in a second kernel.
-  const long long tiles = (static_cast<long long>(rows) / BM + L->E + L->S) * a.ntn;   // groups with rows
-  int ks = 1;
-  if (L->splitk && rows <= kSplitRows && tiles * 2 <= L->num_sms) {
-    ks = int(L->num_sms / tiles);
-    ks = ks < kSplitMax ? ks : kSplitMax;
-    ks = ks < a.nkb / 4 ? ks : a.nkb / 4;   // at least 4 K blocks per split
-  }
+  const int ks = down_ksplit(L, rows);
   if (ks < 2) return launch_gemm<MODE_DOWN, EPI_FUSED>(L, tmH, L->tm_down, L->tm_down, tmY, a, st);
   a.ksplit = ks;
   a.part = L->splitk;

@@ -69,6 +69,7 @@ constexpr int kNoAllocMaxExperts = 256;
 // SMs): at most kSplitMax splits over at most kSplitRows rows.
 constexpr int kSplitMax = 8;
 constexpr int kSplitRows = 256;
+int down_ksplit(const moe_layer_s* L, int rows);
 cudaError_t launch_permute_noalloc(const moe_layer_s* L, const uint16_t* x, int T, int ldx, const int32_t* idx,
                                    int32_t* offsets, int32_t* perm, int32_t* inv, uint8_t* xq, float* xs,
                                    cudaStream_t st);

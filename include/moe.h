@@ -241,6 +241,11 @@ moe_status moe_layer_forward(moe_layer_t layer, const uint16_t* x, int T, int ld
  * If `detail` is not NULL it receives the raw status bits. */
 moe_status moe_get_device_status(moe_layer_t layer, void* stream, uint32_t* detail);
 
+/* Number of kernels moe_layer_forward launches for T tokens (route 2,
+ * permute 5, gate/up 1, down 1 plus 1 when its K blocks are split, combine
+ * 1); 0 for T = 0 or bad arguments. */
+int moe_kernels_per_forward(moe_layer_t layer, int T);
+
 /* Test hook for the grouped FP8 GEMM with per-128-K-block promotion: writes
  * the promoted FP32 accumulators instead of the fused epilogue.
  *   which = 0: gate/up GEMM; a = xq [rows][H], as = [H/128][rows];

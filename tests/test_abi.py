@@ -99,6 +99,7 @@ def test_create_rejects_bad_weights():
 def test_null_layer_everywhere():
     L = fx.lib()
     assert L.moe_workspace_size(None, 64) == 0
+    assert L.moe_kernels_per_forward(None, 64) == 0
     assert L.moe_layer_destroy(None) == fx.MOE_OK
     assert L.moe_route(None, 16, 1, 5120, 16, 16, None, 16, 1 << 20, None) == fx.MOE_ERR_INVALID_ARG
     assert L.moe_permute(None, 16, 1, 5120, 16, 16, 16, 16, 16, 16, 16, 1 << 20, None) == fx.MOE_ERR_INVALID_ARG

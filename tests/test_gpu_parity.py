@@ -526,3 +526,13 @@ def test_split_k_down_exact_integers():
     exact = ints[hq].astype(np.int64) @ ints[layer.w_down[0]].astype(np.int64).T
     want = tu.bf16_bits(torch.tensor(exact.astype(np.float32)).to(torch.bfloat16))
     assert np.array_equal(tu.bf16_bits(y), want)
+
+
+def test_kernels_per_forward():
+    """The launch count bench.py reports: 10 kernels per forward, 11 when the
+    down GEMM splits its K blocks (the dense FFN at T = 64)."""
+    _, _, c = get_case("decode")
+    assert fx.moe_kernels_per_forward(c.dev, c.T) == 10
+    assert fx.moe_kernels_per_forward(c.dev, 0) == 0
+    _, _, cd = get_case("dense")
+    assert fx.moe_kernels_per_forward(cd.dev, cd.T) == 11
