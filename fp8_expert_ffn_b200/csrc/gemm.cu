@@ -20,16 +20,20 @@
 //     quantises it per row per 128 channels (s = amax/448, E4M3 RNE), so the
 //     quantisation group is exactly one tile's channel block;
 //   down GEMM: tile = 128 rows x 256 output columns (two 128-column weight
-//     blocks); the epilogue rounds y to bf16.
+//     blocks); the epilogue rounds y to bf16 (or, with the K blocks split
+//     over CTAs for batches with few tiles, writes its FP32 partial).
 //
 // Kernel layout (one CTA per SM, persistent over a device-side tile list):
 //   warp 0      TMA producer: A tile 128 x 128 B, two B tiles 128 x 128 B per
 //               stage, 4-stage mbarrier ring (48 KB per stage, 128-byte swizzle)
 //   warp 1      TMEM allocator (512 columns) and single-thread MMA issuer;
 //               two 256-column TMEM buffers hold consecutive K-block partials
-//   warps 2-9   epilogue: warp w reads TMEM lanes 32*(w%4).. (its rows) and
+//   warp 2      decodes the tile list one tile ahead into a two-slot ring and
+//               pulls each tile's first scales into L1; warp 3 idles
+//   warps 4-11  epilogue: warp w reads TMEM lanes 32*(w%4).. (its rows) and
 //               one half of the 256 columns; promotion, then the fused
-//               SwiGLU+quant or bf16 store.
+//               SwiGLU+quant or bf16 tail, written through swizzled shared
+//               memory boxes by bulk tensor stores.
 // Tile order: per group (expert), chunks of up to 8 row tiles, then the
 // n tiles, then the row tiles of the chunk -- the row tiles that share one
 // weight tile run side by side, so that weight tile comes from HBM once.
