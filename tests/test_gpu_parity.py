@@ -536,3 +536,29 @@ def test_kernels_per_forward():
     assert fx.moe_kernels_per_forward(c.dev, 0) == 0
     _, _, cd = get_case("dense")
     assert fx.moe_kernels_per_forward(cd.dev, cd.T) == 11
+
+
+def test_forward_is_cuda_graph_capturable():
+    """The calls are asynchronous, allocate nothing and chain their kernels
+    with programmatic dependent launch: a captured moe_layer_forward replays
+    to the same bits as the eager call."""
+    wl, layer, c = get_case("toy_t2048")
+    sh = layer.shape
+    ws = tu.workspace(c.dev, c.T)
+    eager = torch.empty((c.T, sh.H), dtype=torch.bfloat16, device="cuda")
+    fx.moe_layer_forward(c.dev, c.x, c.T, sh.H, eager, sh.H, ws, ws.numel())
+    torch.cuda.synchronize()
+    out = torch.zeros_like(eager)
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            fx.moe_layer_forward(c.dev, c.x, c.T, sh.H, out, sh.H, ws, ws.numel())
+    for _ in range(2):
+        out.zero_()
+        g.replay()
+    torch.cuda.synchronize()
+    code, bits = fx.moe_get_device_status(c.dev)
+    assert code == fx.MOE_OK, f"{bits:#x}"
+    assert torch.equal(out.view(torch.int16), eager.view(torch.int16))
+    del g
