@@ -1,8 +1,7 @@
-"""Host logic of bench.py's multi-rank path on CPU: world size 2 over gloo.
-
-Each rank is an independent replica of the layer (no data-path collective);
-the job's throughput is all ranks' tokens over the slowest rank's time, and
-the reference arm runs on rank 0 only."""
+"""Host logic of bench.py on CPU: the multi-rank path at world size 2 over
+gloo (each rank an independent replica, no data-path collective; the job's
+throughput is all ranks' tokens over the slowest rank's time; the reference
+arm runs on rank 0 only) and the roofline numerators."""
 import json
 import os
 import socket
@@ -64,3 +63,33 @@ def test_reference_arm_other_ranks_exit_without_work():
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2",
                         "--steps", "3", "--warmup", "3"], env=env, capture_output=True, text=True, timeout=120)
     assert r.returncode == 0 and r.stdout.strip() == ""
+
+
+def test_algorithmic_work_closed_forms():
+    """The roofline numerators against closed forms of the full layer: one
+    touched expert's gate+up+down codes and scales are 23,598,720 bytes, and
+    a forward's expert FLOPs are rows x 2 x 3 x 5120 x 1536."""
+    import numpy as np
+    sys.path.insert(0, ROOT)
+    import bench
+    import gen
+    wl = gen.WORKLOADS["decode"]
+    sh = wl.shape
+    T = 64
+    rows = T * (sh.K + sh.S)
+    offsets = np.zeros(sh.E + 2, np.int64)
+    counts = np.zeros(sh.E + 1, np.int64)
+    counts[:T * sh.K // 2] = 2        # 256 experts touched by 512 routed rows
+    counts[sh.E] = T                  # the shared expert
+    offsets[1:] = np.cumsum(counts)
+    w = bench.algorithmic_work(wl, T, offsets)
+    assert w["touched_groups"] == 257 and w["rows"] == rows
+    act_gu = rows * (5120 + 160) + rows * (1536 + 48)
+    act_dn = rows * (1536 + 48) + rows * 5120 * 2
+    assert w["bytes"]["gate_up"] + w["bytes"]["down"] == 257 * 23_598_720 + act_gu + act_dn
+    assert w["flops"]["gate_up"] + w["flops"]["down"] == rows * 47_185_920
+    # a group with no rows costs nothing
+    counts[5] = 0
+    counts[6] = 4
+    offsets[1:] = np.cumsum(counts)
+    assert bench.algorithmic_work(wl, T, offsets)["touched_groups"] == 256
