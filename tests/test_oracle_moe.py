@@ -462,3 +462,100 @@ def test_route_layer_reads_the_layer_options():
     a = moe.route_layer(x, layer)
     b = moe.route(x, layer.router_w, sh.K)
     assert np.array_equal(a.idx, b.idx) and np.array_equal(a.w, b.w)
+
+
+# ----------------------------------------------------------------------------- BF16 cross-check path
+
+def _torch_bf16_via_f32(v64: np.ndarray) -> np.ndarray:
+    """torch's own casts, f64 -> f32 -> bf16 (each round to nearest even), back to f64."""
+    t = torch.from_numpy(np.ascontiguousarray(v64, np.float64))
+    return t.to(torch.float32).to(torch.bfloat16).to(torch.float64).numpy()
+
+
+def test_bf16_rounding_matches_torch_cast_bit_for_bit():
+    """f64_to_bf16_f64 against torch's cast on a stride sweep of every finite
+    fp32 bit pattern, every tie pattern (low half 0x8000, both parities of the
+    kept last bit), the patterns one below and one above each tie, subnormals
+    and the values that round up to infinity. A truncating cast, or one that
+    breaks ties away from zero, fails the tie and round-up cases."""
+    sweep = np.arange(0, 0x7F800000, 4099, dtype=np.uint64).astype(np.uint32)
+    hi = (np.arange(0, 0x7F80, 37, dtype=np.uint32) << 16)
+    ties = np.concatenate([hi | 0x8000, (hi | 0x10000) | 0x8000])            # even and odd kept bit
+    near = np.concatenate([ties - 1, ties + 1])
+    sub = np.arange(1, 0x00800000, 997, dtype=np.uint32)                      # fp32 subnormals
+    top = np.arange(0x7F7F0000, 0x7F800000, 97, dtype=np.uint32)              # includes round-up to inf
+    bits = np.concatenate([sweep, ties, near, sub, top])
+    bits = np.concatenate([bits, bits | 0x80000000])                          # both signs
+    v32 = bits.view(np.float32)
+    got = moe.f64_to_bf16_f64(v32.astype(np.float64))
+    want = _torch_bf16_via_f32(v32.astype(np.float64))
+    assert np.array_equal(got.view(np.uint64), want.view(np.uint64))
+    # ties go to the even bf16 mantissa: 1 + 2^-8 -> 1, 1 + 3 * 2^-8 -> 1 + 2^-6
+    assert moe.f64_to_bf16_f64(np.array([1 + 2.0 ** -8]))[0] == 1.0
+    assert moe.f64_to_bf16_f64(np.array([1 + 3 * 2.0 ** -8]))[0] == 1 + 2.0 ** -6
+    # f64 values between fp32 numbers are rounded to fp32 first (the checkpoint's fp32 dequantisation)
+    rng = np.random.default_rng(31)
+    v64 = rng.standard_normal(20000) * np.exp(rng.uniform(-30, 30, 20000))
+    assert np.array_equal(moe.f64_to_bf16_f64(v64).view(np.uint64), _torch_bf16_via_f32(v64).view(np.uint64))
+
+
+def _bf16_weight(codes, scales, n, k):
+    """W[n', k'] = bf16(fp32(decode(codes) * scale of its 128 x 128 block)) with explicit indices."""
+    d = torch_decode(codes)
+    w = np.zeros((n, k))
+    for i in range(n):
+        for j in range(k):
+            p = np.float32(np.float32(d[i, j]) * np.float32(scales[i // 128, j // 128]))
+            w[i, j] = float(torch.tensor(float(p), dtype=torch.float32).to(torch.bfloat16).item())
+    return w
+
+
+def test_bf16_layer_path_vs_textbook_loops():
+    """layer_forward_bf16 against loops over every index: weights bf16(q s),
+    no activation or h quantisation, FP64 sums, shared expert added with 1."""
+    layer, sh = small_layer(H=256, E=4, K=2, F=130, ld_f=144, seed=21)
+    rng = np.random.default_rng(22)
+    for name in ("s_gate", "s_up", "s_down"):
+        arr = getattr(layer, name)
+        arr *= rng.uniform(0.5, 2.0, arr.shape).astype(np.float32)
+    x = gen.f32_to_bf16_bits(rng.standard_normal((3, sh.H)).astype(np.float32))
+    got = moe.layer_forward_bf16(x, layer)
+    r = moe.route_layer(x, layer)
+    xf = moe.bf16_to_f64(x)
+    Wg = [_bf16_weight(layer.w_gate[g], layer.s_gate[g], sh.F, sh.H) for g in range(sh.E + 1)]
+    Wu = [_bf16_weight(layer.w_up[g], layer.s_up[g], sh.F, sh.H) for g in range(sh.E + 1)]
+    Wd = [_bf16_weight(layer.w_down[g], layer.s_down[g], sh.H, sh.F) for g in range(sh.E + 1)]
+    for t in range(3):
+        ref = np.zeros(sh.H)
+        for g, wt in [(int(r.idx[t, k]), float(r.w[t, k])) for k in range(sh.K)] + [(sh.E, 1.0)]:
+            h = np.zeros(sh.F)
+            for n in range(sh.F):
+                gsum = sum(xf[t, k] * Wg[g][n, k] for k in range(sh.H))
+                usum = sum(xf[t, k] * Wu[g][n, k] for k in range(sh.H))
+                h[n] = gsum / (1.0 + math.exp(-gsum)) * usum
+            for m in range(sh.H):
+                ref[m] += wt * sum(h[n] * Wd[g][m, n] for n in range(sh.F))
+        assert np.allclose(got[t], ref, rtol=1e-12, atol=1e-12 * np.abs(ref).max())
+
+
+def test_expert_down_rows_vs_textbook_loops():
+    """expert_down_rows over a multi-group offset vector (with empty groups and
+    a partial F block): each row uses its own group's down weights and scales."""
+    layer, sh = small_layer(H=256, E=5, K=2, F=130, ld_f=144, seed=23)
+    rng = np.random.default_rng(24)
+    layer.s_down *= rng.uniform(0.5, 2.0, layer.s_down.shape).astype(np.float32)
+    counts = np.array([2, 0, 3, 1, 0, 2])                # groups 0..E (E = shared)
+    off = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    rows = int(off[-1])
+    hq = rng.integers(0, 256, (rows, sh.F)).astype(np.uint8)
+    hq[(hq & 0x7F) == 0x7F] = 0x3C                       # no NaN codes
+    hs = rng.uniform(0.01, 0.1, (rows, sh.FB)).astype(np.float32)
+    y = moe.expert_down_rows(hq, hs, off, layer)
+    hd = torch_decode(hq)
+    for r in range(rows):
+        g = int(np.searchsorted(off, r, side="right") - 1)
+        dd = torch_decode(layer.w_down[g])
+        sd = layer.s_down[g]
+        ref = np.array([sum(hd[r, n] * float(hs[r, n // 128]) * dd[m, n] * float(sd[m // 128, n // 128])
+                            for n in range(sh.F)) for m in range(sh.H)])
+        assert np.allclose(y[r], ref, rtol=1e-12, atol=1e-12 * np.abs(ref).max()), f"row {r} (group {g})"
