@@ -17,3 +17,28 @@ def pytest_configure(config):
 def toy():
     import gen
     return gen.workload_inputs("toy")
+
+
+def _numpy_oracle():
+    """The numpy oracle under the names the C++ oracle's wrapper uses."""
+    from types import SimpleNamespace
+    from oracle import e4m3, moe
+    ns = SimpleNamespace(**{k: getattr(moe, k) for k in dir(moe) if not k.startswith("_")})
+    ns.e4m3_table = lambda: e4m3.DECODE
+    ns.e4m3_decode = e4m3.decode
+    ns.e4m3_encode = e4m3.encode
+    ns.name = "numpy"
+    return ns
+
+
+def _cpp_oracle():
+    from oracle import cpp
+    cpp.name = "cpp"
+    return cpp
+
+
+@pytest.fixture(scope="session", params=["numpy", "cpp"])
+def O(request):
+    """Each oracle pin runs on both oracle implementations: the numpy one and
+    the plain-loop C++ one."""
+    return _numpy_oracle() if request.param == "numpy" else _cpp_oracle()

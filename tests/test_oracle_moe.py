@@ -69,25 +69,25 @@ def small_layer(H=256, E=6, K=2, F=130, ld_f=144, seed=5):
 
 # ---------------------------------------------------------------- config
 
-def test_layer_shape_matches_pages():
+def test_layer_shape_matches_pages(O):
     cfg = json.load(open(os.path.join(GOLDEN, "dots3_text_config.json")))
     s = gen.DOTS3
     assert (s.H, s.E, s.K, s.F) == (cfg["hidden_size"], cfg["n_routed_experts"],
                                     cfg["num_experts_per_tok"], cfg["moe_intermediate_size"])
     assert cfg["shared_experts_intermediate_size"] == s.F and cfg["n_shared_experts"] == 1
-    assert cfg["weight_block_size"] == [moe.GROUP, moe.GROUP]
+    assert cfg["weight_block_size"] == [O.GROUP, O.GROUP]
     assert cfg["routed_scaling_factor"] == 1.0 and cfg["norm_topk_prob"] is True
     assert cfg["hidden_act"] == "silu" and cfg["mlp_bias"] is False
 
 
 # ---------------------------------------------------------------- quantiser
 
-def test_quantize_matches_textbook_rows():
+def test_quantize_matches_textbook_rows(O):
     rng = np.random.default_rng(2)
     v = (rng.standard_normal((5, 300)) * np.exp(rng.uniform(-3, 3, (5, 1)))).astype(np.float32)
     v[1, 128:256] = 0.0                       # an all-zero group
     v[2, 256:] = 0.0; v[2, 299] = -7.5        # partial last group (44 channels)
-    q, s = moe.quantize_rows(v)
+    q, s = O.quantize_rows(v)
     for r in range(5):
         tq, ts = textbook_quant_row(v[r])
         assert np.array_equal(q[r], tq) and np.array_equal(s[r], ts)
@@ -95,77 +95,77 @@ def test_quantize_matches_textbook_rows():
     assert s[2, 2] == np.float32(np.float32(7.5) / np.float32(448))
 
 
-def test_quantize_error_bound_and_amax_code():
+def test_quantize_error_bound_and_amax_code(O):
     rng = np.random.default_rng(3)
     v = (rng.standard_normal((64, 512)) * 3).astype(np.float32)
-    q, s = moe.quantize_rows(v)
-    d = moe.dequant_rows(q, s)
+    q, s = O.quantize_rows(v)
+    d = O.dequant_rows(q, s)
     # RNE to 3 mantissa bits: |error| <= 2^-4 |value| + half the subnormal step
     bound = np.abs(v) * 2.0 ** -4 + np.repeat(s, 128, axis=1) * 2.0 ** -10 * 1.0001
     assert np.all(np.abs(d - v) <= bound)
     # the amax element of every group lands on +-448
     for g in range(4):
         j = np.argmax(np.abs(v[:, g * 128:(g + 1) * 128]), axis=1) + g * 128
-        assert np.all(np.abs(e4m3.DECODE[q[np.arange(64), j]]) == 448.0)
+        assert np.all(np.abs(O.e4m3_table()[q[np.arange(64), j]]) == 448.0)
 
 
-def test_quantize_power_of_two_invariance():
+def test_quantize_power_of_two_invariance(O):
     rng = np.random.default_rng(4)
     v = rng.standard_normal((8, 256)).astype(np.float32)
-    q0, s0 = moe.quantize_rows(v)
+    q0, s0 = O.quantize_rows(v)
     for k in (-20, -3, 5, 30):
-        q1, s1 = moe.quantize_rows(v * np.float32(2.0 ** k))
+        q1, s1 = O.quantize_rows(v * np.float32(2.0 ** k))
         assert np.array_equal(q0, q1)
         assert np.array_equal(s1, s0 * np.float32(2.0 ** k))
 
 
 # ---------------------------------------------------------------- routing
 
-def test_topk_vs_full_sort_with_ties():
+def test_topk_vs_full_sort_with_ties(O):
     rng = np.random.default_rng(5)
     E, K = 24, 5
     logits = rng.standard_normal((200, E)).round(1)       # many exact ties
-    probs = moe.softmax(logits)
-    idx, w, gap = moe.select_topk(probs, K)
+    probs = O.softmax(logits)
+    idx, w, gap = O.select_topk(probs, K)
     for t in range(200):
         ref = sorted(range(E), key=lambda e: (-probs[t, e], e))
         assert list(idx[t]) == sorted(ref[:K])
         assert gap[t] == probs[t, ref[K - 1]] - probs[t, ref[K]]
 
 
-def test_route_weights_closed_form():
+def test_route_weights_closed_form(O):
     rng = np.random.default_rng(6)
     logits = rng.standard_normal((50, 32)) * 2
-    probs = moe.softmax(logits)
-    idx, w, _ = moe.select_topk(probs, 8)
+    probs = O.softmax(logits)
+    idx, w, _ = O.select_topk(probs, 8)
     assert np.allclose(w.sum(1), 1.0, atol=1e-15)
     sel = np.take_along_axis(logits, idx.astype(np.int64), 1)
     closed = np.exp(sel - sel.max(1, keepdims=True))
     closed /= closed.sum(1, keepdims=True)
     assert np.allclose(w, closed, rtol=1e-13, atol=0)
-    assert np.allclose(moe.softmax(logits), torch.softmax(torch.from_numpy(logits), 1).numpy(), rtol=1e-14)
+    assert np.allclose(O.softmax(logits), torch.softmax(torch.from_numpy(logits), 1).numpy(), rtol=1e-14)
 
 
-def test_route_zero_input():
+def test_route_zero_input(O):
     sh = gen.TOY
     x = np.zeros((4, sh.H), np.uint16)
-    r = moe.route(x, gen.make_router(sh, 0), sh.K)
+    r = O.route(x, gen.make_router(sh, 0), sh.K)
     assert np.array_equal(r.idx, np.tile(np.arange(sh.K), (4, 1)))
     assert np.all(r.w == 1.0 / sh.K)
 
 
-def test_near_tie_flag():
+def test_near_tie_flag(O):
     sh = gen.TOY
     router = np.zeros((sh.E, sh.H), np.float32)
     router[:, 0] = np.linspace(1.0, -1.0, sh.E).astype(np.float32)
     router[sh.K, 0] = router[sh.K - 1, 0]                # 4th and 5th exactly tied
     x = np.zeros((2, sh.H), np.uint16)
     x[:, 0] = gen.f32_to_bf16_bits(np.float32([1.0]))[0]
-    r = moe.route(x, router, sh.K)
+    r = O.route(x, router, sh.K)
     assert r.near_tie.all() and np.all(r.gap == 0)
     assert list(r.idx[0]) == list(range(sh.K))          # tie -> lower id
     router[sh.K, 0] = -1.0
-    assert not moe.route(x, router, sh.K).near_tie.any()
+    assert not O.route(x, router, sh.K).near_tie.any()
 
 
 # ---------------------------------------------------------------- permutation
@@ -194,11 +194,11 @@ def brute_permute(idx, E):
     return np.array(offsets), np.array(perm), inv
 
 
-def test_permute_vs_brute_and_invariants():
+def test_permute_vs_brute_and_invariants(O):
     rng = np.random.default_rng(7)
     T, K, E = 123, 4, 16
     idx = np.sort(np.array([rng.choice(E, K, replace=False) for _ in range(T)]), axis=1)
-    p = moe.permute(idx, E)
+    p = O.permute(idx, E)
     o, pr, iv = brute_permute(idx, E)
     assert np.array_equal(p.offsets, o) and np.array_equal(p.perm, pr) and np.array_equal(p.inv, iv)
     R = T * K
@@ -213,22 +213,22 @@ def test_permute_vs_brute_and_invariants():
     assert np.array_equal(p.perm[R:], np.arange(T))
 
 
-def test_permute_empty_and_all_to_one():
-    p = moe.permute(np.zeros((0, 4), np.int32), 8)
+def test_permute_empty_and_all_to_one(O):
+    p = O.permute(np.zeros((0, 4), np.int32), 8)
     assert p.offsets.tolist() == [0] * 10 and len(p.perm) == 0
     idx = np.tile(np.array([[3, 5]]), (6, 1))
-    p = moe.permute(idx, 8)
+    p = O.permute(idx, 8)
     assert p.offsets.tolist() == [0, 0, 0, 0, 6, 6, 12, 12, 12, 18]
 
 
 # ---------------------------------------------------------------- expert FFN
 
-def test_silu_matches_torch():
+def test_silu_matches_torch(O):
     g = np.linspace(-80, 80, 1001)
-    assert np.allclose(moe.silu(g), torch.nn.functional.silu(torch.from_numpy(g)).numpy(), rtol=1e-15, atol=1e-300)
+    assert np.allclose(O.silu(g), torch.nn.functional.silu(torch.from_numpy(g)).numpy(), rtol=1e-15, atol=1e-300)
 
 
-def test_expert_ffn_vs_textbook_loops():
+def test_expert_ffn_vs_textbook_loops(O):
     layer, sh = small_layer()
     rng = np.random.default_rng(8)
     # scales vary block to block so a transposed scale index shows up
@@ -236,40 +236,40 @@ def test_expert_ffn_vs_textbook_loops():
         arr = getattr(layer, name)
         arr *= rng.uniform(0.5, 2.0, arr.shape).astype(np.float32)
     x = gen.f32_to_bf16_bits(rng.standard_normal((3, sh.H)).astype(np.float32) * 2)
-    xf = moe.bf16_to_f64(x)
+    xf = O.bf16_to_f64(x)
     e = 4
-    tq, ts = moe.quantize_tokens(x)
-    f = moe.expert_ffn_rows(tq, ts, np.array([0] * (e + 1) + [3] * (sh.E + 1 - e)), layer, groups=[e])
+    tq, ts = O.quantize_tokens(x)
+    f = O.expert_ffn_rows(tq, ts, np.array([0] * (e + 1) + [3] * (sh.E + 1 - e)), layer, groups=[e])
     for r in range(3):
         ref = textbook_ffn(xf[r], layer.w_gate[e], layer.s_gate[e], layer.w_up[e], layer.s_up[e],
                            layer.w_down[e], layer.s_down[e], sh.F, sh.H)
         assert np.allclose(f["y"][r], ref, rtol=1e-12, atol=1e-12 * np.abs(ref).max())
 
 
-def test_gemm_exact_integers():
+def test_gemm_exact_integers(O):
     """Scales 1 and codes with values in {-4..4}: every dot product is an exact integer."""
     rng = np.random.default_rng(9)
     vals = np.array([0x00, 0x38, 0x40, 0x44, 0x48, 0xB8, 0xC0, 0xC4, 0xC8], np.uint8)  # 0,1,2,3,4,-1,-2,-3,-4
     ints = np.array([0, 1, 2, 3, 4, -1, -2, -3, -4])
     ia, ib = rng.integers(0, 9, (7, 384)), rng.integers(0, 9, (200, 384))
-    a = moe.dequant_rows(vals[ia], np.ones((7, 3), np.float32))
-    w = moe.dequant_block(vals[ib], np.ones((2, 3), np.float32), 200, 384)
+    a = O.dequant_rows(vals[ia], np.ones((7, 3), np.float32))
+    w = O.dequant_block(vals[ib], np.ones((2, 3), np.float32), 200, 384)
     assert np.array_equal(a @ w.T, (ints[ia] @ ints[ib].T).astype(np.float64))
 
 
-def test_dequant_block_index_order():
+def test_dequant_block_index_order(O):
     codes = np.full((256, 384), 0x38, np.uint8)           # all 1.0
     s = np.arange(6, dtype=np.float32).reshape(2, 3) + 1  # s[n_blk, k_blk]
-    w = moe.dequant_block(codes, s, 200, 300)
+    w = O.dequant_block(codes, s, 200, 300)
     assert w[0, 0] == 1 and w[0, 299] == 3 and w[199, 0] == 4 and w[130, 260] == 6
 
 
-def test_combine_closed_form():
+def test_combine_closed_form(O):
     T, K, H = 3, 2, 4
     y = np.arange((T * K + T) * H, dtype=np.float64).reshape(T * K + T, H)
     inv = np.array([[4, 0], [1, 5], [2, 3]])
     w = np.array([[0.25, 0.75], [0.5, 0.5], [1.0, 0.0]])
-    out = moe.combine(y, inv, w)
+    out = O.combine(y, inv, w)
     for t in range(T):
         ref = sum(w[t, k] * y[inv[t, k]] for k in range(K)) + y[T * K + t]
         assert np.array_equal(out[t], ref)
@@ -277,14 +277,14 @@ def test_combine_closed_form():
 
 # ---------------------------------------------------------------- whole layer
 
-def test_zero_input_gives_zero_output(toy):
+def test_zero_input_gives_zero_output(O, toy):
     _, layer, _ = toy
     x = np.zeros((5, layer.shape.H), np.uint16)
-    r = moe.layer_forward(x, layer)
+    r = O.layer_forward(x, layer)
     assert np.all(r["out"] == 0.0) and np.all(r["xs"] == 0) and not r["xq"].any()
 
 
-def test_one_hot_router_selects_one_expert(toy):
+def test_one_hot_router_selects_one_expert(O, toy):
     _, layer0, x = toy
     sh = layer0.shape
     estar, c0 = 11, 0
@@ -294,24 +294,24 @@ def test_one_hot_router_selects_one_expert(toy):
                       layer0.w_down, layer0.s_down)
     xs = x[:3].copy()
     xs[:, c0] = gen.f32_to_bf16_bits(np.float32([1.0]))[0]
-    r = moe.layer_forward(xs, layer)
+    r = O.layer_forward(xs, layer)
     assert np.array_equal(r["route"].idx, np.tile([0, 1, 2, estar], (3, 1)))
     assert np.all(r["route"].w[:, 3] == 1.0) and np.all(r["route"].w[:, :3] < 1e-80)
-    xf = moe.bf16_to_f64(xs)
+    xf = O.bf16_to_f64(xs)
     for t in range(3):
         ref = sum(textbook_ffn(xf[t], layer.w_gate[g], layer.s_gate[g], layer.w_up[g], layer.s_up[g],
                                layer.w_down[g], layer.s_down[g], sh.F, sh.H) for g in (estar, sh.E))
         assert np.allclose(r["out"][t], ref, rtol=1e-11, atol=1e-11 * np.abs(ref).max())
 
 
-def test_permuted_path_equals_direct_per_token(toy):
+def test_permuted_path_equals_direct_per_token(O, toy):
     _, layer, x = toy
-    r = moe.layer_forward(x, layer)
-    d = moe.token_outputs(x, layer, np.arange(x.shape[0]))
+    r = O.layer_forward(x, layer)
+    d = O.token_outputs(x, layer, np.arange(x.shape[0]))
     assert np.max(np.abs(d - r["out"])) <= 1e-12 * np.max(np.abs(r["out"]))
 
 
-def test_partial_blocks_equal_zero_padded_layer():
+def test_partial_blocks_equal_zero_padded_layer(O):
     """F=250 (not a multiple of 128) equals the same layer zero-padded to F=256."""
     layer, sh = small_layer(H=256, E=4, K=2, F=250, ld_f=256, seed=11)
     sp = gen.LayerShape(H=256, E=4, K=2, F=256, ld_f=256)
@@ -320,87 +320,87 @@ def test_partial_blocks_equal_zero_padded_layer():
                    layer.w_down.copy(), layer.s_down)
     lp.w_down[:, :, 250:] = 0
     x = gen.make_x(9, 256, 3)
-    a, b = moe.layer_forward(x, layer)["out"], moe.layer_forward(x, lp)["out"]
+    a, b = O.layer_forward(x, layer)["out"], O.layer_forward(x, lp)["out"]
     assert np.max(np.abs(a - b)) <= 1e-13 * np.max(np.abs(a))
     # the tail scale block was taken over the real rows only
     w = gen.normal_f32(11, gen.STREAM_GATE, 5 * 250 * 256, 1 / 16).reshape(5, 250, 256)
     assert layer.s_gate[2, 1, 0] == np.float32(np.abs(w[2, 128:250, :128]).max() / np.float32(448))
 
 
-def test_bf16_checkpoint_cross_check(toy):
+def test_bf16_checkpoint_cross_check(O, toy):
     _, layer, x = toy
-    a = moe.layer_forward(x, layer)["out"]
-    b = moe.layer_forward_bf16(x, layer)
+    a = O.layer_forward(x, layer)["out"]
+    b = O.layer_forward_bf16(x, layer)
     rel = np.linalg.norm(a - b) / np.linalg.norm(b)
     assert 1e-4 < rel < 8e-2
 
 
-def test_no_shared_expert_and_single_expert_layer():
+def test_no_shared_expert_and_single_expert_layer(O):
     """S = 0: no shared rows; E = 1, K = 1: the layer is that expert's FFN."""
     rng = np.random.default_rng(12)
     idx = np.sort(np.array([rng.choice(8, 2, replace=False) for _ in range(10)]), axis=1)
-    p = moe.permute(idx, 8, S=0)
+    p = O.permute(idx, 8, S=0)
     assert p.offsets[8] == p.offsets[9] == 20 and len(p.perm) == 20
     y = rng.standard_normal((20, 3))
     w = rng.uniform(size=(10, 2))
-    out = moe.combine(y, p.inv, w, S=0)
+    out = O.combine(y, p.inv, w, S=0)
     assert np.array_equal(out, sum(w[:, k:k + 1] * y[p.inv[:, k]] for k in range(2)))
     sh = gen.LayerShape(H=256, E=1, K=1, F=200, ld_f=208, S=0)
     layer = gen.make_layer(sh, 9)
     assert layer.w_gate.shape[0] == 1
     x = gen.make_x(5, 256, 2)
-    r = moe.layer_forward(x, layer)
+    r = O.layer_forward(x, layer)
     assert np.all(r["route"].idx == 0) and np.all(r["route"].w == 1.0)
-    xf = moe.bf16_to_f64(x)
+    xf = O.bf16_to_f64(x)
     for t in range(5):
         ref = textbook_ffn(xf[t], layer.w_gate[0], layer.s_gate[0], layer.w_up[0], layer.s_up[0],
                            layer.w_down[0], layer.s_down[0], sh.F, sh.H)
         assert np.allclose(r["out"][t], ref, rtol=1e-11, atol=1e-11 * np.abs(ref).max())
 
 
-def test_routed_scaling_in_oracle():
+def test_routed_scaling_in_oracle(O):
     sh = gen.TOY
     x = gen.make_x(6, sh.H, 1)
-    r1 = moe.route(x, gen.make_router(sh, 0), sh.K)
-    r2 = moe.route(x, gen.make_router(sh, 0), sh.K, routed_scaling=2.5)
+    r1 = O.route(x, gen.make_router(sh, 0), sh.K)
+    r2 = O.route(x, gen.make_router(sh, 0), sh.K, routed_scaling=2.5)
     assert np.array_equal(r1.idx, r2.idx) and np.allclose(r2.w, 2.5 * r1.w, rtol=1e-15)
 
 
 # ----------------------------------------------------------------------------- router variants
 
-def test_group_limited_hand_example():
+def test_group_limited_hand_example(O):
     """8 experts in 4 groups of 2, two groups eligible, top-3 (worked by hand):
     group maxima 0.30, 0.20, 0.03, 0.25 keep groups 0 and 3, so expert 2
     (0.20, group 1) loses to expert 6 (0.04); ungrouped the top-3 is 0, 2, 7."""
     p = np.array([[0.30, 0.01, 0.20, 0.15, 0.02, 0.03, 0.04, 0.25]])
-    idx, w, gap = moe.select_topk(p, 3, n_group=4, topk_group=2)
+    idx, w, gap = O.select_topk(p, 3, n_group=4, topk_group=2)
     assert idx.tolist() == [[0, 6, 7]]
     np.testing.assert_allclose(w[0], np.array([0.30, 0.04, 0.25]) / 0.59, rtol=1e-15)
     assert gap[0] == pytest.approx(min(0.04 - 0.01, 0.25 - 0.20))
-    idx0, _, _ = moe.select_topk(p, 3)
+    idx0, _, _ = O.select_topk(p, 3)
     assert idx0.tolist() == [[0, 2, 7]]
 
 
-def test_group_limited_reduces_to_ungrouped():
+def test_group_limited_reduces_to_ungrouped(O):
     rng = np.random.default_rng(21)
     p = rng.dirichlet(np.ones(16), size=64)
-    ref = moe.select_topk(p, 4)
+    ref = O.select_topk(p, 4)
     # every group eligible
-    got = moe.select_topk(p, 4, n_group=4, topk_group=4)
+    got = O.select_topk(p, 4, n_group=4, topk_group=4)
     assert np.array_equal(got[0], ref[0]) and np.allclose(got[1], ref[1])
     # one expert per group, K groups eligible: the K best experts
-    got = moe.select_topk(p, 4, n_group=16, topk_group=4)
+    got = O.select_topk(p, 4, n_group=16, topk_group=4)
     assert np.array_equal(got[0], ref[0]) and np.allclose(got[1], ref[1])
 
 
-def test_group_limited_properties():
+def test_group_limited_properties(O):
     """Checked on the output only: at most topk_group groups are used, every
     dropped group's best member is no better than every kept group's, and no
     eligible expert left out beats a selected one."""
     rng = np.random.default_rng(22)
     E, G, TG, K = 64, 8, 3, 6
     p = rng.dirichlet(np.ones(E) * 0.3, size=200)
-    idx, w, _ = moe.select_topk(p, K, n_group=G, topk_group=TG)
+    idx, w, _ = O.select_topk(p, K, n_group=G, topk_group=TG)
     gs = E // G
     for t in range(len(p)):
         used = set(int(e) // gs for e in idx[t])
@@ -417,21 +417,21 @@ def test_group_limited_properties():
         assert w[t].sum() == pytest.approx(1.0)
 
 
-def test_selection_bias_selects_but_does_not_weight():
+def test_selection_bias_selects_but_does_not_weight(O):
     rng = np.random.default_rng(23)
     E, K = 32, 4
     logits = rng.normal(0, 1, (50, E))
     p = np.exp(logits - logits.max(1, keepdims=True))
     p /= p.sum(1, keepdims=True)
-    ref = moe.select_topk(p, K)
+    ref = O.select_topk(p, K)
     # a constant bias changes nothing
-    got = moe.select_topk(p, K, bias=np.full(E, 0.7))
+    got = O.select_topk(p, K, bias=np.full(E, 0.7))
     assert np.array_equal(got[0], ref[0]) and np.allclose(got[1], ref[1], rtol=1e-14)
     # a large negative bias removes an expert, a large positive one forces one in
     b = np.zeros(E)
     b[5] = -1000.0
     b[9] = 1000.0
-    idx, w, _ = moe.select_topk(p, K, bias=b)
+    idx, w, _ = O.select_topk(p, K, bias=b)
     assert (idx != 5).all() and (idx == 9).any(axis=1).all()
     for t in range(len(p)):
         # the weights are the unbiased probabilities of the selected experts,
@@ -441,26 +441,26 @@ def test_selection_bias_selects_but_does_not_weight():
         np.testing.assert_allclose(w[t], ex / ex.sum(), rtol=1e-12)
 
 
-def test_norm_topk_off_keeps_the_softmax_weights():
+def test_norm_topk_off_keeps_the_softmax_weights(O):
     import scipy.special
     rng = np.random.default_rng(24)
     sh = gen.TOY
     x = gen.make_x(9, sh.H, 2)
     router = gen.make_router(sh, 0)
-    r = moe.route(x, router, sh.K, routed_scaling=2.0, norm_topk=False)
-    full = scipy.special.softmax(moe.bf16_to_f64(x) @ router.astype(np.float64).T, axis=1)
+    r = O.route(x, router, sh.K, routed_scaling=2.0, norm_topk=False)
+    full = scipy.special.softmax(O.bf16_to_f64(x) @ router.astype(np.float64).T, axis=1)
     np.testing.assert_allclose(r.w, 2.0 * np.take_along_axis(full, r.idx.astype(np.int64), 1), rtol=1e-12)
     assert (r.w.sum(1) < 2.0).all()
-    r1 = moe.route(x, router, sh.K)
+    r1 = O.route(x, router, sh.K)
     assert np.array_equal(r.idx, r1.idx)
 
 
-def test_route_layer_reads_the_layer_options():
+def test_route_layer_reads_the_layer_options(O):
     sh = gen.TOY
     x = gen.make_x(10, sh.H, 1)
     wl, layer, _ = gen.workload_inputs("toy")
-    a = moe.route_layer(x, layer)
-    b = moe.route(x, layer.router_w, sh.K)
+    a = O.route_layer(x, layer)
+    b = O.route(x, layer.router_w, sh.K)
     assert np.array_equal(a.idx, b.idx) and np.array_equal(a.w, b.w)
 
 
@@ -472,7 +472,7 @@ def _torch_bf16_via_f32(v64: np.ndarray) -> np.ndarray:
     return t.to(torch.float32).to(torch.bfloat16).to(torch.float64).numpy()
 
 
-def test_bf16_rounding_matches_torch_cast_bit_for_bit():
+def test_bf16_rounding_matches_torch_cast_bit_for_bit(O):
     """f64_to_bf16_f64 against torch's cast on a stride sweep of every finite
     fp32 bit pattern, every tie pattern (low half 0x8000, both parities of the
     kept last bit), the patterns one below and one above each tie, subnormals
@@ -487,16 +487,16 @@ def test_bf16_rounding_matches_torch_cast_bit_for_bit():
     bits = np.concatenate([sweep, ties, near, sub, top])
     bits = np.concatenate([bits, bits | 0x80000000])                          # both signs
     v32 = bits.view(np.float32)
-    got = moe.f64_to_bf16_f64(v32.astype(np.float64))
+    got = O.f64_to_bf16_f64(v32.astype(np.float64))
     want = _torch_bf16_via_f32(v32.astype(np.float64))
     assert np.array_equal(got.view(np.uint64), want.view(np.uint64))
     # ties go to the even bf16 mantissa: 1 + 2^-8 -> 1, 1 + 3 * 2^-8 -> 1 + 2^-6
-    assert moe.f64_to_bf16_f64(np.array([1 + 2.0 ** -8]))[0] == 1.0
-    assert moe.f64_to_bf16_f64(np.array([1 + 3 * 2.0 ** -8]))[0] == 1 + 2.0 ** -6
+    assert O.f64_to_bf16_f64(np.array([1 + 2.0 ** -8]))[0] == 1.0
+    assert O.f64_to_bf16_f64(np.array([1 + 3 * 2.0 ** -8]))[0] == 1 + 2.0 ** -6
     # f64 values between fp32 numbers are rounded to fp32 first (the checkpoint's fp32 dequantisation)
     rng = np.random.default_rng(31)
     v64 = rng.standard_normal(20000) * np.exp(rng.uniform(-30, 30, 20000))
-    assert np.array_equal(moe.f64_to_bf16_f64(v64).view(np.uint64), _torch_bf16_via_f32(v64).view(np.uint64))
+    assert np.array_equal(O.f64_to_bf16_f64(v64).view(np.uint64), _torch_bf16_via_f32(v64).view(np.uint64))
 
 
 def _bf16_weight(codes, scales, n, k):
@@ -510,7 +510,7 @@ def _bf16_weight(codes, scales, n, k):
     return w
 
 
-def test_bf16_layer_path_vs_textbook_loops():
+def test_bf16_layer_path_vs_textbook_loops(O):
     """layer_forward_bf16 against loops over every index: weights bf16(q s),
     no activation or h quantisation, FP64 sums, shared expert added with 1."""
     layer, sh = small_layer(H=256, E=4, K=2, F=130, ld_f=144, seed=21)
@@ -519,9 +519,9 @@ def test_bf16_layer_path_vs_textbook_loops():
         arr = getattr(layer, name)
         arr *= rng.uniform(0.5, 2.0, arr.shape).astype(np.float32)
     x = gen.f32_to_bf16_bits(rng.standard_normal((3, sh.H)).astype(np.float32))
-    got = moe.layer_forward_bf16(x, layer)
-    r = moe.route_layer(x, layer)
-    xf = moe.bf16_to_f64(x)
+    got = O.layer_forward_bf16(x, layer)
+    r = O.route_layer(x, layer)
+    xf = O.bf16_to_f64(x)
     Wg = [_bf16_weight(layer.w_gate[g], layer.s_gate[g], sh.F, sh.H) for g in range(sh.E + 1)]
     Wu = [_bf16_weight(layer.w_up[g], layer.s_up[g], sh.F, sh.H) for g in range(sh.E + 1)]
     Wd = [_bf16_weight(layer.w_down[g], layer.s_down[g], sh.H, sh.F) for g in range(sh.E + 1)]
@@ -538,7 +538,7 @@ def test_bf16_layer_path_vs_textbook_loops():
         assert np.allclose(got[t], ref, rtol=1e-12, atol=1e-12 * np.abs(ref).max())
 
 
-def test_expert_down_rows_vs_textbook_loops():
+def test_expert_down_rows_vs_textbook_loops(O):
     """expert_down_rows over a multi-group offset vector (with empty groups and
     a partial F block): each row uses its own group's down weights and scales."""
     layer, sh = small_layer(H=256, E=5, K=2, F=130, ld_f=144, seed=23)
@@ -550,7 +550,7 @@ def test_expert_down_rows_vs_textbook_loops():
     hq = rng.integers(0, 256, (rows, sh.F)).astype(np.uint8)
     hq[(hq & 0x7F) == 0x7F] = 0x3C                       # no NaN codes
     hs = rng.uniform(0.01, 0.1, (rows, sh.FB)).astype(np.float32)
-    y = moe.expert_down_rows(hq, hs, off, layer)
+    y = O.expert_down_rows(hq, hs, off, layer)
     hd = torch_decode(hq)
     for r in range(rows):
         g = int(np.searchsorted(off, r, side="right") - 1)
