@@ -33,9 +33,13 @@ EncodeTiledFn encode_fn() {
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+std::mutex g_device_setup_mutex;
+
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 }  // namespace
+
+std::mutex& device_setup_mutex() { return g_device_setup_mutex; }
 
 bool encode_tmap(CUtensorMap* tm, bool bf16, const void* base, uint64_t inner, uint64_t rows, uint64_t depth,
                  uint64_t ld_bytes, uint64_t depth_stride_bytes, bool force3d) {

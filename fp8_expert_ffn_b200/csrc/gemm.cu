@@ -591,8 +591,8 @@ template <int MODE, int EPI>
 cudaError_t launch_gemm(const moe_layer_s* L, const CUtensorMap& tmA, const CUtensorMap& tmB0,
                         const CUtensorMap& tmB1, const CUtensorMap& tmY, const GemmArgs& a, cudaStream_t st) {
   constexpr int SMEM_DYN = smem_dyn(MODE);
-  static bool configured = false;  // per process; the attribute is per function
-  if (!configured) {
+  static std::atomic<bool> configured[kMaxDevices];   // the attribute is per device
+  cudaError_t ce = once_per_device(configured, []() {
     // setmaxnreg.inc waits until the registers it asks for are free; they
     // come only from this CTA's launch allocation, so refuse to launch a
     // build whose register count cannot fund the split.
@@ -600,10 +600,10 @@ cudaError_t launch_gemm(const moe_layer_s* L, const CUtensorMap& tmA, const CUte
     cudaError_t e = cudaFuncGetAttributes(&fa, grouped_gemm_kernel<MODE, EPI>);
     if (e != cudaSuccess) return e;
     if (fa.numRegs * THREADS < 128 * PRODUCER_REGS + 256 * EPILOGUE_REGS) return cudaErrorInvalidConfiguration;
-    e = cudaFuncSetAttribute(grouped_gemm_kernel<MODE, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_DYN);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+    return cudaFuncSetAttribute(grouped_gemm_kernel<MODE, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                SMEM_DYN);
+  });
+  if (ce != cudaSuccess) return ce;
   // upper bound on the number of tiles: every group may add one partial row tile
   const long long bound = (static_cast<long long>(a.rows) / BM + a.ngroups) * a.ntn * a.ksplit;
   const int grid = int(bound < L->num_sms ? bound : L->num_sms);

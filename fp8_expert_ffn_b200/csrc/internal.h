@@ -4,8 +4,10 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstddef>
 #include <cstdint>
+#include <mutex>
 
 #include "../../include/moe.h"
 
@@ -105,6 +107,26 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
   cfg.attrs = at;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
+// Kernel attributes (the dynamic shared-memory limit) are set per device:
+// once_per_device runs `setup` the first time it is called with each device
+// current and records success in done[device]; a failed setup is retried on
+// the next call. Safe to call from several host threads.
+constexpr int kMaxDevices = 64;
+std::mutex& device_setup_mutex();
+template <typename F>
+cudaError_t once_per_device(std::atomic<bool>* done, F setup) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  if (done[dev].load(std::memory_order_acquire)) return cudaSuccess;
+  std::lock_guard<std::mutex> lock(device_setup_mutex());
+  if (done[dev].load(std::memory_order_relaxed)) return cudaSuccess;
+  e = setup();
+  if (e == cudaSuccess) done[dev].store(true, std::memory_order_release);
+  return e;
 }
 
 bool encode_tmap_store(CUtensorMap* tm, bool bf16, const void* base, uint64_t inner, uint64_t rows, uint64_t ld_bytes);

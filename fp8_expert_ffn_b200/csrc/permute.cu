@@ -228,7 +228,6 @@ namespace {
 constexpr int kNoAllocWords = kNoAllocMaxExperts * ((kNoAllocMaxTokens + 31) / 32);
 static __device__ __align__(256) uint32_t g_permute_scratch[2 * kNoAllocWords + kNoAllocMaxExperts];
 
-constexpr int kMaxDevices = 64;
 uint32_t* g_scratch_addr[kMaxDevices] = {};
 std::mutex g_scratch_mutex;
 

@@ -419,12 +419,11 @@ cudaError_t launch_router_split(const float* w, int E, int H, uint16_t* out, cud
 
 cudaError_t launch_route(const moe_layer_s* L, const uint16_t* x, int T, int ldx, int32_t* idx, float* w,
                          float* logits, float* partial, cudaStream_t st) {
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(route_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, R_SMEM_DYN);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  static std::atomic<bool> configured[kMaxDevices];   // the attribute is per device
+  cudaError_t ce = once_per_device(configured, []() {
+    return cudaFuncSetAttribute(route_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, R_SMEM_DYN);
+  });
+  if (ce != cudaSuccess) return ce;
   const int nkb = L->H / RK;
   const int S = route_splits(L, T);
   const int kb_per = (nkb + S - 1) / S;

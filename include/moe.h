@@ -29,9 +29,13 @@
  *
  * Conventions for every call:
  *   - all data pointers are DEVICE pointers owned by the caller; the library
- *     never allocates after moe_layer_create (which allocates a 4-byte
- *     device status word and the router weight's three-term bf16 split,
- *     3*E*H*2 bytes, and nothing else);
+ *     never allocates after moe_layer_create, which allocates, per handle:
+ *     a 4-byte device status word; the router weight's three-term bf16
+ *     split, 3*E*H*2 bytes; the split-K partials of the down GEMM,
+ *     8*256*H*4 bytes (42 MB at H = 5120); and, when a router bias is
+ *     given, an E*4-byte copy of it. Nothing else is allocated (the one
+ *     file-scope array of moe_permute_noalloc, below, is part of the
+ *     library image, not an allocation);
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default);
  *     calls are asynchronous on that stream and never synchronise the host;
  *     the kernels are chained with programmatic dependent launch (each one's
@@ -123,10 +127,13 @@ typedef struct {
 
 typedef struct moe_layer_s* moe_layer_t;
 
-/* Static description of a status code (never NULL). */
+/* Static description of a status code (never NULL). Library plumbing: no
+ * counterpart on the pages. */
 const char* moe_status_string(moe_status s);
 
-/* Validates desc/weights, queries the current device (must be sm_100),
+/* Creates the handle of one MoE layer of the shape moe_layer_desc describes
+ * (Dots3NoteTextConfig, transformers docs page "Dots 3 Note Preview").
+ * Validates desc/weights, queries the current device (must be sm_100),
  * encodes the weights' TMA descriptors once, allocates the 4-byte device
  * status word and writes the router weight as three bf16 terms
  * (hi + mid + lo == router_w exactly; the tensor-core router multiplies the
@@ -140,11 +147,13 @@ const char* moe_status_string(moe_status s);
  * change to either needs a new handle. */
 moe_status moe_layer_create(const moe_layer_desc* desc, const moe_weights* w, moe_layer_t* out);
 
-/* Frees the handle (not the caller's weights). NULL is accepted. */
+/* Frees the handle (not the caller's weights). NULL is accepted. Library
+ * plumbing: no counterpart on the pages. */
 moe_status moe_layer_destroy(moe_layer_t layer);
 
 /* Bytes of workspace that moe_layer_forward needs for T tokens; it also
- * covers the scratch of moe_permute and moe_expert_ffn. 0 on bad input. */
+ * covers the scratch of moe_permute and moe_expert_ffn. 0 on bad input.
+ * Library plumbing: no counterpart on the pages. */
 size_t moe_workspace_size(moe_layer_t layer, int T);
 
 /* Router: logits = x . router_w^T in FP32, p = softmax over the E experts,
@@ -164,6 +173,10 @@ moe_status moe_route(moe_layer_t layer, const uint16_t* x, int T, int ldx, int32
                      float* router_logits, void* ws, size_t ws_bytes, void* stream);
 
 /* Token permutation by expert with fused activation quantisation.
+ * On one GPU this is the "dispatch" of the DeepEP transport that the SGLang
+ * cookbook "Dots3-Note" names for the MoE layer ("2. Configuration Tips");
+ * the activations are quantised dynamically, per token per 128 channels, to
+ * E4M3 (transformers PR #47844, "What does this PR do?").
  * Counting sort of the T*K (token, slot) pairs by expert id, stable in token
  * order; with n_shared = 1, group E (shared expert) holds rows [T*K, T*K+T)
  * in token order (with n_shared = 0 it is empty).
@@ -202,8 +215,13 @@ moe_status moe_permute_noalloc(moe_layer_t layer, const uint16_t* x, int T, int 
                                int32_t* offsets, int32_t* perm, int32_t* inv, uint8_t* xq, float* xs,
                                void* stream);
 
-/* Grouped expert FFN over the permuted rows: for each group g and row r in
- * it, h = silu(xq Wg_g^T) * (xq Wu_g^T) with per-128-K-block scale promotion,
+/* Grouped expert FFN over the permuted rows. The experts are SwiGLU FFNs
+ * (Dots3NoteTextConfig of the transformers docs page "Dots 3 Note Preview":
+ * hidden_act silu, mlp_bias False, moe_intermediate_size 1536; model card
+ * dots-studio/dots3-note-prev, "Model Overview": FFN 1536 per expert) with
+ * fine-grained FP8 weights (transformers PR #47844, "What does this PR do?":
+ * E4M3, one scale per 128 x 128 block, dynamic activations). For each group
+ * g and row r in it, h = silu(xq Wg_g^T) * (xq Wu_g^T) with per-128-K-block scale promotion,
  * h quantised per 128 channels (E4M3, fp32 scale), y = h Wd_g^T in FP32,
  * rounded to bf16.
  *   xq, xs, offsets as written by moe_permute for the same T
@@ -211,7 +229,9 @@ moe_status moe_permute_noalloc(moe_layer_t layer, const uint16_t* x, int T, int 
 moe_status moe_expert_ffn(moe_layer_t layer, const uint8_t* xq, const float* xs, const int32_t* offsets, int T,
                           uint16_t* y, void* ws, size_t ws_bytes, void* stream);
 
-/* The two halves of moe_expert_ffn, for callers that keep h themselves.
+/* The two halves of moe_expert_ffn, for callers that keep h themselves
+ * (SwiGLU experts of Dots3NoteTextConfig with the fine-grained FP8 weights
+ * of transformers PR #47844, as cited at moe_expert_ffn).
  * moe_gate_up: h = quantise(silu(xq Wg^T) * (xq Wu^T)) per row per 128
  * channels.
  *   h   [rows][ceil(F/128)*128] E4M3 bytes (out); channels >= F are zero
@@ -225,29 +245,40 @@ moe_status moe_gate_up(moe_layer_t layer, const uint8_t* xq, const float* xs, co
 moe_status moe_down(moe_layer_t layer, const uint8_t* h, const float* hs, const int32_t* offsets, int T,
                     uint16_t* y, void* stream);
 
-/* out[t] = bf16_RNE( sum_k topk_w[t,k] * y[inv[t,k]] + S * y[T*K + t] ), FP32
+/* Weighted combine of the routed experts' outputs plus the shared expert's
+ * (Dots3NoteTextConfig: norm_topk_prob, routed_scaling_factor,
+ * n_shared_experts 1), the "combine" of the DeepEP transport of the SGLang
+ * cookbook "Dots3-Note" ("2. Configuration Tips") done as a gather on one GPU:
+ * out[t] = bf16_RNE( sum_k topk_w[t,k] * y[inv[t,k]] + S * y[T*K + t] ), FP32
  * sum in slot order, shared row (when n_shared = 1) last.
  *   out [T][ldo] bf16, ldo >= H                                            */
 moe_status moe_combine(moe_layer_t layer, const uint16_t* y, const int32_t* inv, const float* topk_w, int T,
                        uint16_t* out, int ldo, void* stream);
 
-/* The whole layer: moe_route -> moe_permute -> moe_expert_ffn -> moe_combine,
+/* The whole MoE layer of the dots3-note language model (Dots3NoteTextConfig;
+ * model card dots-studio/dots3-note-prev, "Model Overview": 256 routed + 1
+ * shared experts, top-8):
+ * moe_route -> moe_permute -> moe_expert_ffn -> moe_combine,
  * with every intermediate in the workspace. */
 moe_status moe_layer_forward(moe_layer_t layer, const uint16_t* x, int T, int ldx, uint16_t* out, int ldo,
                              void* ws, size_t ws_bytes, void* stream);
 
 /* Synchronises `stream`, returns MOE_ERR_DEVICE if any kernel of this layer
  * flagged an error since the last call (and clears the flag), else MOE_OK.
- * If `detail` is not NULL it receives the raw status bits. */
+ * If `detail` is not NULL it receives the raw status bits. Library plumbing:
+ * no counterpart on the pages. */
 moe_status moe_get_device_status(moe_layer_t layer, void* stream, uint32_t* detail);
 
 /* Number of kernels moe_layer_forward launches for T tokens (route 2,
  * permute 5, gate/up 1, down 1 plus 1 when its K blocks are split, combine
- * 1); 0 for T = 0 or bad arguments. */
+ * 1); 0 for T = 0 or bad arguments. Library plumbing: no counterpart on the
+ * pages. */
 int moe_kernels_per_forward(moe_layer_t layer, int T);
 
-/* Test hook for the grouped FP8 GEMM with per-128-K-block promotion: writes
- * the promoted FP32 accumulators instead of the fused epilogue.
+/* Test hook for the grouped FP8 GEMM with per-128-K-block promotion (the
+ * 128 x 128 weight blocks and per-token activation scales of transformers
+ * PR #47844, "What does this PR do?"): writes the promoted FP32 accumulators
+ * instead of the fused epilogue.
  *   which = 0: gate/up GEMM; a = xq [rows][H], as = [H/128][rows];
  *              out [rows][2*ceil(F/128)*128] fp32, channel block c of the
  *              gate result at columns [256c, 256c+128), of the up result at

@@ -110,3 +110,18 @@ def test_null_layer_everywhere():
     assert L.moe_layer_forward(None, 16, 1, 5120, 16, 5120, 16, 1 << 20, None) == fx.MOE_ERR_INVALID_ARG
     assert L.moe_get_device_status(None, None, None) == fx.MOE_ERR_INVALID_ARG
     assert L.moe_test_grouped_gemm_f32(None, 0, 16, 16, 16, 1, 16, None) == fx.MOE_ERR_INVALID_ARG
+
+
+CITES = ("Dots3NoteTextConfig", "PR #47844", "Dots3-Note", "dots-studio/dots3-note-prev", "Dots 3 Note Preview")
+NO_COUNTERPART = ("no counterpart on the pages", "The pages describe no such call")
+
+
+def test_every_declared_call_cites_its_passage():
+    """The comment in front of each declaration cites the page passage that
+    defines the operation, or says that the pages have no counterpart."""
+    text = open(HEADER).read()
+    for name in header_functions():
+        at = re.search(r"^\s*(?:const\s+)?\w+\s*\*?\s*" + name + r"\s*\(", text, flags=re.M).start()
+        end = text.rfind("*/", 0, at)
+        comment = " ".join(text[text.rfind("/*", 0, end):end].replace("*", " ").split())
+        assert any(c in comment for c in CITES + NO_COUNTERPART), f"{name}: no citation in {comment[:80]!r}"
