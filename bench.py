@@ -1,7 +1,7 @@
 """Benchmark of the FP8 MoE-layer forward (dots3-note preview shape) on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload decode|prefill|zipf|edge] [--no-secondary]
+                    [--workload decode|prefill|zipf|edge|edge_f1500|...] [--no-workloads]
 
 One step = one whole forward of the layer (route, permute + quantise, gate/up
 GEMM + SwiGLU + quantise, down GEMM, combine) over one batch of T tokens
@@ -9,6 +9,13 @@ whose inputs already sit in HBM. With N > 1 (torchrun, one rank per GPU) every
 rank runs an independent replica of the layer on its own batch: the layer has
 no exchange step on one node at this scale, so the job is weak-scaled and the
 value is all ranks' tokens over the slowest rank's device time.
+
+On one GPU the line also carries a `workloads` block: each of the seeded
+workloads of the layer (decode T=64, prefill T=4096, Zipf long prefill
+T=16384, edge T=4099 and its FFN=1500 variant) timed the same way, with both
+roofline fractions (measured HBM copy bandwidth; dense FP8 = 2 x the measured
+BF16 burst GEMM rate), its own clock sample and the C++ FP64 oracle timed on
+that workload's own tokens. The toy layer is a parity case only.
 
 Prints one JSON line (rank 0).
 """
@@ -40,8 +47,10 @@ def parse():
     p.add_argument("--steps", type=int, default=200)
     p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    p.add_argument("--workload", default="decode", choices=["decode", "prefill", "zipf", "edge", "decode_e64", "prefill_e32", "vision", "dense"])
-    p.add_argument("--no-secondary", action="store_true", help="skip the T=16384 Zipf measurement")
+    p.add_argument("--workload", default="decode",
+                   choices=["decode", "prefill", "zipf", "edge", "edge_f1500", "decode_e64", "prefill_e32", "vision",
+                            "dense"])
+    p.add_argument("--no-workloads", action="store_true", help="time only --workload (no workloads block)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     return p.parse_args()
 
@@ -151,7 +160,7 @@ class ClockSampler:
         os.close(fd)
         try:
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
                                          stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
@@ -204,22 +213,33 @@ def algorithmic_work(layer, T, offsets):
             "flops": {"gate_up": gu_flops, "down": dn_flops}}
 
 
+_device_layers: dict = {}
+
+
 def load_layer(name, d, rank):
     """Host inputs on every rank; with several ranks rank 0 generates the
-    expert weights and broadcasts them over NCCL (same checkpoint everywhere)."""
+    expert weights and broadcasts them over NCCL (same checkpoint everywhere).
+    On one rank, workloads of the same layer (shape and weight seed) share
+    the host and device copies of its experts; only the router differs."""
     import gen
     import torch
     from fp8_expert_ffn_b200 import torch_utils as tu
     import fp8_expert_ffn_b200 as fx
     wl = gen.WORKLOADS[name]
     sh = wl.shape
-    x = gen.make_x(wl.T, sh.H, wl.x_seed + 1000 * rank, wl.outliers, wl.zipf)
-    if d.world == 1 or rank == 0:
-        host = gen.make_layer(sh, wl.w_seed, zipf=wl.zipf)
-    else:
-        host = None
     if d.world == 1:
-        return wl, host, tu.upload_layer(host), x
+        wl, host, x = gen.workload_inputs(name)
+        key = (sh, wl.w_seed)
+        prev = _device_layers.get(key)
+        dev = tu.upload_layer(host, share_experts=prev)
+        if prev is None:
+            for k in list(_device_layers):      # keep one layer's experts on the device at a time
+                del _device_layers[k]
+            torch.cuda.empty_cache()
+            _device_layers[key] = dev
+        return wl, host, dev, x
+    x = gen.make_x(wl.T, sh.H, wl.x_seed + 1000 * rank, wl.outliers, wl.zipf)
+    host = gen.make_layer(sh, wl.w_seed, zipf=wl.zipf) if rank == 0 else None
     shapes = {"w_gate": ((sh.E + sh.S, sh.F, sh.H), torch.uint8), "w_up": ((sh.E + sh.S, sh.F, sh.H), torch.uint8),
               "w_down": ((sh.E + sh.S, sh.H, sh.ld_f), torch.uint8),
               "s_gate": ((sh.E + sh.S, sh.FB, sh.HB), torch.float32), "s_up": ((sh.E + sh.S, sh.FB, sh.HB), torch.float32),
@@ -336,22 +356,89 @@ def time_e2e(dev, sh, x_bits, steps, warmup, d: Dist):
     return a.elapsed_time(b), T * H * 2, T * H * 2
 
 
-def cpu_baseline(host_layer, x_bits, budget_s=20.0):
-    """The oracle (FP64 numpy) on a bounded sample of the workload's tokens,
-    timed on this host's cores."""
-    from oracle import moe
-    n, dt = 1, 0.0
-    tokens = np.arange(x_bits.shape[0])
-    while True:
-        t = time.perf_counter()
-        moe.token_outputs(x_bits, host_layer, tokens[:n])
-        dt = time.perf_counter() - t
-        if dt * 2 > budget_s or n * 2 > len(tokens):
-            break
-        n *= 2
-    return {"value": n / dt, "unit": "tokens/s", "cores": moe.WORKERS, "kind": "oracle",
-            "sample": f"{n} of the {len(tokens)} tokens through the whole layer (route, quantise, expert FFNs, "
-                      f"combine; FP64), {dt:.1f} s"}
+ORACLE_TOKENS = 64     # tokens of one oracle sample (the whole decode batch)
+
+
+def oracle_sample(host_layer, x_bits, first: int = 0):
+    """One sample for the CPU baseline: the C++ FP64 oracle (plain loops,
+    all host cores) through the whole layer -- route, permute, quantise,
+    expert FFNs, combine -- on ORACLE_TOKENS consecutive tokens of the
+    workload starting at `first` (wrapping). Returns (tokens, seconds)."""
+    from oracle import cpp
+    T = x_bits.shape[0]
+    n = min(T, ORACLE_TOKENS)
+    tok = (first + np.arange(n)) % T
+    t = time.perf_counter()
+    cpp.layer_forward(np.ascontiguousarray(x_bits[tok]), host_layer)
+    return n, time.perf_counter() - t
+
+
+def cpu_baseline(host_layer, x_bits, budget_s=10.0):
+    """The oracle as it stands, timed on this host's cores: samples of
+    oracle_sample until about budget_s seconds have passed."""
+    from oracle import cpp
+    tokens, secs, i = 0, 0.0, 0
+    while secs < budget_s:
+        n, dt = oracle_sample(host_layer, x_bits, first=i * ORACLE_TOKENS)
+        tokens, secs, i = tokens + n, secs + dt, i + 1
+    return {"value": round(tokens / secs, 3), "unit": "tokens/s", "cores": cpp.threads(), "kind": "oracle",
+            "sample": f"C++ FP64 oracle, {i} x {min(x_bits.shape[0], ORACLE_TOKENS)} consecutive tokens of the "
+                      f"workload through the whole layer (route, permute, quantise, expert FFNs, combine), "
+                      f"{secs:.1f} s"}
+
+
+def fractions(work, per, total_ms, pk):
+    """Both roofline fractions of each GEMM and of the whole step: HBM
+    (algorithmic bytes / time / measured copy bandwidth) and dense FP8
+    (algorithmic FLOPs / time / (2 x measured BF16 burst rate); the sustained
+    BF16 figure gives the sustained fraction beside it)."""
+    fp8 = FP8_OVER_BF16 * pk["bf16_tflops"]
+    fp8_sus = FP8_OVER_BF16 * pk["bf16_tflops_sustained"]
+    out = {}
+    step_bytes = sum(work["bytes"].values())
+    step_flops = sum(work["flops"].values())
+    for k, b, f, ms in (("gate_up", work["bytes"]["gate_up"], work["flops"]["gate_up"], per["gate_up"]),
+                        ("down", work["bytes"]["down"], work["flops"]["down"], per["down"]),
+                        ("step", step_bytes, step_flops, total_ms)):
+        gbs = b / (ms / 1e3) / 1e9
+        tfs = f / (ms / 1e3) / 1e12
+        out[k] = {"ms": round(ms, 5), "hbm_gbs": round(gbs, 1), "frac_hbm": round(gbs / pk["hbm_gbs"], 4),
+                  "tflops": round(tfs, 1), "frac_fp8": round(tfs / fp8, 4), "frac_fp8_sustained": round(tfs / fp8_sus, 4)}
+    ridge = fp8 * 1e12 / (pk["hbm_gbs"] * 1e9)
+    out["binding"] = "hbm" if work["flops"]["gate_up"] / work["bytes"]["gate_up"] < ridge else "tensor"
+    return out
+
+
+def measure_workload(name, d, rank, args, pk, sampler, oracle=True):
+    """One workload: its stages timed over the same number of steps as the
+    headline (at least 10; a timed region of 0.01-0.15 s, like the burst
+    GEMM measurement behind the FP8 peak), with its own clock sample and the
+    oracle on its own tokens."""
+    from fp8_expert_ffn_b200 import torch_utils as tu
+    wl, host, dev, x_bits = load_layer(name, d, rank)
+    st = Stages(dev, wl.shape, wl.T, tu.bf16_tensor(x_bits))
+    steps = max(10, args.steps)
+    total_ms, per, clocks = time_stages(st, steps, max(3, min(args.warmup, 5)), d, sampler)
+    total_ms = d.max(total_ms)
+    off = st.offsets.cpu().numpy()
+    work = algorithmic_work(wl, wl.T, off)
+    counts = np.diff(off)[:wl.shape.E]
+    entry = {"workload": f"{wl.name}: {wl.note}", "T": wl.T, "steps": steps,
+             "tokens_per_s": round(d.sum(float(wl.T * steps)) / (total_ms / 1e3), 1),
+             "ms_per_step": round(total_ms / steps, 5), "stage_ms": {k: round(v, 5) for k, v in per.items()},
+             "roofline": fractions(work, per, total_ms / steps, pk), "clocks": clocks,
+             "touched_groups": work["touched_groups"],
+             "load_max_over_mean": round(float(counts.max() / max(counts.mean(), 1e-9)), 2),
+             "empty_experts": int((counts == 0).sum())}
+    if oracle and rank == 0:
+        n, dt = oracle_sample(host, x_bits)
+        entry["oracle"] = {"tokens_per_s": round(n / dt, 3), "tokens": n, "seconds": round(dt, 2),
+                           "kind": "C++ FP64 oracle on this workload's first tokens, whole layer"}
+    del st
+    return entry
+
+
+WORKLOADS = ("decode", "prefill", "zipf", "edge", "edge_f1500")
 
 
 # ----------------------------------------------------------------------------- arms
@@ -378,12 +465,12 @@ def run_ours(args):
     # gate/up weights (HBM); large batches by the FP8 tensor pipe
     kern = max(("gate_up", "down"), key=lambda k: per[k])
     kern_ms = d.max(per[kern])
-    hbm_bound = work["flops"][kern] / work["bytes"][kern] < (FP8_OVER_BF16 * pk["bf16_tflops"] * 1e12) / (
-        pk["hbm_gbs"] * 1e9)
+    fp8 = FP8_OVER_BF16 * pk["bf16_tflops"]
+    hbm_bound = work["flops"][kern] / work["bytes"][kern] < (fp8 * 1e12) / (pk["hbm_gbs"] * 1e9)
     # both fractions of the dominant kernel; the non-binding one is reported
     # beside the roofline (it matters for mid-size batches such as T = 4096)
     hbm_frac = work["bytes"][kern] / (kern_ms / 1e3) / 1e9 / pk["hbm_gbs"]
-    tensor_frac = work["flops"][kern] / (kern_ms / 1e3) / 1e12 / (FP8_OVER_BF16 * pk["bf16_tflops"])
+    tensor_frac = work["flops"][kern] / (kern_ms / 1e3) / 1e12 / fp8
     other = {"bound": "tensor", "frac": round(tensor_frac, 4)} if hbm_bound else {"bound": "hbm",
                                                                                  "frac": round(hbm_frac, 4)}
     if hbm_bound:
@@ -393,12 +480,12 @@ def run_ours(args):
                 "algorithmic_bytes_per_launch": work["bytes"][kern], "ms_per_launch": round(kern_ms, 5),
                 "peak_source": f"{pk['source']} hbm_gbs"}
     else:
-        peak = FP8_OVER_BF16 * pk["bf16_tflops"]
         ach = work["flops"][kern] / (kern_ms / 1e3) / 1e12
-        roof = {"bound": "tensor", "kernel": kern, "achieved": round(ach, 1), "peak": round(peak, 1),
-                "unit": "TFLOP/s", "frac": round(ach / peak, 4), "traffic": None,
+        roof = {"bound": "tensor", "kernel": kern, "achieved": round(ach, 1), "peak": round(fp8, 1),
+                "unit": "TFLOP/s", "frac": round(ach / fp8, 4), "traffic": None,
                 "algorithmic_flops_per_launch": work["flops"][kern], "ms_per_launch": round(kern_ms, 5),
-                "peak_source": f"{pk['source']} bf16_tflops x {FP8_OVER_BF16} (nominal FP8/BF16 ratio)"}
+                "peak_source": f"{pk['source']} bf16_tflops (burst) x {FP8_OVER_BF16} (nominal FP8/BF16 ratio)",
+                "frac_of_sustained": round(ach / (FP8_OVER_BF16 * pk["bf16_tflops_sustained"]), 4)}
     roof["other_bound"] = other
     e2e_ms, bi, bo = time_e2e(dev, sh, x_bits, args.steps, args.warmup, d)
     e2e_ms = d.max(e2e_ms)
@@ -418,77 +505,53 @@ def run_ours(args):
         "gpu_launches": st.fx.moe_kernels_per_forward(dev, T) * args.steps,
         "clocks": clocks,
     }
-    if not args.no_secondary and args.workload != "zipf":
-        del st
-        sec = secondary(d, rank, args, pk)
-        if sec:
-            line["secondary"] = sec
+    del st
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(host, x_bits)
+    if world == 1 and not args.no_workloads:
+        wls = {}
+        for name in WORKLOADS:
+            wls[name] = measure_workload(name, d, rank, args, pk, ClockSampler(sampler.gpu),
+                                         oracle=not args.no_cpu_baseline)
+        wls["toy"] = {"workload": "toy: T=32, hidden 512, 16+1 experts, top-4, FFN 256",
+                      "purpose": "parity only (every value checked against the oracle), not timed"}
+        line["workloads"] = wls
+        line["peaks"] = {"hbm_gbs": pk["hbm_gbs"], "fp8_tflops_burst": round(fp8, 1),
+                         "fp8_tflops_sustained": round(FP8_OVER_BF16 * pk["bf16_tflops_sustained"], 1),
+                         "source": f"{pk['source']}: HBM copy; FP8 = {FP8_OVER_BF16} x BF16 GEMM (nominal ratio)"}
     if rank == 0:
         print(json.dumps(line), flush=True)
     d.close()
 
 
-def secondary(d, rank, args, pk):
-    """The long-prefill workload (T=16384, Zipf-skewed routing), timed the same way."""
-    import torch
-    from fp8_expert_ffn_b200 import torch_utils as tu
-    wl, host, dev, x_bits = load_layer("zipf", d, rank)
-    st = Stages(dev, wl.shape, wl.T, tu.bf16_tensor(x_bits))
-    steps = max(3, min(args.steps, 20))
-    total_ms, per, _ = time_stages(st, steps, max(3, min(args.warmup, 5)), d)
-    total_ms = d.max(total_ms)
-    off = st.offsets.cpu().numpy()
-    work = algorithmic_work(wl, wl.T, off)
-    flops = work["flops"]["gate_up"] + work["flops"]["down"]
-    gemm_ms = d.max(per["gate_up"] + per["down"])
-    # the GEMMs run back to back inside multi-millisecond steps under the
-    # power cap: the sustained GEMM figure is the denominator (burst for context)
-    peak = FP8_OVER_BF16 * pk["bf16_tflops_sustained"]
-    burst = FP8_OVER_BF16 * pk["bf16_tflops"]
-    kern = max(("gate_up", "down"), key=lambda k: per[k])
-    kms = d.max(per[kern])
-    ach = work["flops"][kern] / (kms / 1e3) / 1e12
-    counts = np.diff(off)[:wl.shape.E]
-    return {"workload": f"{wl.name}: {wl.note}", "T": wl.T, "steps": steps,
-            "value": round(d.sum(float(wl.T * steps)) / (total_ms / 1e3), 1), "unit": "tokens/s",
-            "ms_per_step": round(total_ms / steps, 5), "stage_ms": {k: round(v, 5) for k, v in per.items()},
-            "expert_gemm_tflops": round(flops / (gemm_ms / 1e3) / 1e12, 1),
-            "roofline": {"bound": "tensor", "kernel": kern, "achieved": round(ach, 1), "peak": round(peak, 1),
-                         "unit": "TFLOP/s", "frac": round(ach / peak, 4),
-                         "peak_source": f"{pk['source']} bf16_tflops_sustained x {FP8_OVER_BF16}",
-                         "frac_of_burst": round(ach / burst, 4)},
-            "load_max_over_mean": round(float(counts.max() / counts.mean()), 2),
-            "empty_experts": int((counts == 0).sum())}
-
-
 def run_reference(args):
-    """The oracle timed on this host's cores as the reference arm (rank 0 only)."""
+    """The C++ FP64 oracle timed on this host's cores as the reference arm
+    (rank 0 only): each step is one oracle_sample of the workload (the same
+    sampling rule as the cpu_baseline of the other arm)."""
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     if rank != 0:
         return
     import gen
-    from oracle import moe
-    wl = gen.WORKLOADS[args.workload]
-    host = gen.make_layer(wl.shape, wl.w_seed, zipf=wl.zipf)
-    x_bits = gen.make_x(wl.T, wl.shape.H, wl.x_seed, wl.outliers, wl.zipf)
-    per_step = 1                       # tokens per step: a bounded sample of the batch
+    from oracle import cpp
+    wl, host, x_bits = gen.workload_inputs(args.workload)
+    cpp.build()
     for i in range(args.warmup):
-        moe.token_outputs(x_bits, host, [i % wl.T])
-    t = time.perf_counter()
+        oracle_sample(host, x_bits, first=i * ORACLE_TOKENS)
+    tokens, secs = 0, 0.0
     for i in range(args.steps):
-        moe.token_outputs(x_bits, host, [(args.warmup + i) % wl.T])
-    dt = time.perf_counter() - t
-    value = per_step * args.steps / dt
+        n, dt = oracle_sample(host, x_bits, first=(args.warmup + i) * ORACLE_TOKENS)
+        tokens, secs = tokens + n, secs + dt
+    value = tokens / secs
+    n1 = min(wl.T, ORACLE_TOKENS)
     line = {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "tokens/s", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(secs / args.steps * 1e3, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": f"{wl.name}: {wl.note}", "T": wl.T, "hidden": wl.shape.H,
                        "experts": f"{wl.shape.E}+{wl.shape.S}", "top_k": wl.shape.K, "ffn": wl.shape.F},
-            "cpu_baseline": {"value": round(value, 4), "unit": "tokens/s", "kind": "oracle", "cores": moe.WORKERS,
-                             "sample": f"{per_step} token per step through the whole layer (FP64 oracle)"},
+            "cpu_baseline": {"value": round(value, 4), "unit": "tokens/s", "kind": "oracle", "cores": cpp.threads(),
+                             "sample": f"C++ FP64 oracle, {n1} consecutive tokens of the workload per step "
+                                       f"through the whole layer"},
             "e2e": {"value": round(value, 4), "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)

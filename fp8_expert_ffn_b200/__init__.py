@@ -20,7 +20,7 @@ MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_MISALIGNED, MOE_ERR_UNSUPPORTED, MOE_ERR_WO
 ENTRY_POINTS = ("moe_status_string", "moe_layer_create", "moe_layer_destroy", "moe_workspace_size", "moe_route",
                 "moe_permute", "moe_expert_ffn", "moe_combine", "moe_layer_forward", "moe_get_device_status",
                 "moe_gate_up", "moe_down", "moe_test_grouped_gemm_f32", "moe_permute_noalloc",
-                "moe_kernels_per_forward")
+                "moe_kernels_per_forward", "moe_test_inject_stall")
 
 MOE_NOALLOC_MAX_TOKENS = 4096   # include/moe.h
 
@@ -78,6 +78,7 @@ def lib(build_if_missing: bool = True):
     L.moe_down.argtypes = [P, P, P, P, I, P, P]
     L.moe_test_grouped_gemm_f32.argtypes = [P, I, P, P, P, I, P, P]
     L.moe_kernels_per_forward.argtypes = [P, I]
+    L.moe_test_inject_stall.argtypes = [P, ctypes.c_ulonglong]
     for name in ENTRY_POINTS:
         if name not in ("moe_status_string", "moe_workspace_size"):
             getattr(L, name).restype = I
@@ -158,6 +159,10 @@ class MoeLayer:
 
 def moe_kernels_per_forward(layer: MoeLayer, T: int) -> int:
     return int(lib().moe_kernels_per_forward(layer.handle, T))
+
+
+def moe_test_inject_stall(layer: MoeLayer, wait_limit_ns: int):
+    _check("moe_test_inject_stall", lib().moe_test_inject_stall(layer.handle, int(wait_limit_ns)))
 
 
 def moe_workspace_size(layer: MoeLayer, T: int) -> int:

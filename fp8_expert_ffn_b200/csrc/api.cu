@@ -362,6 +362,12 @@ moe_status moe_get_device_status(moe_layer_t L, void* stream, uint32_t* detail) 
   return v ? MOE_ERR_DEVICE : MOE_OK;
 }
 
+moe_status moe_test_inject_stall(moe_layer_t L, unsigned long long wait_limit_ns) {
+  if (!L || wait_limit_ns == 0) return MOE_ERR_INVALID_ARG;
+  L->test_stall_ns = wait_limit_ns;
+  return MOE_OK;
+}
+
 moe_status moe_test_grouped_gemm_f32(moe_layer_t L, int which, const uint8_t* a, const float* as,
                                      const int32_t* offsets, int T, float* out, void* stream) {
   if (!L || T < 0 || T > kMaxT || (which != 0 && which != 1)) return MOE_ERR_INVALID_ARG;

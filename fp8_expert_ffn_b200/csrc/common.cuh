@@ -72,10 +72,11 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar_addr, uint32_t parity
 }
 
 // Waits for the phase with the given parity to complete. Gives up after
-// kWaitLimitNs or as soon as *abort is set by another role; on giving up it
-// records STATUS_WAIT_TIMEOUT, sets *abort and returns false.
+// limit_ns (kWaitLimitNs unless a test shortens it) or as soon as *abort is
+// set by another role; on giving up it records STATUS_WAIT_TIMEOUT, sets
+// *abort and returns false.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          uint32_t* status) {
+                                          uint32_t* status, unsigned long long limit_ns = kWaitLimitNs) {
   const uint32_t a = smem_u32(bar);
   if (mbar_try_wait(a, parity)) return true;
   const unsigned long long t0 = globaltimer_ns();
@@ -83,7 +84,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     if (mbar_try_wait(a, parity)) return true;
     if ((i & 63u) == 0) {
       if (*abort) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (globaltimer_ns() - t0 > limit_ns) {
         set_status(status, STATUS_WAIT_TIMEOUT);
         *abort = 1;
         return false;

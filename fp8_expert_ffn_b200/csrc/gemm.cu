@@ -107,6 +107,8 @@ struct GemmArgs {
   int ksplit;              // K splits per output tile (1 unless EPI_SPLIT)
   float* part;             // EPI_SPLIT: partials [ksplit][rows][ld_y] fp32
   uint32_t* status;
+  unsigned long long wait_ns;  // limit of every pipeline wait (kWaitLimitNs; a test may shorten it)
+  int withhold;            // test only: CTA 0's producer skips its first stage, so a wait must time out
 };
 
 struct TileInfo {
@@ -150,9 +152,10 @@ __device__ __forceinline__ TileInfo decode_tile(int i, const int* s_prefix, cons
 }
 
 // Bounded wait that ignores the abort flag (used to drain in-flight work).
-__device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity, uint32_t* status) {
+__device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity, uint32_t* status,
+                                                unsigned long long limit_ns) {
   int never = 0;
-  mbar_wait(bar, parity, &never, status);
+  mbar_wait(bar, parity, &never, status, limit_ns);
 }
 
 template <int MODE, int EPI>
@@ -213,11 +216,20 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   // Group offsets and the exclusive prefix of the tile counts (every CTA
   // derives the same tile list from the device-side offsets).
+  // Offsets that decrease, start below 0 or end beyond the row count would
+  // send tiles outside the buffers: the launch then does no work and sets
+  // STATUS_BAD_PLAN.
+  int bad_plan;
   {
     __shared__ int s_wsum[THREADS / 32];
     const int g = threadIdx.x;
     int v = 0;
-    if (g < p.ngroups) v = ((p.offsets[g + 1] - p.offsets[g] + BM - 1) / BM) * p.ntn;
+    bool bad = false;
+    if (g < p.ngroups) {
+      const int o0 = p.offsets[g], o1 = p.offsets[g + 1];
+      bad = o0 < 0 || o1 < o0 || (g == p.ngroups - 1 && o1 > p.rows);
+      if (!bad) v = ((o1 - o0 + BM - 1) / BM) * p.ntn;
+    }
     int incl = v;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
@@ -225,7 +237,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       if ((threadIdx.x & 31) >= off) incl += o;
     }
     if ((threadIdx.x & 31) == 31) s_wsum[threadIdx.x >> 5] = incl;
-    __syncthreads();
+    bad_plan = __syncthreads_or(bad ? 1 : 0);
     int base = 0;
     for (int j = 0; j < (threadIdx.x >> 5); ++j) base += s_wsum[j];
     if (g < p.ngroups) s_prefix[g] = base + incl - v;
@@ -235,8 +247,10 @@ __global__ void __launch_bounds__(THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = tmem_base_s;
-  const int total = s_prefix[p.ngroups] * p.ksplit;
+  if (bad_plan && threadIdx.x == 0) set_status(p.status, STATUS_BAD_PLAN);
+  const int total = bad_plan ? 0 : s_prefix[p.ngroups] * p.ksplit;
   uint32_t issued = 0;
+  uint32_t withheld = 0xFFFFFFFFu;   // the stage a test made the producer skip
 
   // The two warpgroup kinds run to the end of the kernel on separate paths
   // (each with its own copy of the teardown), so that the register limits
@@ -253,7 +267,11 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int kb = t.kb0; kb < t.kb1; ++kb) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1u;
-          if (!mbar_wait(&empty_bar[s], ph ^ 1u, s_abort, p.status)) { ok = false; break; }
+          if (!mbar_wait(&empty_bar[s], ph ^ 1u, s_abort, p.status, p.wait_ns)) { ok = false; break; }
+          if (p.withhold && blockIdx.x == 0 && it == 0) {   // test only: this stage never arrives
+            withheld = it++;
+            continue;
+          }
           uint8_t* a = smem + s * STAGE_BYTES;
           uint8_t* b = a + A_BYTES;
           mbar_arrive_expect_tx(&full_bar[s], STAGE_BYTES);
@@ -282,8 +300,8 @@ __global__ void __launch_bounds__(THREADS, 1)
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1u;
           const uint32_t buf = tb & 1u, tph = (tb >> 1) & 1u;
-          if (!mbar_wait(&tempty_bar[buf], tph ^ 1u, s_abort, p.status)) { ok = false; break; }
-          if (!mbar_wait(&full_bar[s], ph, s_abort, p.status)) { ok = false; break; }
+          if (!mbar_wait(&tempty_bar[buf], tph ^ 1u, s_abort, p.status, p.wait_ns)) { ok = false; break; }
+          if (!mbar_wait(&full_bar[s], ph, s_abort, p.status, p.wait_ns)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a_addr = smem_u32(smem + s * STAGE_BYTES);
           const uint64_t ad = smem_desc_sw128(a_addr);
@@ -300,7 +318,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       s_consumed = it;
       tc_commit(&done_bar);                 // all MMAs issued above have completed
-      mbar_wait_drain(&done_bar, 0, p.status);
+      mbar_wait_drain(&done_bar, 0, p.status, p.wait_ns);
     }
   } else if (warp == 2) {
     // ------------------------------------------------------------ tile list
@@ -311,7 +329,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (int i = blockIdx.x; i < total; i += gridDim.x, ++k) {
       const uint32_t b = k & 1u, ph = (k >> 1) & 1u;
       bool go = true;
-      if (lane == 0) go = mbar_wait(&tinfo_empty[b], ph ^ 1u, s_abort, p.status);
+      if (lane == 0) go = mbar_wait(&tinfo_empty[b], ph ^ 1u, s_abort, p.status, p.wait_ns);
       if (!__shfl_sync(0xFFFFFFFFu, go ? 1 : 0, 0)) break;
       const TileInfo t = decode_tile(i, s_prefix, p.offsets, p.ngroups, p.ntn, p.ksplit, p.nkb);
       if (lane == 0) {
@@ -336,7 +354,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   asm volatile("bar.sync 0;" ::: "memory");
   if (warp == 0 && lane == 0) {
     // copies issued but never consumed (only after an abort) must land first
-    for (uint32_t j = s_consumed; j < issued; ++j) mbar_wait_drain(&full_bar[j % STAGES], (j / STAGES) & 1u, p.status);
+    for (uint32_t j = s_consumed; j < issued; ++j)
+      if (j != withheld) mbar_wait_drain(&full_bar[j % STAGES], (j / STAGES) & 1u, p.status, p.wait_ns);
   }
   tc_fence_before();
   asm volatile("bar.sync 0;" ::: "memory");
@@ -358,7 +377,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       TileInfo t;
       {  // the tile, decoded ahead by warp 2
         const uint32_t b = tile_iter & 1u;
-        if (!mbar_wait(&tinfo_full[b], (tile_iter >> 1) & 1u, s_abort, p.status)) break;
+        if (!mbar_wait(&tinfo_full[b], (tile_iter >> 1) & 1u, s_abort, p.status, p.wait_ns)) break;
         const int4 v = s_tinfo[b][0], u = s_tinfo[b][1];
         t.g = v.x;
         t.nt = v.y;
@@ -418,7 +437,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         pf3 = (valid && kr + 4 < nk) ? __ldg(asp + size_t(kr + 4) * ast) : 0.0f;
         const float f0 = __shfl_sync(0xFFFFFFFFu, wr0, kr & 31) * sa;
         const float f1 = __shfl_sync(0xFFFFFFFFu, wr1, kr & 31) * sa;
-        if (!mbar_wait(&tfull_bar[buf], tph, s_abort, p.status)) { ok = false; break; }
+        if (!mbar_wait(&tfull_bar[buf], tph, s_abort, p.status, p.wait_ns)) { ok = false; break; }
         tc_fence_after();
         if (warp_active) {
           const uint32_t tbase = tmem_base + (uint32_t(q * 32) << 16) + buf * BN;
@@ -493,7 +512,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         s_amax[xb][half][r_in] = amax;
         __syncwarp();
         if (lane == 0) mbar_arrive(&amax_bar[xb][q]);
-        if (!mbar_wait(&amax_bar[xb][q], (tile_iter >> 1) & 1u, s_abort, p.status)) { ok = false; break; }
+        if (!mbar_wait(&amax_bar[xb][q], (tile_iter >> 1) & 1u, s_abort, p.status, p.wait_ns)) { ok = false; break; }
         amax = fmaxf(amax, s_amax[xb][half ^ 1][r_in]);
         if (valid) {
           uint32_t pk[16];
@@ -589,7 +608,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 
 template <int MODE, int EPI>
 cudaError_t launch_gemm(const moe_layer_s* L, const CUtensorMap& tmA, const CUtensorMap& tmB0,
-                        const CUtensorMap& tmB1, const CUtensorMap& tmY, const GemmArgs& a, cudaStream_t st) {
+                        const CUtensorMap& tmB1, const CUtensorMap& tmY, const GemmArgs& args, cudaStream_t st) {
   constexpr int SMEM_DYN = smem_dyn(MODE);
   static std::atomic<bool> configured[kMaxDevices];   // the attribute is per device
   cudaError_t ce = once_per_device(configured, []() {
@@ -604,6 +623,14 @@ cudaError_t launch_gemm(const moe_layer_s* L, const CUtensorMap& tmA, const CUte
                                 SMEM_DYN);
   });
   if (ce != cudaSuccess) return ce;
+  GemmArgs a = args;
+  a.wait_ns = kWaitLimitNs;
+  a.withhold = 0;
+  if (L->test_stall_ns) {   // a test armed a stall for this one launch
+    a.wait_ns = L->test_stall_ns;
+    a.withhold = 1;
+    L->test_stall_ns = 0;
+  }
   // upper bound on the number of tiles: every group may add one partial row tile
   const long long bound = (static_cast<long long>(a.rows) / BM + a.ngroups) * a.ntn * a.ksplit;
   const int grid = int(bound < L->num_sms ? bound : L->num_sms);

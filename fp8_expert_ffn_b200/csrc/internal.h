@@ -29,6 +29,9 @@ struct moe_layer_s {
   CUtensorMap tm_gate;  // [E+1][F][ld_h] E4M3, box 128 x 128 x 1
   CUtensorMap tm_up;
   CUtensorMap tm_down;  // [E+1][H][ld_f] E4M3, box 128 x 128 x 1
+  // test only (moe_test_inject_stall): when nonzero, the next grouped-GEMM
+  // launch withholds one pipeline stage and uses this wait limit
+  mutable unsigned long long test_stall_ns;
 };
 
 namespace moe {

@@ -15,9 +15,10 @@
 //   1. permute_bitmap   one thread per (t, k): validate, set the bit
 //   2. permute_count    one CTA per expert: per-word prefix popcounts, count
 //   3. permute_offsets  one CTA: exclusive scan of counts -> offsets[E+2]
-//   4. permute_gather   one warp per token: rows of its K slots and its
-//                       shared-expert row, inv/perm, then the 128-channel
-//                       groups of x quantised once and stored to all rows.
+//   4. permute_gather   one warp per token and 16 groups of 128 channels:
+//                       rows of its K slots and its shared-expert row,
+//                       inv/perm, then the groups of x quantised once and
+//                       stored to all rows with 16-byte stores.
 #include <mutex>
 
 #include "common.cuh"
@@ -113,10 +114,14 @@ __global__ void __launch_bounds__(256) permute_offsets_kernel(const int32_t* __r
   }
 }
 
-constexpr int GATHER_GROUPS = 8;   // 128-channel groups per warp
+constexpr int GATHER_GROUPS = 16;   // 128-channel groups per warp (4 steps of 4 groups)
 
-// One warp per (token, chunk of GATHER_GROUPS groups). Lane k < K owns slot
-// k; lane K owns the shared row. The chunk-0 warp writes inv and perm.
+// One warp per (token, chunk of GATHER_GROUPS groups). In each step the warp
+// covers 4 consecutive groups: lanes 8j..8j+7 hold group j of the step, 16
+// channels per lane (one 32-byte load of x, one 16-byte store of codes per
+// row), so a row's store instruction writes 512 contiguous bytes. Lane k < K
+// owns slot k's row, lane K the shared row; the chunk-0 warp writes inv and
+// perm.
 __global__ void __launch_bounds__(256) permute_gather_kernel(
     const uint16_t* __restrict__ x, int T, int ldx, int H, const int32_t* __restrict__ idx, int K, int E, int W,
     const uint32_t* __restrict__ bitmap, const uint32_t* __restrict__ wprefix, const int32_t* __restrict__ offsets,
@@ -125,18 +130,27 @@ __global__ void __launch_bounds__(256) permute_gather_kernel(
   pdl_wait();
   pdl_launch_dependents();
   const int lane = threadIdx.x & 31;
+  const int gl = lane & 7, gs = lane >> 3;   // lane within its group, group slot of the step
   const int HB = H / 128;
   const int nchunk = (HB + GATHER_GROUPS - 1) / GATHER_GROUPS;
   const int wid = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int t = wid / nchunk, chunk = wid - t * nchunk;
   if (t >= T) return;
-  const int g0 = chunk * GATHER_GROUPS, g1 = min(HB, g0 + GATHER_GROUPS);
+  const int g0 = chunk * GATHER_GROUPS;
   const uint16_t* xr = x + size_t(t) * ldx;
   // issue the x loads of the whole chunk before anything waits on memory
-  uint2 raw[GATHER_GROUPS];
+  uint4 raw[4][2];
 #pragma unroll
-  for (int i = 0; i < GATHER_GROUPS; ++i)
-    raw[i] = (g0 + i < g1) ? *reinterpret_cast<const uint2*>(xr + (g0 + i) * 128 + lane * 4) : make_uint2(0, 0);
+  for (int i = 0; i < 4; ++i) {
+    const int g = g0 + 4 * i + gs;
+    if (g < HB) {
+      const uint4* src = reinterpret_cast<const uint4*>(xr + g * 128 + gl * 16);
+      raw[i][0] = src[0];
+      raw[i][1] = src[1];
+    } else {
+      raw[i][0] = raw[i][1] = make_uint4(0u, 0u, 0u, 0u);
+    }
+  }
 
   int my_row = -1;
   if (lane < K) {
@@ -158,30 +172,42 @@ __global__ void __launch_bounds__(256) permute_gather_kernel(
   for (int j = 0; j < 9; ++j) rowv[j] = __shfl_sync(0xFFFFFFFFu, my_row, j);
 
 #pragma unroll
-  for (int i = 0; i < GATHER_GROUPS; ++i) {
-    const int g = g0 + i;
-    if (g >= g1) break;
-    // lane holds channels g*128 + lane*4 .. +3
-    float v[4] = {bf16_bits_to_f32(uint16_t(raw[i].x & 0xFFFFu)), bf16_bits_to_f32(uint16_t(raw[i].x >> 16)),
-                  bf16_bits_to_f32(uint16_t(raw[i].y & 0xFFFFu)), bf16_bits_to_f32(uint16_t(raw[i].y >> 16))};
-    float amax = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
+  for (int i = 0; i < 4; ++i) {
+    const int g = g0 + 4 * i + gs;
+    const bool valid = g < HB;   // uniform over the 8 lanes of a group
+    const uint32_t w32[8] = {raw[i][0].x, raw[i][0].y, raw[i][0].z, raw[i][0].w,
+                             raw[i][1].x, raw[i][1].y, raw[i][1].z, raw[i][1].w};
+    float v[16];
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
-    uint32_t packed = 0;
+    for (int j = 0; j < 8; ++j) {
+      v[2 * j] = bf16_bits_to_f32(uint16_t(w32[j] & 0xFFFFu));
+      v[2 * j + 1] = bf16_bits_to_f32(uint16_t(w32[j] >> 16));
+    }
+    float amax = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) amax = fmaxf(amax, fabsf(v[j]));
+#pragma unroll
+    for (int off = 1; off < 8; off <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
+    uint32_t packed[4] = {0u, 0u, 0u, 0u};
     float s = 0.0f;
     if (amax > 0.0f) {
       s = __fdiv_rn(amax, 448.0f);
-      const uint32_t lo = e4m3x2(__fdiv_rn(v[0], s), __fdiv_rn(v[1], s));
-      const uint32_t hi = e4m3x2(__fdiv_rn(v[2], s), __fdiv_rn(v[3], s));
-      packed = lo | (hi << 16);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t lo = e4m3x2(__fdiv_rn(v[4 * j], s), __fdiv_rn(v[4 * j + 1], s));
+        const uint32_t hi = e4m3x2(__fdiv_rn(v[4 * j + 2], s), __fdiv_rn(v[4 * j + 3], s));
+        packed[j] = lo | (hi << 16);
+      }
     }
+    if (!valid) continue;
+    const uint4 q = make_uint4(packed[0], packed[1], packed[2], packed[3]);
 #pragma unroll
     for (int j = 0; j < 9; ++j) {
       if (j > K) break;
       const int r = rowv[j];
       if (r < 0) continue;
-      *reinterpret_cast<uint32_t*>(xq + size_t(r) * H + g * 128 + lane * 4) = packed;
-      if (lane == j) xs[size_t(g) * rows + r] = s;
+      *reinterpret_cast<uint4*>(xq + size_t(r) * H + g * 128 + gl * 16) = q;
+      if (gl == (j & 7)) xs[size_t(g) * rows + r] = s;
     }
   }
 }

@@ -263,10 +263,16 @@ moe_status moe_combine(moe_layer_t layer, const uint16_t* y, const int32_t* inv,
 moe_status moe_layer_forward(moe_layer_t layer, const uint16_t* x, int T, int ldx, uint16_t* out, int ldo,
                              void* ws, size_t ws_bytes, void* stream);
 
+/* Bits of the device status word (moe_get_device_status's `detail`). */
+#define MOE_STATUS_BAD_EXPERT 0x1u   /* an expert id outside [0, E) was skipped */
+#define MOE_STATUS_DUP_EXPERT 0x2u   /* an expert repeated in one token's slots */
+#define MOE_STATUS_WAIT_TIMEOUT 0x4u /* a pipeline wait gave up; that launch's outputs are incomplete */
+#define MOE_STATUS_BAD_PLAN 0x8u     /* group offsets not ascending within [0, rows]; no GEMM work done */
+
 /* Synchronises `stream`, returns MOE_ERR_DEVICE if any kernel of this layer
  * flagged an error since the last call (and clears the flag), else MOE_OK.
- * If `detail` is not NULL it receives the raw status bits. Library plumbing:
- * no counterpart on the pages. */
+ * If `detail` is not NULL it receives the raw status bits (MOE_STATUS_*).
+ * Library plumbing: no counterpart on the pages. */
 moe_status moe_get_device_status(moe_layer_t layer, void* stream, uint32_t* detail);
 
 /* Number of kernels moe_layer_forward launches for T tokens (route 2,
@@ -274,6 +280,18 @@ moe_status moe_get_device_status(moe_layer_t layer, void* stream, uint32_t* deta
  * 1); 0 for T = 0 or bad arguments. Library plumbing: no counterpart on the
  * pages. */
 int moe_kernels_per_forward(moe_layer_t layer, int T);
+
+/* Test hook for failure detection (library plumbing: no counterpart on the
+ * pages). Arms a one-shot stall for the next grouped-GEMM launch on this
+ * handle (moe_gate_up, moe_down, or those inside moe_expert_ffn and
+ * moe_layer_forward): the first CTA's TMA producer skips its first pipeline
+ * stage, so the MMA issuer's wait for it can never complete, and every
+ * pipeline wait of that launch gives up after wait_limit_ns (> 0) instead of
+ * the normal 1 s. The kernel then records MOE_STATUS_WAIT_TIMEOUT, every
+ * role leaves its loop, the producer waits (bounded) for the copies it did
+ * issue, and the TMEM is freed; that launch's outputs are incomplete, the
+ * next launch runs normally. Nothing traps or hangs. */
+moe_status moe_test_inject_stall(moe_layer_t layer, unsigned long long wait_limit_ns);
 
 /* Test hook for the grouped FP8 GEMM with per-128-K-block promotion (the
  * 128 x 128 weight blocks and per-token activation scales of transformers

@@ -161,6 +161,66 @@ def test_layer_end_to_end(name):
     assert torch.equal(y2.view(torch.int16), c.y.view(torch.int16))
 
 
+def _check_rows_teacher_forced(name, rows):
+    """h codes against the oracle fed the GPU's xq/xs, and y against the
+    oracle fed the GPU's h, on every one of the given permuted rows."""
+    wl, layer, c = get_case(name)
+    sh = layer.shape
+    rows = np.unique(rows)
+    off = c.np("offsets")
+    rt = torch.from_numpy(rows).cuda()
+    xq = c.xq[rt].cpu().numpy()
+    xs = c.np("xs")[:, rows].T.copy()
+    ref = gc.oracle_ffn_on_rows(layer, np.arange(len(rows)), xq, xs, np.searchsorted(rows, off).astype(np.int64))
+    hq = c.hq[rt].cpu().numpy()[:, :sh.F]
+    match = np.mean(hq == ref["hq"])
+    assert match >= 0.995, f"{name}: h code match {match:.5f} over {len(rows)} rows"
+    assert gc.e4m3_step_diff(hq, ref["hq"]).max() <= 1
+    hs = c.hs.cpu().numpy()[:, rows].T.copy()
+    E1 = sh.E + 1
+    groups = np.searchsorted(off, rows, side="right") - 1
+    sub_off = np.zeros(E1 + 1, np.int64)
+    sub_off[1:] = np.cumsum(np.bincount(groups, minlength=E1)[:E1])
+    y_tf = moe.expert_down_rows(hq, hs, sub_off, layer, groups=np.unique(groups))
+    yg = moe.bf16_to_f64(tu.bf16_bits(c.y[rt]))
+    rms = np.sqrt(np.mean(y_tf ** 2))
+    bad = np.abs(yg - y_tf) > 2.0 ** -8 * np.abs(y_tf) + 1e-4 * rms
+    assert not bad.any(), f"{name}: y differs beyond bf16 rounding on {np.unique(np.nonzero(bad)[0]).size} rows"
+
+
+def test_zipf_hottest_group_and_partial_tiles_every_row():
+    """Long prefill with Zipf routing, full size: every row of the busiest
+    expert's group (about 40 row tiles, several chunks of the tile order) and
+    every row of every group's partial last tile (the rows the GEMM epilogues
+    store without the bulk tensor path) -- h codes and y, teacher forced."""
+    wl, layer, c = get_case("zipf")
+    off = c.np("offsets").astype(np.int64)
+    counts = np.diff(off)[:layer.shape.E]
+    hot = int(np.argmax(counts))
+    rows = [np.arange(off[hot], off[hot + 1])]
+    for g in range(layer.shape.E + 1):
+        n = off[g + 1] - off[g]
+        if n % 128:
+            rows.append(np.arange(off[g] + (n // 128) * 128, off[g + 1]))
+    rows = np.concatenate(rows)
+    assert counts[hot] >= 10 * 128 and len(rows) > counts[hot] + 1000
+    _check_rows_teacher_forced("zipf", rows)
+
+
+def test_edge_last_tokens_end_to_end():
+    """The last 3 tokens of the ragged T=4099 batch (beyond the last full
+    128-token block), end to end against the oracle."""
+    wl, layer, c = get_case("edge")
+    toks = np.arange(c.T - 3, c.T)
+    r = moe.route(c.x_bits[toks], layer.router_w, layer.shape.K)
+    keep = toks[~r.near_tie]
+    assert len(keep) >= 2
+    ref = moe.token_outputs(c.x_bits, layer, keep)
+    gc.assert_output_close(moe.bf16_to_f64(c.np("out"))[keep], ref, "edge: last tokens")
+    rows = gc.rows_of_tokens(c.np("inv"), c.T, layer.shape.K, toks, layer.shape.S)
+    _check_rows_teacher_forced("edge", rows)
+
+
 def test_bf16_checkpoint_cross_check():
     """FP8 path vs the oracle's BF16-weight path (no activation quantisation)
     on the F=1500 variant: catches a wrong dequantisation (scale index or
@@ -562,3 +622,62 @@ def test_forward_is_cuda_graph_capturable():
     assert code == fx.MOE_OK, f"{bits:#x}"
     assert torch.equal(out.view(torch.int16), eager.view(torch.int16))
     del g
+
+
+# ----------------------------------------------------------------------------- failure detection
+
+def test_timed_out_wait_is_reported_and_the_handle_recovers():
+    """A pipeline wait that runs out (a stage the producer withholds, with a
+    1 ms limit) ends the GEMM launch with MOE_STATUS_WAIT_TIMEOUT instead of
+    hanging; the next forward on the same handle is bit-identical to one
+    before the fault."""
+    wl, layer, c = get_case("toy")
+    sh, T = layer.shape, c.T
+    fx.moe_gate_up(c.dev, c.xq, c.xs, c.offsets, T, c.hq, c.hs)
+    assert fx.moe_get_device_status(c.dev) == (fx.MOE_OK, 0)
+    h_ref = c.hq.clone()
+    for stage in ("gate_up", "down"):
+        fx.moe_test_inject_stall(c.dev, 1_000_000)
+        h = torch.zeros_like(c.hq)
+        hs = torch.zeros_like(c.hs)
+        y = torch.zeros_like(c.y)
+        if stage == "gate_up":
+            fx.moe_gate_up(c.dev, c.xq, c.xs, c.offsets, T, h, hs)
+        else:
+            fx.moe_down(c.dev, c.hq, c.hs, c.offsets, T, y)
+        code, bits = fx.moe_get_device_status(c.dev)
+        assert code == fx.MOE_ERR_DEVICE and bits & 0x4, (stage, code, hex(bits))
+        # the handle is usable at once: the same launch again is complete and exact
+        if stage == "gate_up":
+            fx.moe_gate_up(c.dev, c.xq, c.xs, c.offsets, T, h, hs)
+            assert fx.moe_get_device_status(c.dev) == (fx.MOE_OK, 0)
+            assert torch.equal(h, h_ref)
+        else:
+            fx.moe_down(c.dev, c.hq, c.hs, c.offsets, T, y)
+            assert fx.moe_get_device_status(c.dev) == (fx.MOE_OK, 0)
+            assert torch.equal(y.view(torch.int16), c.y.view(torch.int16))
+    ws = tu.workspace(c.dev, T)
+    out = torch.empty_like(c.out)
+    fx.moe_layer_forward(c.dev, c.x, T, sh.H, out, sh.H, ws, ws.numel())
+    assert fx.moe_get_device_status(c.dev) == (fx.MOE_OK, 0)
+    assert torch.equal(out.view(torch.int16), c.out.view(torch.int16))
+
+
+def test_inconsistent_offsets_set_bad_plan_and_do_no_work():
+    """Group offsets that decrease or run past the row count are caught by the
+    GEMM's own check before any tile is planned: MOE_STATUS_BAD_PLAN, and the
+    output buffers are left untouched."""
+    wl, layer, c = get_case("toy")
+    sh, T = layer.shape, c.T
+    good = c.np("offsets")
+    for bad in (np.concatenate([good[:5], good[4:5] - 1, good[6:]]),      # a decreasing step
+                np.concatenate([good[:-1], [good[-1] + 128]])):          # past the last row
+        off = torch.from_numpy(bad.astype(np.int32)).cuda()
+        h = torch.full_like(c.hq, 0x5A)
+        hs = torch.full_like(c.hs, 7.0)
+        fx.moe_gate_up(c.dev, c.xq, c.xs, off, T, h, hs)
+        code, bits = fx.moe_get_device_status(c.dev)
+        assert code == fx.MOE_ERR_DEVICE and bits == 0x8, hex(bits)
+        assert bool((h == 0x5A).all()) and bool((hs == 7.0).all())
+    fx.moe_gate_up(c.dev, c.xq, c.xs, c.offsets, T, h, hs)
+    assert fx.moe_get_device_status(c.dev) == (fx.MOE_OK, 0)

@@ -65,6 +65,26 @@ def test_noalloc_permute_matches_workspace_permute_twice():
             assert np.array_equal(a.view(np.uint8), b.view(np.uint8)), f"T={T}: {name} differs"
 
 
+def test_noalloc_permute_full_layer_at_the_size_limit():
+    """The 256-expert layer at T = MOE_NOALLOC_MAX_TOKENS: bitmap, prefix
+    words and counts of the shared array all at their largest, twice."""
+    wl, layer, x_bits = gen.workload_inputs("prefill")
+    sh = layer.shape
+    T = fx.MOE_NOALLOC_MAX_TOKENS
+    assert sh.E == 256 and x_bits.shape[0] >= T
+    dev = tu.upload_layer(layer)
+    ws = tu.workspace(dev, T)
+    for first in (0, 1):    # two calls in a row on different tokens
+        x = tu.bf16_tensor(np.ascontiguousarray(np.roll(x_bits, -first, axis=0)[:T]))
+        idx = torch.empty((T, sh.K), dtype=torch.int32, device="cuda")
+        w = torch.empty((T, sh.K), dtype=torch.float32, device="cuda")
+        fx.moe_route(dev, x, T, sh.H, idx, w, None, ws, ws.numel())
+        ref, got = _run_both(dev, sh, x, idx, T)
+        for name, a, b in zip(("offsets", "perm", "inv", "xq", "xs"), ref, got):
+            assert np.array_equal(a.view(np.uint8), b.view(np.uint8)), f"call {first}: {name} differs"
+    del dev
+
+
 def test_noalloc_permute_rejects_too_many_tokens():
     wl, layer, _ = gen.workload_inputs("toy")
     sh = layer.shape
