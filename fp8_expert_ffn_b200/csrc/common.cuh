@@ -233,6 +233,28 @@ __device__ __forceinline__ float rcp_approx(float x) {
   return y;
 }
 
+// (r0, r1) = (1/d0, 1/d1) for d in [1, 2^127) on the FMA pipe: the seed
+// 0x7EF311C3 - bits(d) is within 12.5% of 1/d (an exponent flip plus a
+// linear mantissa fit), and each Newton step r <- r + r (1 - d r) squares
+// the relative error, so three steps (done in packed f32x2 arithmetic) end
+// within about one fp32 ulp.
+__device__ __forceinline__ void rcp2_newton(float d0, float d1, float& r0, float& r1) {
+  r0 = __int_as_float(0x7EF311C3 - __float_as_int(d0));
+  r1 = __int_as_float(0x7EF311C3 - __float_as_int(d1));
+#pragma unroll
+  for (int i = 0; i < 3; ++i) {
+    asm("{\n\t.reg .b64 r, d, e, one;\n\t"
+        "mov.b64 r, {%0, %1};\n\t"
+        "mov.b64 d, {%2, %3};\n\t"
+        "mov.b64 one, {%4, %4};\n\t"
+        "fma.rn.f32x2 e, d, r, one;\n\t"
+        "fma.rn.f32x2 r, r, e, r;\n\t"
+        "mov.b64 {%0, %1}, r;\n\t}"
+        : "+f"(r0), "+f"(r1)
+        : "f"(-d0), "f"(-d1), "f"(1.0f));
+  }
+}
+
 // (a0, a1) += (v0, v1) * f with one packed f32x2 FMA (round to nearest).
 __device__ __forceinline__ void ffma2(float& a0, float& a1, float v0, float v1, float f) {
   asm("{\n\t.reg .b64 a, v, s, r;\n\t"

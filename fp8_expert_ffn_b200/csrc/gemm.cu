@@ -498,14 +498,21 @@ __global__ void __launch_bounds__(THREADS, 1)
         float amax = 0.0f;
         if (warp_active) {
 #pragma unroll
-          for (int j = 0; j < 64; ++j) {
-            const float g = acc[j];
-            // silu(g) * u = g * u / (1 + 2^(-g log2 e)) with the approximate
-            // exponential and reciprocal of the special-function unit (a few
-            // ulp of fp32; h is re-quantised to 3 mantissa bits next)
-            const float hv = g * acc[64 + j] * rcp_approx(1.0f + ex2_approx(-1.4426950408889634f * g));
-            acc[j] = hv;
-            amax = fmaxf(amax, fabsf(hv));
+          for (int j = 0; j < 64; j += 2) {
+            // silu(g) * u = g * u / (1 + 2^(-g log2 e)): the exponential on
+            // the special-function unit, the reciprocal on the FMA pipe
+            // (rcp2_newton), so the unit does one operation per channel; the
+            // exponent is capped at 126 so that the denominator stays finite
+            // (gates below -87 give |h| < 2^-120 either way)
+            const float g0 = acc[j], g1 = acc[j + 1];
+            const float d0 = 1.0f + ex2_approx(fminf(-1.4426950408889634f * g0, 126.0f));
+            const float d1 = 1.0f + ex2_approx(fminf(-1.4426950408889634f * g1, 126.0f));
+            float r0, r1;
+            rcp2_newton(d0, d1, r0, r1);
+            const float h0 = g0 * acc[64 + j] * r0, h1 = g1 * acc[65 + j] * r1;
+            acc[j] = h0;
+            acc[j + 1] = h1;
+            amax = fmaxf(amax, fmaxf(fabsf(h0), fabsf(h1)));
           }
         }
         const uint32_t xb = tile_iter & 1u;
