@@ -20,7 +20,8 @@ MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_MISALIGNED, MOE_ERR_UNSUPPORTED, MOE_ERR_WO
 ENTRY_POINTS = ("moe_status_string", "moe_layer_create", "moe_layer_destroy", "moe_workspace_size", "moe_route",
                 "moe_permute", "moe_expert_ffn", "moe_combine", "moe_layer_forward", "moe_get_device_status",
                 "moe_gate_up", "moe_down", "moe_test_grouped_gemm_f32", "moe_permute_noalloc",
-                "moe_kernels_per_forward", "moe_test_inject_stall")
+                "moe_kernels_per_forward", "moe_test_inject_stall", "moe_grouped_gate_up", "moe_grouped_down",
+                "moe_ep_pack_scales", "moe_ep_regroup", "moe_ep_unregroup")
 
 MOE_NOALLOC_MAX_TOKENS = 4096   # include/moe.h
 
@@ -79,6 +80,11 @@ def lib(build_if_missing: bool = True):
     L.moe_test_grouped_gemm_f32.argtypes = [P, I, P, P, P, I, P, P]
     L.moe_kernels_per_forward.argtypes = [P, I]
     L.moe_test_inject_stall.argtypes = [P, ctypes.c_ulonglong]
+    L.moe_grouped_gate_up.argtypes = [P, P, P, P, I, P, P, P]
+    L.moe_grouped_down.argtypes = [P, P, P, P, I, P, P]
+    L.moe_ep_pack_scales.argtypes = [P, P, I, P, P]
+    L.moe_ep_regroup.argtypes = [P, I, P, I, P, P, P, P, I, P, P, P, P]
+    L.moe_ep_unregroup.argtypes = [P, I, P, I, P, I, P, P, P]
     for name in ENTRY_POINTS:
         if name not in ("moe_status_string", "moe_workspace_size"):
             getattr(L, name).restype = I
@@ -159,6 +165,32 @@ class MoeLayer:
 
 def moe_kernels_per_forward(layer: MoeLayer, T: int) -> int:
     return int(lib().moe_kernels_per_forward(layer.handle, T))
+
+
+def moe_grouped_gate_up(layer, xq, xs, offsets, rows, h, hs, stream=None):
+    _check("moe_grouped_gate_up", lib().moe_grouped_gate_up(layer.handle, _ptr(xq), _ptr(xs), _ptr(offsets), rows,
+                                                            _ptr(h), _ptr(hs), _stream(stream)))
+
+
+def moe_grouped_down(layer, h, hs, offsets, rows, y, stream=None):
+    _check("moe_grouped_down", lib().moe_grouped_down(layer.handle, _ptr(h), _ptr(hs), _ptr(offsets), rows, _ptr(y),
+                                                      _stream(stream)))
+
+
+def moe_ep_pack_scales(layer, xs, T, xs_rows, stream=None):
+    _check("moe_ep_pack_scales", lib().moe_ep_pack_scales(layer.handle, _ptr(xs), T, _ptr(xs_rows), _stream(stream)))
+
+
+def moe_ep_regroup(layer, ranks, seg_counts, n_recv, recv_q, recv_s, own_q, own_s, T, out_q, out_s, out_offsets,
+                   stream=None):
+    _check("moe_ep_regroup", lib().moe_ep_regroup(layer.handle, ranks, _ptr(seg_counts), n_recv, _ptr(recv_q),
+                                                  _ptr(recv_s), _ptr(own_q), _ptr(own_s), T, _ptr(out_q),
+                                                  _ptr(out_s), _ptr(out_offsets), _stream(stream)))
+
+
+def moe_ep_unregroup(layer, ranks, seg_counts, n_recv, y_g, T, y_send, y_own, stream=None):
+    _check("moe_ep_unregroup", lib().moe_ep_unregroup(layer.handle, ranks, _ptr(seg_counts), n_recv, _ptr(y_g), T,
+                                                      _ptr(y_send), _ptr(y_own), _stream(stream)))
 
 
 def moe_test_inject_stall(layer: MoeLayer, wait_limit_ns: int):

@@ -42,12 +42,12 @@ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 std::mutex& device_setup_mutex() { return g_device_setup_mutex; }
 
 bool encode_tmap(CUtensorMap* tm, bool bf16, const void* base, uint64_t inner, uint64_t rows, uint64_t depth,
-                 uint64_t ld_bytes, uint64_t depth_stride_bytes, bool force3d) {
+                 uint64_t ld_bytes, uint64_t depth_stride_bytes, bool force3d, uint32_t box_rows) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[3] = {inner, rows, depth};
   cuuint64_t strides[2] = {ld_bytes, depth_stride_bytes};
-  cuuint32_t box[3] = {bf16 ? 64u : 128u, 128, 1};   // 128 bytes of K per box row
+  cuuint32_t box[3] = {bf16 ? 64u : 128u, box_rows, 1};   // 128 bytes of K per box row
   cuuint32_t estr[3] = {1, 1, 1};
   const cuuint32_t rank = (depth > 1 || force3d) ? 3 : 2;
   CUresult r = fn(tm, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, rank,
@@ -91,7 +91,7 @@ Scratch carve(const moe_layer_s* L, int T, void* base) {
   s.route_partial = static_cast<float*>(take(sizeof(float) * size_t(route_splits(L, T)) * T * E));
   s.bitmap = static_cast<uint32_t*>(take(sizeof(uint32_t) * E * W));
   s.wprefix = static_cast<uint32_t*>(take(sizeof(uint32_t) * E * W));
-  s.counts = static_cast<int32_t*>(take(sizeof(int32_t) * E));
+  s.counts = static_cast<int32_t*>(take(sizeof(int32_t) * (E + 1)));   // + the count kernel's completion counter
   s.h = static_cast<uint8_t*>(take(rows * L->ld_hh));
   s.hs = static_cast<float*>(take(sizeof(float) * L->FB * rows));
   s.idx = static_cast<int32_t*>(take(sizeof(int32_t) * size_t(T) * K));
@@ -162,13 +162,20 @@ moe_status moe_layer_create(const moe_layer_desc* d, const moe_weights* w, moe_l
       d->topk_group > d->n_group || d->top_k > d->topk_group * (d->n_routed / d->n_group))
     return MOE_ERR_UNSUPPORTED;
   if (!(d->routed_scaling == d->routed_scaling)) return MOE_ERR_INVALID_ARG;
-  if (!w->w_gate || !w->w_up || !w->w_down || !w->s_gate || !w->s_up || !w->s_down || !w->router_w)
-    return MOE_ERR_INVALID_ARG;
-  if (w->ld_h < d->hidden || w->ld_f < d->ffn) return MOE_ERR_INVALID_ARG;
-  if (w->ld_h % 16 != 0 || w->ld_f % 16 != 0) return MOE_ERR_MISALIGNED;
-  const void* ptrs[] = {w->w_gate, w->w_up, w->w_down, w->s_gate, w->s_up, w->s_down, w->router_w};
-  for (const void* p : ptrs)
-    if (!aligned16(p)) return MOE_ERR_MISALIGNED;
+  if (!w->router_w) return MOE_ERR_INVALID_ARG;
+  // all six expert arrays, or none (a routing-only handle: route, permute, combine)
+  const void* experts[] = {w->w_gate, w->w_up, w->w_down, w->s_gate, w->s_up, w->s_down};
+  int given = 0;
+  for (const void* p : experts) given += p != nullptr;
+  if (given != 0 && given != 6) return MOE_ERR_INVALID_ARG;
+  const bool has_experts = given == 6;
+  if (has_experts) {
+    if (w->ld_h < d->hidden || w->ld_f < d->ffn) return MOE_ERR_INVALID_ARG;
+    if (w->ld_h % 16 != 0 || w->ld_f % 16 != 0) return MOE_ERR_MISALIGNED;
+    for (const void* p : experts)
+      if (!aligned16(p)) return MOE_ERR_MISALIGNED;
+  }
+  if (!aligned16(w->router_w)) return MOE_ERR_MISALIGNED;
   if (w->router_bias && !aligned16(w->router_bias)) return MOE_ERR_MISALIGNED;
 
   int dev = 0;
@@ -191,18 +198,21 @@ moe_status moe_layer_create(const moe_layer_desc* d, const moe_weights* w, moe_l
   L->ld_hh = L->FB * 128;
   L->device = dev;
   L->num_sms = prop.multiProcessorCount;
+  L->has_experts = has_experts;
   // weight maps are always 3-D (expert index = z), even with a single expert
   const uint64_t E1 = uint64_t(L->E) + L->S;
-  if (!encode_tmap(&L->tm_gate, false, w->w_gate, L->H, L->F, E1, w->ld_h, uint64_t(L->F) * w->ld_h, true) ||
-      !encode_tmap(&L->tm_up, false, w->w_up, L->H, L->F, E1, w->ld_h, uint64_t(L->F) * w->ld_h, true) ||
-      !encode_tmap(&L->tm_down, false, w->w_down, L->F, L->H, E1, w->ld_f, uint64_t(L->H) * w->ld_f, true)) {
+  if (has_experts &&
+      (!encode_tmap(&L->tm_gate, false, w->w_gate, L->H, L->F, E1, w->ld_h, uint64_t(L->F) * w->ld_h, true) ||
+       !encode_tmap(&L->tm_up, false, w->w_up, L->H, L->F, E1, w->ld_h, uint64_t(L->F) * w->ld_h, true) ||
+       !encode_tmap(&L->tm_down, false, w->w_down, L->F, L->H, E1, w->ld_f, uint64_t(L->H) * w->ld_f, true))) {
     delete L;
     return MOE_ERR_CUDA;
   }
   const size_t split_bytes = 3 * size_t(L->E) * L->H * sizeof(uint16_t);
   bool ok = cudaMalloc(&L->status, sizeof(uint32_t)) == cudaSuccess;
   ok = ok && cudaMalloc(&L->router_split, split_bytes) == cudaSuccess;
-  ok = ok && cudaMalloc(&L->splitk, sizeof(float) * size_t(kSplitMax) * kSplitRows * L->H) == cudaSuccess;
+  if (has_experts)
+    ok = ok && cudaMalloc(&L->splitk, sizeof(float) * size_t(kSplitMax) * kSplitRows * L->H) == cudaSuccess;
   ok = ok && cudaMemset(L->status, 0, sizeof(uint32_t)) == cudaSuccess;
   if (w->router_bias) {
     ok = ok && cudaMalloc(&L->router_bias, sizeof(float) * L->E) == cudaSuccess;
@@ -212,7 +222,7 @@ moe_status moe_layer_create(const moe_layer_desc* d, const moe_weights* w, moe_l
   ok = ok && launch_router_split(w->router_w, L->E, L->H, L->router_split, nullptr) == cudaSuccess;
   ok = ok && cudaDeviceSynchronize() == cudaSuccess;
   ok = ok && encode_tmap(&L->tm_router, true, L->router_split, L->H, L->E, 3, uint64_t(L->H) * 2,
-                         uint64_t(L->E) * L->H * 2);
+                         uint64_t(L->E) * L->H * 2, false, kRouterExperts);
   if (!ok) {
     cudaFree(L->status);
     cudaFree(L->router_split);
@@ -287,24 +297,79 @@ moe_status moe_permute_noalloc(moe_layer_t L, const uint16_t* x, int T, int ldx,
 moe_status moe_gate_up(moe_layer_t L, const uint8_t* xq, const float* xs, const int32_t* offsets, int T,
                        uint8_t* h, float* hs, void* stream) {
   if (!L || T < 0 || T > kMaxT) return MOE_ERR_INVALID_ARG;
+  if (!L->has_experts) return MOE_ERR_INVALID_ARG;   // a routing-only handle
   if (T == 0) return MOE_OK;
   if (!xq || !xs || !offsets || !h || !hs) return MOE_ERR_INVALID_ARG;
   if (!aligned16(xq) || !aligned16(h)) return MOE_ERR_MISALIGNED;
-  return from_cuda(launch_gate_up(L, xq, xs, offsets, T, h, hs, static_cast<cudaStream_t>(stream)));
+  return from_cuda(launch_gate_up(L, xq, xs, offsets, T * (L->K + L->S), h, hs, static_cast<cudaStream_t>(stream)));
 }
 
 moe_status moe_down(moe_layer_t L, const uint8_t* h, const float* hs, const int32_t* offsets, int T, uint16_t* y,
                     void* stream) {
   if (!L || T < 0 || T > kMaxT) return MOE_ERR_INVALID_ARG;
+  if (!L->has_experts) return MOE_ERR_INVALID_ARG;   // a routing-only handle
   if (T == 0) return MOE_OK;
   if (!h || !hs || !offsets || !y) return MOE_ERR_INVALID_ARG;
   if (!aligned16(h) || !aligned16(y)) return MOE_ERR_MISALIGNED;
-  return from_cuda(launch_down(L, h, hs, offsets, T, y, static_cast<cudaStream_t>(stream)));
+  return from_cuda(launch_down(L, h, hs, offsets, T * (L->K + L->S), y, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_grouped_gate_up(moe_layer_t L, const uint8_t* xq, const float* xs, const int32_t* offsets, int rows,
+                               uint8_t* h, float* hs, void* stream) {
+  if (!L || rows < 0 || rows > kMaxT * 9) return MOE_ERR_INVALID_ARG;
+  if (!L->has_experts) return MOE_ERR_INVALID_ARG;
+  if (rows == 0) return MOE_OK;
+  if (!xq || !xs || !offsets || !h || !hs) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(xq) || !aligned16(h)) return MOE_ERR_MISALIGNED;
+  return from_cuda(launch_gate_up(L, xq, xs, offsets, rows, h, hs, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_grouped_down(moe_layer_t L, const uint8_t* h, const float* hs, const int32_t* offsets, int rows,
+                            uint16_t* y, void* stream) {
+  if (!L || rows < 0 || rows > kMaxT * 9) return MOE_ERR_INVALID_ARG;
+  if (!L->has_experts) return MOE_ERR_INVALID_ARG;
+  if (rows == 0) return MOE_OK;
+  if (!h || !hs || !offsets || !y) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(h) || !aligned16(y)) return MOE_ERR_MISALIGNED;
+  return from_cuda(launch_down(L, h, hs, offsets, rows, y, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_ep_pack_scales(moe_layer_t L, const float* xs, int T, float* xs_rows, void* stream) {
+  if (!L || T < 0 || T > kMaxT) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!xs || !xs_rows) return MOE_ERR_INVALID_ARG;
+  return from_cuda(launch_ep_pack_scales(L, xs, T, xs_rows, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_ep_regroup(moe_layer_t L, int ranks, const int32_t* seg_counts, int n_recv, const uint8_t* recv_q,
+                          const float* recv_s, const uint8_t* own_q, const float* own_s, int T, uint8_t* out_q,
+                          float* out_s, int32_t* out_offsets, void* stream) {
+  if (!L || ranks < 1 || ranks * L->E > kEpMaxSegments || n_recv < 0 || T < 0 || T > kMaxT)
+    return MOE_ERR_INVALID_ARG;
+  if (!seg_counts || !out_q || !out_s || !out_offsets) return MOE_ERR_INVALID_ARG;
+  if (n_recv > 0 && (!recv_q || !recv_s)) return MOE_ERR_INVALID_ARG;
+  if (T * L->S > 0 && (!own_q || !own_s)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(recv_q) || !aligned16(own_q) || !aligned16(out_q)) return MOE_ERR_MISALIGNED;
+  return from_cuda(launch_ep_regroup(L, ranks, seg_counts, n_recv, recv_q, recv_s, own_q, own_s, T, out_q, out_s,
+                                     out_offsets, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_ep_unregroup(moe_layer_t L, int ranks, const int32_t* seg_counts, int n_recv, const uint16_t* y_g,
+                            int T, uint16_t* y_send, uint16_t* y_own, void* stream) {
+  if (!L || ranks < 1 || ranks * L->E > kEpMaxSegments || n_recv < 0 || T < 0 || T > kMaxT)
+    return MOE_ERR_INVALID_ARG;
+  if (!seg_counts || !y_g) return MOE_ERR_INVALID_ARG;
+  if ((n_recv > 0 && !y_send) || (T * L->S > 0 && !y_own)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(y_g) || !aligned16(y_send) || !aligned16(y_own)) return MOE_ERR_MISALIGNED;
+  if (n_recv + T * L->S == 0) return MOE_OK;
+  return from_cuda(launch_ep_unregroup(L, ranks, seg_counts, n_recv, y_g, T, y_send, y_own,
+                                       static_cast<cudaStream_t>(stream)));
 }
 
 moe_status moe_expert_ffn(moe_layer_t L, const uint8_t* xq, const float* xs, const int32_t* offsets, int T,
                           uint16_t* y, void* ws, size_t ws_bytes, void* stream) {
   if (!L || T < 0 || T > kMaxT) return MOE_ERR_INVALID_ARG;
+  if (!L->has_experts) return MOE_ERR_INVALID_ARG;   // a routing-only handle
   if (T == 0) return MOE_OK;
   if (!xq || !xs || !offsets || !y) return MOE_ERR_INVALID_ARG;
   if (!aligned16(xq) || !aligned16(y)) return MOE_ERR_MISALIGNED;
@@ -312,8 +377,9 @@ moe_status moe_expert_ffn(moe_layer_t L, const uint8_t* xq, const float* xs, con
   if ((s = check_ws(L, T, ws, ws_bytes)) != MOE_OK) return s;
   Scratch sc = carve(L, T, ws);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  cudaError_t e = launch_gate_up(L, xq, xs, offsets, T, sc.h, sc.hs, st);
-  if (e == cudaSuccess) e = launch_down(L, sc.h, sc.hs, offsets, T, y, st);
+  const int rows = T * (L->K + L->S);
+  cudaError_t e = launch_gate_up(L, xq, xs, offsets, rows, sc.h, sc.hs, st);
+  if (e == cudaSuccess) e = launch_down(L, sc.h, sc.hs, offsets, rows, y, st);
   return from_cuda(e);
 }
 
@@ -329,6 +395,7 @@ moe_status moe_combine(moe_layer_t L, const uint16_t* y, const int32_t* inv, con
 moe_status moe_layer_forward(moe_layer_t L, const uint16_t* x, int T, int ldx, uint16_t* out, int ldo, void* ws,
                              size_t ws_bytes, void* stream) {
   if (!L || T < 0 || T > kMaxT) return MOE_ERR_INVALID_ARG;
+  if (!L->has_experts) return MOE_ERR_INVALID_ARG;   // a routing-only handle
   if (T == 0) return MOE_OK;
   moe_status s;
   if ((s = check_x(L, x, ldx)) != MOE_OK) return s;
@@ -339,8 +406,9 @@ moe_status moe_layer_forward(moe_layer_t L, const uint16_t* x, int T, int ldx, u
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e = launch_route(L, x, T, ldx, sc.idx, sc.topw, nullptr, sc.route_partial, st);
   if (e == cudaSuccess) e = launch_permute(L, x, T, ldx, sc.idx, sc.offsets, sc.perm, sc.inv, sc.xq, sc.xs, sc, st);
-  if (e == cudaSuccess) e = launch_gate_up(L, sc.xq, sc.xs, sc.offsets, T, sc.h, sc.hs, st);
-  if (e == cudaSuccess) e = launch_down(L, sc.h, sc.hs, sc.offsets, T, sc.y, st);
+  const int rows = T * (L->K + L->S);
+  if (e == cudaSuccess) e = launch_gate_up(L, sc.xq, sc.xs, sc.offsets, rows, sc.h, sc.hs, st);
+  if (e == cudaSuccess) e = launch_down(L, sc.h, sc.hs, sc.offsets, rows, sc.y, st);
   if (e == cudaSuccess) e = launch_combine(L, sc.y, sc.inv, sc.topw, T, out, ldo, st);
   return from_cuda(e);
 }
@@ -348,7 +416,7 @@ moe_status moe_layer_forward(moe_layer_t L, const uint16_t* x, int T, int ldx, u
 int moe_kernels_per_forward(moe_layer_t L, int T) {
   if (!L || T <= 0 || T > kMaxT) return 0;
   const int rows = T * (L->K + L->S);
-  return 2 + 5 + 1 + 1 + (down_ksplit(L, rows) > 1 ? 1 : 0) + 1;
+  return 2 + 4 + 1 + 1 + (down_ksplit(L, rows) > 1 ? 1 : 0) + 1;
 }
 
 moe_status moe_get_device_status(moe_layer_t L, void* stream, uint32_t* detail) {
@@ -371,6 +439,7 @@ moe_status moe_test_inject_stall(moe_layer_t L, unsigned long long wait_limit_ns
 moe_status moe_test_grouped_gemm_f32(moe_layer_t L, int which, const uint8_t* a, const float* as,
                                      const int32_t* offsets, int T, float* out, void* stream) {
   if (!L || T < 0 || T > kMaxT || (which != 0 && which != 1)) return MOE_ERR_INVALID_ARG;
+  if (!L->has_experts) return MOE_ERR_INVALID_ARG;   // a routing-only handle
   if (T == 0) return MOE_OK;
   if (!a || !as || !offsets || !out) return MOE_ERR_INVALID_ARG;
   if (!aligned16(a)) return MOE_ERR_MISALIGNED;

@@ -721,9 +721,8 @@ static GemmArgs down_args(const moe_layer_s* L, const int32_t* offsets, int rows
   return a;
 }
 
-cudaError_t launch_gate_up(const moe_layer_s* L, const uint8_t* xq, const float* xs, const int32_t* offsets, int T,
+cudaError_t launch_gate_up(const moe_layer_s* L, const uint8_t* xq, const float* xs, const int32_t* offsets, int rows,
                            uint8_t* h, float* hs, cudaStream_t st) {
-  const int rows = T * (L->K + L->S);
   CUtensorMap tmX, tmHst;
   if (!encode_tmap_u8(&tmX, xq, L->H, rows, 1, L->H, 0)) return cudaErrorInvalidValue;
   if (!encode_tmap_store(&tmHst, false, h, L->ld_hh, rows, L->ld_hh)) return cudaErrorInvalidValue;
@@ -734,9 +733,8 @@ cudaError_t launch_gate_up(const moe_layer_s* L, const uint8_t* xq, const float*
   return launch_gemm<MODE_GATEUP, EPI_FUSED>(L, tmX, L->tm_gate, L->tm_up, tmHst, a, st);
 }
 
-cudaError_t launch_down(const moe_layer_s* L, const uint8_t* h, const float* hs, const int32_t* offsets, int T,
+cudaError_t launch_down(const moe_layer_s* L, const uint8_t* h, const float* hs, const int32_t* offsets, int rows,
                         uint16_t* y, cudaStream_t st) {
-  const int rows = T * (L->K + L->S);
   CUtensorMap tmH;
   if (!encode_tmap_u8(&tmH, h, L->F, rows, 1, L->ld_hh, 0)) return cudaErrorInvalidValue;
   CUtensorMap tmY;

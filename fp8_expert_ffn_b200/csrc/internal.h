@@ -21,11 +21,12 @@ struct moe_layer_s {
   int ld_hh;     // row stride of the quantised SwiGLU output h: FB * 128
   int device;
   int num_sms;
+  bool has_experts;  // false: a routing-only handle (route, permute, combine)
   uint32_t* status;  // device status word
   uint16_t* router_split;  // [3][E][H] bf16 terms of router_w (library-owned)
   float* router_bias;      // [E] selection-only bias (library-owned copy) or null
   float* splitk;           // [kSplitMax][kSplitRows][H] fp32 partials of the split down GEMM
-  CUtensorMap tm_router;   // over router_split, box 64 x 128 x 1
+  CUtensorMap tm_router;   // over router_split, box 64 x 256 x 1
   CUtensorMap tm_gate;  // [E+1][F][ld_h] E4M3, box 128 x 128 x 1
   CUtensorMap tm_up;
   CUtensorMap tm_down;  // [E+1][H][ld_f] E4M3, box 128 x 128 x 1
@@ -43,7 +44,7 @@ struct Scratch {
   // permute
   uint32_t* bitmap;       // [E][W]
   uint32_t* wprefix;      // [E][W]
-  int32_t* counts;        // [E]
+  int32_t* counts;        // [E] + 1 word: the count kernel's completion counter
   // expert ffn
   uint8_t* h;             // [rows][ld_hh]
   float* hs;              // [FB][rows]
@@ -78,10 +79,19 @@ int down_ksplit(const moe_layer_s* L, int rows);
 cudaError_t launch_permute_noalloc(const moe_layer_s* L, const uint16_t* x, int T, int ldx, const int32_t* idx,
                                    int32_t* offsets, int32_t* perm, int32_t* inv, uint8_t* xq, float* xs,
                                    cudaStream_t st);
-cudaError_t launch_gate_up(const moe_layer_s* L, const uint8_t* xq, const float* xs, const int32_t* offsets, int T,
+// rows: the permuted row count (the group stride of the scale arrays)
+cudaError_t launch_gate_up(const moe_layer_s* L, const uint8_t* xq, const float* xs, const int32_t* offsets, int rows,
                            uint8_t* h, float* hs, cudaStream_t st);
-cudaError_t launch_down(const moe_layer_s* L, const uint8_t* h, const float* hs, const int32_t* offsets, int T,
+cudaError_t launch_down(const moe_layer_s* L, const uint8_t* h, const float* hs, const int32_t* offsets, int rows,
                         uint16_t* y, cudaStream_t st);
+// Expert parallelism (ep.cu): at most kEpMaxSegments = ranks x local experts.
+constexpr int kEpMaxSegments = 2048;
+cudaError_t launch_ep_pack_scales(const moe_layer_s* L, const float* xs, int T, float* out, cudaStream_t st);
+cudaError_t launch_ep_regroup(const moe_layer_s* L, int P, const int32_t* cnt, int N, const uint8_t* recv_q,
+                              const float* recv_s, const uint8_t* own_q, const float* own_s, int T, uint8_t* out_q,
+                              float* out_s, int32_t* out_offsets, cudaStream_t st);
+cudaError_t launch_ep_unregroup(const moe_layer_s* L, int P, const int32_t* cnt, int N, const uint16_t* y_g, int T,
+                                uint16_t* y_send, uint16_t* y_own, cudaStream_t st);
 cudaError_t launch_test_gemm_f32(const moe_layer_s* L, int which, const uint8_t* a, const float* as,
                                  const int32_t* offsets, int T, float* out, cudaStream_t st);
 cudaError_t launch_combine(const moe_layer_s* L, const uint16_t* y, const int32_t* inv, const float* w, int T,
@@ -137,7 +147,9 @@ bool encode_tmap_u8(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t 
                     uint64_t ld, uint64_t depth_stride);
 // Same for bf16 (box 64 x 128 elements = 128 bytes of K per row) or u8.
 bool encode_tmap(CUtensorMap* tm, bool bf16, const void* base, uint64_t inner, uint64_t rows, uint64_t depth,
-                 uint64_t ld_bytes, uint64_t depth_stride_bytes, bool force3d = false);
+                 uint64_t ld_bytes, uint64_t depth_stride_bytes, bool force3d = false, uint32_t box_rows = 128);
+// Experts per router tile (the router weight map's box height).
+constexpr uint32_t kRouterExperts = 128;
 
 // Router weight split into three bf16 terms (hi + mid + lo == w exactly for
 // normal-range fp32 w), [3][E][H]; written once at layer creation.

@@ -13,8 +13,8 @@
 // (t, k) inside expert e's group is the number of earlier tokens that chose
 // e: a prefix popcount over e's bitmap words. Kernels:
 //   1. permute_bitmap   one thread per (t, k): validate, set the bit
-//   2. permute_count    one CTA per expert: per-word prefix popcounts, count
-//   3. permute_offsets  one CTA: exclusive scan of counts -> offsets[E+2]
+//   2. permute_count    one CTA per expert: per-word prefix popcounts, count;
+//                       the last CTA to finish scans the counts -> offsets[E+2]
 //   4. permute_gather   one warp per token and 16 groups of 128 channels:
 //                       rows of its K slots and its shared-expert row,
 //                       inv/perm, then the groups of x quantised once and
@@ -28,10 +28,13 @@ namespace moe {
 
 namespace {
 
-// Zeroes the token bitmap (n words) that the bitmap kernel ORs into.
-__global__ void __launch_bounds__(256) permute_clear_kernel(uint32_t* __restrict__ bitmap, size_t n) {
+// Zeroes the token bitmap (n words) that the bitmap kernel ORs into, and the
+// count kernel's completion counter.
+__global__ void __launch_bounds__(256) permute_clear_kernel(uint32_t* __restrict__ bitmap, size_t n,
+                                                            uint32_t* __restrict__ done) {
   pdl_wait();
   pdl_launch_dependents();
+  if (blockIdx.x == 0 && threadIdx.x == 0) *done = 0u;
   const size_t i = (size_t(blockIdx.x) * blockDim.x + threadIdx.x) * 4;
   if (i + 4 <= n) *reinterpret_cast<uint4*>(bitmap + i) = make_uint4(0u, 0u, 0u, 0u);
   else for (size_t k = i; k < n; ++k) bitmap[k] = 0u;
@@ -55,13 +58,19 @@ __global__ void permute_bitmap_kernel(const int32_t* __restrict__ idx, int T, in
 }
 
 // One CTA (256 threads) per expert: wprefix[e][w] = set bits of e's words
-// before word w; counts[e] = all set bits.
+// before word w; counts[e] = all set bits. The last CTA to finish (a device
+// counter, zeroed by the clear kernel) turns the counts into the offsets:
+// offsets[g] = sum of counts[0..g), offsets[E+1] = offsets[E] + T*S. The
+// offsets depend only on the counts, so the result is the same whichever CTA
+// is last.
 __global__ void __launch_bounds__(256) permute_count_kernel(const uint32_t* __restrict__ bitmap, int W,
-                                                            uint32_t* __restrict__ wprefix,
-                                                            int32_t* __restrict__ counts) {
+                                                            uint32_t* __restrict__ wprefix, int32_t* counts, int E,
+                                                            int T, int S, int32_t* __restrict__ offsets,
+                                                            uint32_t* done) {
   pdl_wait();
   pdl_launch_dependents();
   __shared__ uint32_t warp_sums[8];
+  __shared__ bool s_last;
   const int e = blockIdx.x, tid = threadIdx.x;
   const uint32_t* row = bitmap + size_t(e) * W;
   uint32_t* out = wprefix + size_t(e) * W;
@@ -87,30 +96,29 @@ __global__ void __launch_bounds__(256) permute_count_kernel(const uint32_t* __re
     run += __popc(row[w]);
   }
   if (tid == 255) counts[e] = int32_t(base + incl);
-}
-
-// offsets[g] = sum of counts[0..g), offsets[E+1] = offsets[E] + T.
-__global__ void __launch_bounds__(256) permute_offsets_kernel(const int32_t* __restrict__ counts, int E, int T,
-                                                              int S, int32_t* __restrict__ offsets) {
-  pdl_wait();
-  pdl_launch_dependents();
-  __shared__ int32_t warp_sums[8];
-  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-  const int v = tid < E ? counts[tid] : 0;
-  int incl = v;
+  __threadfence();   // this CTA's count is visible device-wide before it signals
+  __syncthreads();
+  if (tid == 0) s_last = atomicAdd(done, 1u) == uint32_t(E - 1);
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  // the last CTA: exclusive scan of the E <= 256 counts (read past L1)
+  const int v = tid < E ? __ldcg(counts + tid) : 0;
+  int inc = v;
 #pragma unroll
   for (int off = 1; off < 32; off <<= 1) {
-    int o = __shfl_up_sync(0xFFFFFFFFu, incl, off);
-    if (lane >= off) incl += o;
+    const int o = __shfl_up_sync(0xFFFFFFFFu, inc, off);
+    if (lane >= off) inc += o;
   }
-  if (lane == 31) warp_sums[wid] = incl;
+  __syncthreads();   // warp_sums is reused below
+  if (lane == 31) warp_sums[wid] = uint32_t(inc);
   __syncthreads();
-  int base = 0;
-  for (int j = 0; j < wid; ++j) base += warp_sums[j];
-  if (tid < E) offsets[tid] = base + incl - v;
+  int b = 0;
+  for (int j = 0; j < wid; ++j) b += int(warp_sums[j]);
+  if (tid < E) offsets[tid] = b + inc - v;
   if (tid == E - 1) {
-    offsets[E] = base + incl;
-    offsets[E + 1] = base + incl + T * S;
+    offsets[E] = b + inc;
+    offsets[E + 1] = b + inc + T * S;
   }
 }
 
@@ -221,17 +229,15 @@ cudaError_t launch_permute(const moe_layer_s* L, const uint16_t* x, int T, int l
   const int S = L->S;
   const int rows = T * (K + S);
   const size_t nwords = size_t(E) * W;
+  uint32_t* done = reinterpret_cast<uint32_t*>(s.counts + E);
   cudaError_t e = launch_pdl(permute_clear_kernel, dim3(unsigned((nwords + 1023) / 1024)), dim3(256), 0, st,
-                             s.bitmap, nwords);
+                             s.bitmap, nwords, done);
   if (e != cudaSuccess) return e;
   e = launch_pdl(permute_bitmap_kernel, dim3((T * K + 255) / 256), dim3(256), 0, st, idx, T, K, E, W, s.bitmap,
                  L->status);
   if (e != cudaSuccess) return e;
   e = launch_pdl(permute_count_kernel, dim3(E), dim3(256), 0, st, static_cast<const uint32_t*>(s.bitmap), W,
-                 s.wprefix, s.counts);
-  if (e != cudaSuccess) return e;
-  e = launch_pdl(permute_offsets_kernel, dim3(1), dim3(256), 0, st, static_cast<const int32_t*>(s.counts), E, T, S,
-                 offsets);
+                 s.wprefix, s.counts, E, T, S, offsets, done);
   if (e != cudaSuccess) return e;
   const int nchunk = (L->HB + GATHER_GROUPS - 1) / GATHER_GROUPS;
   const long long warps = static_cast<long long>(T) * nchunk;
@@ -252,7 +258,7 @@ cudaError_t launch_permute(const moe_layer_s* L, const uint16_t* x, int T, int l
 namespace {
 
 constexpr int kNoAllocWords = kNoAllocMaxExperts * ((kNoAllocMaxTokens + 31) / 32);
-static __device__ __align__(256) uint32_t g_permute_scratch[2 * kNoAllocWords + kNoAllocMaxExperts];
+static __device__ __align__(256) uint32_t g_permute_scratch[2 * kNoAllocWords + kNoAllocMaxExperts + 1];
 
 uint32_t* g_scratch_addr[kMaxDevices] = {};
 std::mutex g_scratch_mutex;

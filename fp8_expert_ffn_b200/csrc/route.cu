@@ -19,9 +19,9 @@
 // Kernel 1 (route_tc_kernel): CTA tile 128 tokens x 128 experts over a range of
 // 64-channel K blocks (split-K when there are fewer tiles than SMs); warp 0
 // TMA (x box 128 x 64 bf16 plus three 128 x 64 weight boxes per stage, 3
-// stages), warp 1 tcgen05.mma kind::f16 (M 128, N 128, K 16; 12 per stage)
-// into two 128-column TMEM buffers, warps 2-5 promote. Partial sums go to
-// partial[s][t][e].
+// stages of 64 KB), warp 1 tcgen05.mma kind::f16 (M 128, N 128, K 16; 12 per
+// stage) into two 128-column TMEM buffers, warps 4-11 promote (two per TMEM
+// lane quarter, one per 64-column half). Partial sums go to partial[s][t][e].
 // Kernel 2 (route_topk): one warp per token sums the S partials in order,
 // selects the top K by logit with ties to the lower id (an order-preserving
 // 64-bit key), and writes the slots in ascending expert id with weights
@@ -39,16 +39,23 @@ namespace moe {
 namespace {
 
 constexpr int RM = 128;                  // tokens per tile
-constexpr int RN = 128;                  // experts per tile
+constexpr int RN = int(kRouterExperts);  // experts per tile
 constexpr int RK = 64;                   // channels per K block (128 bytes of bf16)
 constexpr int R_STAGES = 3;
 constexpr int R_A_BYTES = RM * RK * 2;   // 16 KB
 constexpr int R_B_BYTES = RN * RK * 2;   // 16 KB per split term
-constexpr int R_STAGE_BYTES = R_A_BYTES + 3 * R_B_BYTES;
-constexpr int R_EPI_WARPS = 4;
-constexpr int R_THREADS = 64 + 32 * R_EPI_WARPS;
+constexpr int R_STAGE_BYTES = R_A_BYTES + 3 * R_B_BYTES;   // 64 KB
+constexpr int R_EPI_WARPS = 8;
+constexpr int R_FIRST_EPI_WARP = 4;
+constexpr int R_THREADS = 32 * (R_FIRST_EPI_WARP + R_EPI_WARPS);   // 384
 constexpr int R_SMEM_DYN = R_STAGES * R_STAGE_BYTES + 1024;
-constexpr uint32_t R_TMEM_COLS = 256;
+constexpr uint32_t R_TMEM_COLS = 2 * RN;   // two partial buffers
+// register split as in the grouped GEMM: the first warpgroup (TMA, MMA)
+// drops to R_PRODUCER_REGS, the two epilogue warpgroups rise to R_EPILOGUE_REGS
+constexpr int R_LAUNCH_REGS = 168;
+constexpr int R_PRODUCER_REGS = 40;
+constexpr int R_EPILOGUE_REGS = 232;
+static_assert(128 * R_PRODUCER_REGS + 256 * R_EPILOGUE_REGS <= R_THREADS * R_LAUNCH_REGS, "register split");
 
 // kind::f16 instruction descriptor: A = B = BF16, D = F32, both K-major.
 constexpr uint32_t idesc_bf16_f32(int M, int N) {
@@ -114,106 +121,119 @@ __global__ void __launch_bounds__(R_THREADS, 1)
   const uint32_t tmem_base = tmem_base_s;
   uint32_t issued = 0;
 
-  if (warp == 0) {
-    if (lane == 0) {
-      uint32_t it = 0;
-      for (int kb = 0; kb < n; ++kb) {
-        const int s = it % R_STAGES;
-        const uint32_t ph = (it / R_STAGES) & 1u;
-        if (!mbar_wait(&empty_bar[s], ph ^ 1u, s_abort, status)) break;
-        uint8_t* a = smem + s * R_STAGE_BYTES;
-        mbar_arrive_expect_tx(&full_bar[s], R_STAGE_BYTES);
-        const int k = (kb0 + kb) * RK;
-        tma_load_2d(a, &tmX, &full_bar[s], k, t0);
+  // The two warpgroup kinds run to the end on separate paths (each with its
+  // own copy of the teardown) so the setmaxnreg limits hold throughout.
+  if (warp < R_FIRST_EPI_WARP) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(R_PRODUCER_REGS));
+    if (warp == 0) {
+      if (lane == 0) {
+        uint32_t it = 0;
+        for (int kb = 0; kb < n; ++kb) {
+          const int s = it % R_STAGES;
+          const uint32_t ph = (it / R_STAGES) & 1u;
+          if (!mbar_wait(&empty_bar[s], ph ^ 1u, s_abort, status)) break;
+          uint8_t* a = smem + s * R_STAGE_BYTES;
+          mbar_arrive_expect_tx(&full_bar[s], R_STAGE_BYTES);
+          const int k = (kb0 + kb) * RK;
+          tma_load_2d(a, &tmX, &full_bar[s], k, t0);
 #pragma unroll
-        for (int j = 0; j < 3; ++j) tma_load_3d(a + R_A_BYTES + j * R_B_BYTES, &tmW, &full_bar[s], k, e0, j);
-        ++it;
-      }
-      issued = it;
-    }
-  } else if (warp == 1) {
-    if (lane == 0) {
-      uint32_t it = 0;
-      for (int kb = 0; kb < n; ++kb) {
-        const int s = it % R_STAGES;
-        const uint32_t ph = (it / R_STAGES) & 1u;
-        const uint32_t buf = it & 1u, tph = (it >> 1) & 1u;
-        if (!mbar_wait(&tempty_bar[buf], tph ^ 1u, s_abort, status)) break;
-        if (!mbar_wait(&full_bar[s], ph, s_abort, status)) break;
-        tc_fence_after();
-        const uint32_t a_addr = smem_u32(smem + s * R_STAGE_BYTES);
-        const uint64_t ad = smem_desc_sw128(a_addr);
-        const uint32_t d = tmem_base + buf * RN;
-#pragma unroll
-        for (int j = 0; j < 3; ++j) {
-          const uint64_t bd = smem_desc_sw128(a_addr + R_A_BYTES + j * R_B_BYTES);
-#pragma unroll
-          for (int k = 0; k < RK / 16; ++k)   // 16 bf16 = 32 bytes = 2 in the 16-byte address field
-            mma_bf16(d, ad + uint64_t(2 * k), bd + uint64_t(2 * k), R_IDESC, (j | k) ? 1u : 0u);
+          for (int j = 0; j < 3; ++j) tma_load_3d(a + R_A_BYTES + j * R_B_BYTES, &tmW, &full_bar[s], k, e0, j);
+          ++it;
         }
-        tc_commit(&empty_bar[s]);
-        tc_commit(&tfull_bar[buf]);
-        ++it;
+        issued = it;
       }
-      s_consumed = it;
-      tc_commit(&done_bar);
+    } else if (warp == 1) {
+      if (lane == 0) {
+        uint32_t it = 0;
+        for (int kb = 0; kb < n; ++kb) {
+          const int s = it % R_STAGES;
+          const uint32_t ph = (it / R_STAGES) & 1u;
+          const uint32_t buf = it & 1u, tph = (it >> 1) & 1u;
+          if (!mbar_wait(&tempty_bar[buf], tph ^ 1u, s_abort, status)) break;
+          if (!mbar_wait(&full_bar[s], ph, s_abort, status)) break;
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smem + s * R_STAGE_BYTES);
+          const uint64_t ad = smem_desc_sw128(a_addr);
+          const uint32_t d = tmem_base + buf * RN;
+#pragma unroll
+          for (int j = 0; j < 3; ++j) {
+            const uint64_t bd = smem_desc_sw128(a_addr + R_A_BYTES + j * R_B_BYTES);
+#pragma unroll
+            for (int k = 0; k < RK / 16; ++k)   // 16 bf16 = 32 bytes = 2 in the 16-byte address field
+              mma_bf16(d, ad + uint64_t(2 * k), bd + uint64_t(2 * k), R_IDESC, (j | k) ? 1u : 0u);
+          }
+          tc_commit(&empty_bar[s]);
+          tc_commit(&tfull_bar[buf]);
+          ++it;
+        }
+        s_consumed = it;
+        tc_commit(&done_bar);
+        int never = 0;
+        mbar_wait(&done_bar, 0, &never, status);
+      }
+    }
+    asm volatile("bar.sync 0;" ::: "memory");
+    if (warp == 0 && lane == 0) {
       int never = 0;
-      mbar_wait(&done_bar, 0, &never, status);
+      for (uint32_t j = s_consumed; j < issued; ++j)
+        mbar_wait(&full_bar[j % R_STAGES], (j / R_STAGES) & 1u, &never, status);
+    }
+    tc_fence_before();
+    asm volatile("bar.sync 0;" ::: "memory");
+    if (warp == 1) {
+      tc_fence_after();
+      tmem_dealloc(tmem_base, R_TMEM_COLS);
     }
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(R_EPILOGUE_REGS));
+    // warp w reads TMEM lanes 32*(w%4).. (its 32 tokens) and one half of the
+    // 256 expert columns
     const int q = warp & 3;
-    const int r_in = q * 32 + lane;
-    const int t = t0 + r_in;
-    float acc[RN];
+    const int half = (warp - R_FIRST_EPI_WARP) >> 2;
+    const int t = t0 + q * 32 + lane;
+    float acc[RN / 2];
 #pragma unroll
-    for (int j = 0; j < RN; ++j) acc[j] = 0.0f;
+    for (int j = 0; j < RN / 2; ++j) acc[j] = 0.0f;
     bool ok = true;
     for (int kb = 0; kb < n; ++kb) {
       const uint32_t buf = kb & 1u, tph = (kb >> 1) & 1u;
       if (!mbar_wait(&tfull_bar[buf], tph, s_abort, status)) { ok = false; break; }
       tc_fence_after();
-      const uint32_t tbase = tmem_base + (uint32_t(q * 32) << 16) + buf * RN;
+      const uint32_t tbase = tmem_base + (uint32_t(q * 32) << 16) + buf * RN + half * (RN / 2);
 #pragma unroll
-      for (int c = 0; c < RN / 32; c += 2) {
+      for (int c = 0; c < RN / 2 / 32; c += 2) {
         float va[32], vb[32];
         tmem_ld32(tbase + c * 32, va);
         tmem_ld32(tbase + c * 32 + 32, vb);
         tmem_ld_wait();
+        if (c + 2 >= RN / 2 / 32) {   // the buffer is in registers: hand it back
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tempty_bar[buf]);
+        }
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
           acc[c * 32 + j] += va[j];
           acc[c * 32 + 32 + j] += vb[j];
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty_bar[buf]);
     }
+    const int eh = e0 + half * (RN / 2);
     if (ok && t < T) {
-      float* dst = partial + (size_t(split) * T + t) * E + e0;
-      if (e0 + RN <= E && (E % 4) == 0) {
+      float* dst = partial + (size_t(split) * T + t) * E + eh;
+      if (eh + RN / 2 <= E && (E % 4) == 0) {
 #pragma unroll
-        for (int j = 0; j < RN; j += 4)
+        for (int j = 0; j < RN / 2; j += 4)
           *reinterpret_cast<float4*>(dst + j) = make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
       } else {
 #pragma unroll
-        for (int j = 0; j < RN; ++j)
-          if (e0 + j < E) dst[j] = acc[j];
+        for (int j = 0; j < RN / 2; ++j)
+          if (eh + j < E) dst[j] = acc[j];
       }
     }
-  }
-
-  __syncthreads();
-  if (warp == 0 && lane == 0) {
-    int never = 0;
-    for (uint32_t j = s_consumed; j < issued; ++j)
-      mbar_wait(&full_bar[j % R_STAGES], (j / R_STAGES) & 1u, &never, status);
-  }
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem_base, R_TMEM_COLS);
+    asm volatile("bar.sync 0;" ::: "memory");
+    tc_fence_before();
+    asm volatile("bar.sync 0;" ::: "memory");
   }
 }
 
@@ -284,7 +304,20 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const TopkArgs a) {
   for (int j = 0; j < 8; ++j) l[j] = 0.0f;
   const float* pt = a.partial + size_t(t) * E + lane;
   const size_t ps = size_t(a.T) * E;
-  for (int s = 0; s < a.S; ++s) {
+  // four split slices in flight at a time; the sum stays in split order
+  int s = 0;
+  for (; s + 4 <= a.S; s += 4) {
+    float v[4][8];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[u][j] = (lane + 32 * j < E) ? __ldg(pt + (s + u) * ps + 32 * j) : 0.0f;
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int j = 0; j < 8; ++j) l[j] += v[u][j];
+  }
+  for (; s < a.S; ++s) {
     float v[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) v[j] = (lane + 32 * j < E) ? __ldg(pt + s * ps + 32 * j) : 0.0f;
@@ -421,6 +454,12 @@ cudaError_t launch_route(const moe_layer_s* L, const uint16_t* x, int T, int ldx
                          float* logits, float* partial, cudaStream_t st) {
   static std::atomic<bool> configured[kMaxDevices];   // the attribute is per device
   cudaError_t ce = once_per_device(configured, []() {
+    // setmaxnreg.inc draws on the CTA's launch registers: refuse a build
+    // whose register count cannot fund the split
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, route_tc_kernel);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs * R_THREADS < 128 * R_PRODUCER_REGS + 256 * R_EPILOGUE_REGS) return cudaErrorInvalidConfiguration;
     return cudaFuncSetAttribute(route_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, R_SMEM_DYN);
   });
   if (ce != cudaSuccess) return ce;

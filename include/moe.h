@@ -111,7 +111,10 @@ typedef struct {
  *   router_w     : [E][H] fp32, row-major
  *   router_bias  : [E] fp32 or NULL; selection-only bias of routers balanced
  *                  by a bias instead of an auxiliary loss (added to the
- *                  softmax probabilities to choose experts, not to weigh them) */
+ *                  softmax probabilities to choose experts, not to weigh them)
+ * The six expert arrays may all be NULL (then ld_h/ld_f are ignored): a
+ * routing-only handle for route, permute and combine, as the source side of
+ * expert parallelism uses (see moe_ep_regroup). */
 typedef struct {
   const uint8_t* w_gate;
   const uint8_t* w_up;
@@ -245,6 +248,55 @@ moe_status moe_gate_up(moe_layer_t layer, const uint8_t* xq, const float* xs, co
 moe_status moe_down(moe_layer_t layer, const uint8_t* h, const float* hs, const int32_t* offsets, int T,
                     uint16_t* y, void* stream);
 
+/* moe_gate_up / moe_down over an explicit row count instead of T (the rows
+ * of an expert-parallel owner: the routed rows it received plus its own
+ * shared rows; see moe_ep_regroup). The SwiGLU experts of
+ * Dots3NoteTextConfig with the fine-grained FP8 weights of transformers
+ * PR #47844, as cited at moe_expert_ffn.
+ *   rows     the permuted row count: xq/h have `rows` rows and the scale
+ *            arrays are group-major with group stride `rows`
+ *   offsets  [E+2] group offsets over those rows (group E: shared rows) */
+moe_status moe_grouped_gate_up(moe_layer_t layer, const uint8_t* xq, const float* xs, const int32_t* offsets,
+                               int rows, uint8_t* h, float* hs, void* stream);
+moe_status moe_grouped_down(moe_layer_t layer, const uint8_t* h, const float* hs, const int32_t* offsets, int rows,
+                            uint16_t* y, void* stream);
+
+/* Expert parallelism (SGLang cookbook "Dots3-Note", "2. Configuration
+ * Tips": the MoE layer served with expert parallelism across the GPUs of a
+ * node, DeepEP carrying the dispatch and combine all-to-alls). The routed
+ * experts are split into `ranks` contiguous blocks of El experts (rank p
+ * owns experts [p*El, (p+1)*El)); the shared expert and the router are on
+ * every rank. A source rank routes and permutes its own tokens with a
+ * routing-only handle (moe_layer_create with all six expert arrays NULL:
+ * route, permute and combine work, the GEMM calls return
+ * MOE_ERR_INVALID_ARG); its rows for rank p are then one contiguous range.
+ * An owner rank runs the GEMMs with a handle of its El experts plus the
+ * shared expert (n_routed = El). These three calls move rows around the two
+ * exchanges (which the caller performs, e.g. NCCL all-to-all); with
+ * seg_counts[s*El + e] = the rows sender s sent for local expert e and
+ * n_recv = their sum:
+ * moe_ep_pack_scales (source side, route handle): xs_rows [T*K][H/128] fp32
+ *   = the routed rows' scales of xs [H/128][T*(K+S)] made row-major, so a
+ *   destination's rows and their scales are contiguous.
+ * moe_ep_regroup (owner side, expert handle): recv_q [n_recv][H] bytes and
+ *   recv_s [n_recv][H/128] fp32 in sender-major order (sender 0's rows for
+ *   local experts 0..El-1, then sender 1's, ...), plus the owner's own
+ *   shared rows (own_q/own_s: its moe_permute outputs for T tokens, rows
+ *   [T*K, T*K + T*S)) -> out_q [n_recv + T*S][H] expert-major with the shared
+ *   rows last, out_s [H/128][n_recv + T*S] group-major, out_offsets [El+2]
+ *   (for moe_grouped_gate_up / moe_grouped_down with rows = n_recv + T*S).
+ * moe_ep_unregroup (owner side, expert handle): y_g [n_recv + T*S][H] bf16
+ *   (the grouped GEMM output) -> y_send [n_recv][H] in the sender-major
+ *   order of recv_q (for the return exchange) and the shared rows into
+ *   y_own rows [T*K, T*K + T*S) (the owner's own moe_combine input).
+ * seg_counts is a device array; ranks * El <= 2048. */
+moe_status moe_ep_pack_scales(moe_layer_t route_layer, const float* xs, int T, float* xs_rows, void* stream);
+moe_status moe_ep_regroup(moe_layer_t expert_layer, int ranks, const int32_t* seg_counts, int n_recv,
+                          const uint8_t* recv_q, const float* recv_s, const uint8_t* own_q, const float* own_s, int T,
+                          uint8_t* out_q, float* out_s, int32_t* out_offsets, void* stream);
+moe_status moe_ep_unregroup(moe_layer_t expert_layer, int ranks, const int32_t* seg_counts, int n_recv,
+                            const uint16_t* y_g, int T, uint16_t* y_send, uint16_t* y_own, void* stream);
+
 /* Weighted combine of the routed experts' outputs plus the shared expert's
  * (Dots3NoteTextConfig: norm_topk_prob, routed_scaling_factor,
  * n_shared_experts 1), the "combine" of the DeepEP transport of the SGLang
@@ -276,7 +328,7 @@ moe_status moe_layer_forward(moe_layer_t layer, const uint16_t* x, int T, int ld
 moe_status moe_get_device_status(moe_layer_t layer, void* stream, uint32_t* detail);
 
 /* Number of kernels moe_layer_forward launches for T tokens (route 2,
- * permute 5, gate/up 1, down 1 plus 1 when its K blocks are split, combine
+ * permute 4, gate/up 1, down 1 plus 1 when its K blocks are split, combine
  * 1); 0 for T = 0 or bad arguments. Library plumbing: no counterpart on the
  * pages. */
 int moe_kernels_per_forward(moe_layer_t layer, int T);

@@ -1,0 +1,136 @@
+"""Expert parallelism on CPU ranks over gloo: the library's orchestration
+(fp8_expert_ffn_b200.ep: dispatch planning, count exchange, the three
+all-to-alls and their split sizes) driven with CPU stand-ins for the
+kernels, built from the oracle (test infrastructure). Each rank's output must
+equal the oracle's single-rank layer on the same tokens, which holds only if
+every row reaches the rank that owns its expert and comes back to its place.
+The kernels themselves are checked on one GPU with emulated ranks
+(tests/test_gpu_ep.py)."""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+class HostOps:
+    """The layer's steps on CPU (oracle arithmetic), in the interface of
+    fp8_expert_ffn_b200.ep.CudaOps."""
+
+    def __init__(self, layer, rank, ranks):
+        import gen
+        from oracle import moe
+        self.moe, self.layer = moe, layer
+        sh = layer.shape
+        self.H, self.E, self.K, self.S, self.HB = sh.H, sh.E, sh.K, sh.S, sh.HB
+        self.ranks, self.rank = ranks, rank
+        self.El = sh.E // ranks
+        self.device = "cpu"
+        e0 = rank * self.El
+        keep = list(range(e0, e0 + self.El)) + ([sh.E] if sh.S else [])
+        ls = gen.LayerShape(H=sh.H, E=self.El, K=sh.K, F=sh.F, ld_f=sh.ld_f, S=sh.S)
+        self.local = gen.Layer(ls, layer.router_w[e0:e0 + self.El], layer.w_gate[keep], layer.s_gate[keep],
+                               layer.w_up[keep], layer.s_up[keep], layer.w_down[keep], layer.s_down[keep])
+
+    def route_permute(self, x, T):
+        m = self.moe
+        r = m.route_layer(x, self.layer)
+        p = m.permute(r.idx, self.E, self.S)
+        tq, ts = m.quantize_tokens(x)
+        return {"w": r.w, "inv": p.inv, "xq": tq[p.perm], "xs": ts[p.perm]}, p.offsets
+
+    def send_buffers(self, st, T):
+        R = T * self.K
+        return torch.from_numpy(np.ascontiguousarray(st["xq"][:R])), torch.from_numpy(np.ascontiguousarray(st["xs"][:R]))
+
+    def recv_buffers(self, n):
+        return torch.empty((n, self.H), dtype=torch.uint8), torch.empty((n, self.HB), dtype=torch.float32)
+
+    def experts(self, st, disp, recv_q, recv_s, T):
+        P, El, R = self.ranks, self.El, T * self.K
+        cnt = disp.recv                                     # [sender][local expert]
+        start = np.concatenate([[0], np.cumsum(cnt.ravel())])[:-1].reshape(P, El)   # sender-major
+        order = [np.arange(start[s, e], start[s, e] + cnt[s, e]) for e in range(El) for s in range(P)]
+        order = np.concatenate(order).astype(np.int64) if order else np.zeros(0, np.int64)
+        q = np.concatenate([recv_q.numpy()[order], st["xq"][R:R + T * self.S]])
+        s = np.concatenate([recv_s.numpy()[order], st["xs"][R:R + T * self.S]])
+        off = np.concatenate([[0], np.cumsum(cnt.sum(0)), [len(order) + T * self.S]]).astype(np.int64)
+        y = self.moe.expert_ffn_rows(q, s, off, self.local)["y"]
+        y_send = np.empty((disp.n_recv, self.H))
+        y_send[order] = y[:len(order)]
+        y_own = np.zeros((T * (self.K + self.S), self.H))
+        y_own[R:] = y[len(order):]
+        return torch.from_numpy(y_send), torch.from_numpy(y_own)
+
+    def combine(self, st, y_own, T):
+        return self.moe.combine(y_own.numpy(), st["inv"], st["w"], self.S)
+
+
+def _worker(rank, world, port, T, q, idle_rank=-1):
+    import sys
+    sys.path.insert(0, ROOT)
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        import gen
+        from fp8_expert_ffn_b200 import ep
+        from oracle import moe
+        _, layer, _ = gen.workload_inputs("toy")
+        Tr = 0 if rank == idle_rank else T
+        x = gen.make_x(Tr, layer.shape.H, 100 + rank, outliers=2)   # each rank has its own tokens
+        out = ep.ep_forward(HostOps(layer, rank, world), ep.TorchExchange(), x, Tr)
+        if Tr == 0:
+            err = 0.0 if out.shape == (0, layer.shape.H) else 1.0
+        else:
+            ref = moe.layer_forward(x, layer)["out"]
+            err = float(np.max(np.abs(out - ref)) / np.max(np.abs(ref)))
+        sent = ep.plan_dispatch(moe.permute(moe.route_layer(x, layer).idx, layer.shape.E).offsets,
+                                layer.shape.E, world)
+        q.put((rank, err, int(sent.sum()) + (T * 4 if Tr == 0 else 0)))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,idle", [(2, -1), (4, -1), (2, 1)])
+def test_expert_parallel_forward_matches_single_rank(world, idle):
+    """world ranks of 24 tokens each; with idle >= 0 that rank has no tokens
+    (it still serves its experts and takes part in every exchange)."""
+    T = 24
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, T, q, idle)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=180)
+    assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]
+    res = sorted(q.get(timeout=10) for _ in range(world))
+    for rank, err, sent in res:
+        assert err <= 1e-12, (rank, err)
+        assert sent == T * 4          # every routed row (T x top-4) is dispatched once
+
+
+def test_plan_dispatch_splits_rows_by_owner():
+    from fp8_expert_ffn_b200 import ep
+    E, P = 8, 4
+    counts = np.array([3, 0, 2, 5, 1, 1, 0, 4])
+    offsets = np.concatenate([[0], np.cumsum(counts), [counts.sum() + 6]])
+    plan = ep.plan_dispatch(offsets, E, P)
+    assert plan.tolist() == [[3, 0], [2, 5], [1, 1], [0, 4]]
+    d = ep.Dispatch(plan, plan[::-1].copy())
+    assert d.send_rows == [3, 7, 2, 4] and d.recv_rows == [4, 2, 7, 3] and d.n_recv == 16
+    with pytest.raises(ValueError):
+        ep.local_experts(10, 4)

@@ -1,0 +1,167 @@
+"""Expert parallelism through the library's kernels on one GPU: P emulated
+ranks run as threads, each with a routing-only handle over all experts and
+an expert handle over its own block of experts plus the shared expert; an
+in-process exchange stands in for the all-to-alls (no collective, no kernel
+waits on another). Each rank's output must be bit-identical to the
+single-GPU forward of the whole layer on the same tokens: a row's GEMM
+result does not depend on which rows share its tile, so any row sent to the
+wrong expert or returned to the wrong place shows up."""
+import threading
+
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+import gen  # noqa: E402
+
+pytestmark = pytest.mark.gpu
+
+if not torch.cuda.is_available():
+    pytest.skip("needs a GPU", allow_module_level=True)
+
+import fp8_expert_ffn_b200 as fx  # noqa: E402
+from fp8_expert_ffn_b200 import ep  # noqa: E402
+from fp8_expert_ffn_b200 import torch_utils as tu  # noqa: E402
+
+
+class LocalExchange:
+    """The all-to-alls between emulated ranks (threads of this process)."""
+
+    def __init__(self, ranks):
+        self.ranks = ranks
+        self.bar = threading.Barrier(ranks, timeout=300)
+        self.box = [None] * ranks
+
+    def view(self, rank):
+        return _RankView(self, rank)
+
+
+class _RankView:
+    def __init__(self, ex, rank):
+        self.ex, self.rank, self.ranks = ex, rank, ex.ranks
+
+    def counts(self, send, device):
+        self.ex.box[self.rank] = np.asarray(send)
+        self.ex.bar.wait()
+        recv = np.stack([self.ex.box[s][self.rank] for s in range(self.ranks)]).astype(np.int64)
+        self.ex.bar.wait()
+        return recv
+
+    def rows(self, src, send_rows, recv_rows, out):
+        torch.cuda.synchronize()
+        self.ex.box[self.rank] = (src, list(send_rows))
+        self.ex.bar.wait()
+        o = 0
+        for s in range(self.ranks):
+            ssrc, ssend = self.ex.box[s]
+            a, n = sum(ssend[:self.rank]), ssend[self.rank]
+            assert n == recv_rows[s]
+            if n:
+                out[o:o + n].copy_(ssrc[a:a + n])
+            o += n
+        torch.cuda.synchronize()
+        self.ex.bar.wait()
+        return out
+
+
+def _rank_layers(dev, sh, ranks):
+    """(routing-only handle, expert handle) per rank; the expert handle holds
+    experts [r*El, (r+1)*El) and the shared expert, contiguous."""
+    El = sh.E // ranks
+    w = dev.weights
+    route = fx.MoeLayer(sh.H, sh.E, sh.K, sh.F, fx.LayerWeights(None, None, None, None, None, None, w.router_w),
+                        n_shared=sh.S)
+    out = []
+    for r in range(ranks):
+        keep = torch.tensor(list(range(r * El, (r + 1) * El)) + [sh.E], device="cuda")
+        lw = fx.LayerWeights(*(getattr(w, k).index_select(0, keep).contiguous()
+                               for k in ("w_gate", "w_up", "w_down", "s_gate", "s_up", "s_down")),
+                             router_w=w.router_w[r * El:(r + 1) * El].contiguous())
+        out.append((route, fx.MoeLayer(sh.H, El, sh.K, sh.F, lw, ld_h=sh.H, ld_f=sh.ld_f, n_shared=sh.S)))
+    return out
+
+
+def _run(name, ranks, T, layer=None, xs=None):
+    wl, layer0, _ = gen.workload_inputs(name)
+    layer = layer0 if layer is None else layer
+    sh = layer.shape
+    dev = tu.upload_layer(layer)
+    if xs is None:
+        xs = [gen.make_x(T, sh.H, 200 + r, outliers=wl.outliers) for r in range(ranks)]
+    refs = []
+    for x in xs:
+        xt = tu.bf16_tensor(x)
+        o = torch.empty((T, sh.H), dtype=torch.bfloat16, device="cuda")
+        ws = tu.workspace(dev, T)
+        fx.moe_layer_forward(dev, xt, T, sh.H, o, sh.H, ws, ws.numel())
+        refs.append(o)
+    layers = _rank_layers(dev, sh, ranks)
+    ex = LocalExchange(ranks)
+    outs, errs = [None] * ranks, []
+
+    def one(r):
+        try:
+            torch.cuda.set_device(0)
+            ops = ep.CudaOps(layers[r][0], layers[r][1], ranks)
+            outs[r] = ep.ep_forward(ops, ex.view(r), tu.bf16_tensor(xs[r]), T)
+        except BaseException as e:   # noqa: BLE001 - re-raised below
+            errs.append(e)
+            ex.bar.abort()
+
+    th = [threading.Thread(target=one, args=(r,)) for r in range(ranks)]
+    for t in th:
+        t.start()
+    for t in th:
+        t.join()
+    if errs:
+        raise errs[0]
+    for r in range(ranks):
+        code, bits = fx.moe_get_device_status(layers[r][1])
+        assert code == fx.MOE_OK, hex(bits)
+        assert torch.equal(outs[r].view(torch.int16), refs[r].view(torch.int16)), f"rank {r} differs"
+
+
+@pytest.mark.parametrize("ranks", [2, 4])
+def test_expert_parallel_toy_layer_matches_single_gpu(ranks):
+    _run("toy", ranks, 512)
+
+
+def test_expert_parallel_full_layer_two_ranks():
+    """256 routed experts split 128 + 128, 64 tokens per rank."""
+    _run("decode", 2, 64)
+
+
+def test_expert_parallel_rank_with_no_routed_rows():
+    """A router whose top-4 always falls in rank 0's experts: rank 1 receives
+    no routed rows (n_recv = 0) and runs only its own shared rows."""
+    from oracle import moe
+    wl, layer, _ = gen.workload_inputs("toy")
+    sh = layer.shape
+    router = layer.router_w.copy()
+    router[sh.E // 2:, :] = 0.0
+    router[sh.E // 2:, 0] = -30.0       # with x[:, 0] = 1: logit -30 for experts 8..15
+    biased = gen.Layer(sh, router, layer.w_gate, layer.s_gate, layer.w_up, layer.s_up, layer.w_down, layer.s_down)
+    T = 512
+    xs = []
+    for r in range(2):
+        x = gen.make_x(T, sh.H, 200 + r, outliers=2)
+        x[:, 0] = gen.f32_to_bf16_bits(np.float32([1.0]))[0]
+        assert moe.route(x, router, sh.K).idx.max() < sh.E // 2
+        xs.append(x)
+    _run("toy", 2, T, layer=biased, xs=xs)
+
+
+def test_routing_only_handle_refuses_gemm_calls():
+    wl, layer, _ = gen.workload_inputs("toy")
+    sh = layer.shape
+    dev = tu.upload_layer(layer)
+    route = fx.MoeLayer(sh.H, sh.E, sh.K, sh.F, fx.LayerWeights(None, None, None, None, None, None,
+                                                                 dev.weights.router_w), n_shared=sh.S)
+    T = 8
+    x = torch.zeros((T, sh.H), dtype=torch.bfloat16, device="cuda")
+    out = torch.empty_like(x)
+    ws = tu.workspace(route, T)
+    with pytest.raises(fx.MoeError) as e:
+        fx.moe_layer_forward(route, x, T, sh.H, out, sh.H, ws, ws.numel())
+    assert e.value.code == fx.MOE_ERR_INVALID_ARG
