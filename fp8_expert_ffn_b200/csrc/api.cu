@@ -416,7 +416,7 @@ moe_status moe_layer_forward(moe_layer_t L, const uint16_t* x, int T, int ldx, u
 int moe_kernels_per_forward(moe_layer_t L, int T) {
   if (!L || T <= 0 || T > kMaxT) return 0;
   const int rows = T * (L->K + L->S);
-  return 2 + 4 + 1 + 1 + (down_ksplit(L, rows) > 1 ? 1 : 0) + 1;
+  return 2 + permute_kernels(L, T) + 1 + 1 + (down_ksplit(L, rows) > 1 ? 1 : 0) + 1;
 }
 
 moe_status moe_get_device_status(moe_layer_t L, void* stream, uint32_t* detail) {

@@ -68,6 +68,9 @@ cudaError_t launch_route(const moe_layer_s* L, const uint16_t* x, int T, int ldx
 cudaError_t launch_permute(const moe_layer_s* L, const uint16_t* x, int T, int ldx, const int32_t* idx,
                            int32_t* offsets, int32_t* perm, int32_t* inv, uint8_t* xq, float* xs,
                            const Scratch& s, cudaStream_t st);
+// Kernels launch_permute issues for T tokens: 2 when the token bitmap fits
+// one CTA's shared memory (one plan kernel + the gather), else 4.
+int permute_kernels(const moe_layer_s* L, int T);
 // Limits of the allocation-free permutation (moe_permute_noalloc).
 constexpr int kNoAllocMaxTokens = MOE_NOALLOC_MAX_TOKENS;
 constexpr int kNoAllocMaxExperts = 256;

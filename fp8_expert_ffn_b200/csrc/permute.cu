@@ -15,6 +15,8 @@
 //   1. permute_bitmap   one thread per (t, k): validate, set the bit
 //   2. permute_count    one CTA per expert: per-word prefix popcounts, count;
 //                       the last CTA to finish scans the counts -> offsets[E+2]
+//   (small batches: 1-3 in one CTA, permute_plan_small, when the bitmap fits
+//   in shared memory)
 //   4. permute_gather   one warp per token and 16 groups of 128 channels:
 //                       rows of its K slots and its shared-expert row,
 //                       inv/perm, then the groups of x quantised once and
@@ -122,6 +124,67 @@ __global__ void __launch_bounds__(256) permute_count_kernel(const uint32_t* __re
   }
 }
 
+// Small batches: the whole plan in one CTA. When the token bitmap (E x W
+// words) fits in shared memory, one CTA zeroes it, sets the bits, counts and
+// scans: the bitmap, the per-word prefixes and the offsets it writes are the
+// same as those of the three-kernel path (clear, bitmap, count).
+constexpr int kPlanSmallWords = 8192;     // 32 KB of shared memory
+constexpr int kPlanSmallThreads = 1024;
+
+__global__ void __launch_bounds__(kPlanSmallThreads) permute_plan_small_kernel(
+    const int32_t* __restrict__ idx, int T, int K, int E, int W, int S, uint32_t* __restrict__ bitmap,
+    uint32_t* __restrict__ wprefix, int32_t* __restrict__ counts, int32_t* __restrict__ offsets, uint32_t* status) {
+  pdl_wait();
+  pdl_launch_dependents();
+  __shared__ uint32_t s_bits[kPlanSmallWords];
+  __shared__ int s_cnt[256];
+  __shared__ int s_wsum[kPlanSmallThreads / 32];
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  const int nw = E * W;
+  for (int i = tid; i < nw; i += kPlanSmallThreads) s_bits[i] = 0u;
+  __syncthreads();
+  for (int i = tid; i < T * K; i += kPlanSmallThreads) {
+    const int t = i / K, e = idx[i];
+    if (e < 0 || e >= E) {
+      set_status(status, STATUS_BAD_EXPERT);
+      continue;
+    }
+    const uint32_t bit = 1u << (t & 31);
+    if (atomicOr(&s_bits[e * W + (t >> 5)], bit) & bit) set_status(status, STATUS_DUP_EXPERT);
+  }
+  __syncthreads();
+  // expert e: prefix popcounts over its W words (one thread per expert)
+  for (int e = tid; e < E; e += kPlanSmallThreads) {
+    uint32_t run = 0;
+    for (int w = 0; w < W; ++w) {
+      const uint32_t b = s_bits[e * W + w];
+      bitmap[size_t(e) * W + w] = b;
+      wprefix[size_t(e) * W + w] = run;
+      run += __popc(b);
+    }
+    s_cnt[e] = int(run);
+    counts[e] = int(run);
+  }
+  __syncthreads();
+  // exclusive scan of the E <= 256 counts
+  const int v = tid < E ? s_cnt[tid] : 0;
+  int inc = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int o = __shfl_up_sync(0xFFFFFFFFu, inc, off);
+    if (lane >= off) inc += o;
+  }
+  if (lane == 31) s_wsum[wid] = inc;
+  __syncthreads();
+  int base = 0;
+  for (int j = 0; j < wid; ++j) base += s_wsum[j];
+  if (tid < E) offsets[tid] = base + inc - v;
+  if (tid == E - 1) {
+    offsets[E] = base + inc;
+    offsets[E + 1] = base + inc + T * S;
+  }
+}
+
 constexpr int GATHER_GROUPS = 16;   // 128-channel groups per warp (4 steps of 4 groups)
 
 // One warp per (token, chunk of GATHER_GROUPS groups). In each step the warp
@@ -222,6 +285,10 @@ __global__ void __launch_bounds__(256) permute_gather_kernel(
 
 }  // namespace
 
+int permute_kernels(const moe_layer_s* L, int T) {
+  return size_t(L->E) * ((T + 31) / 32) <= size_t(kPlanSmallWords) ? 2 : 4;
+}
+
 cudaError_t launch_permute(const moe_layer_s* L, const uint16_t* x, int T, int ldx, const int32_t* idx,
                            int32_t* offsets, int32_t* perm, int32_t* inv, uint8_t* xq, float* xs,
                            const Scratch& s, cudaStream_t st) {
@@ -229,16 +296,23 @@ cudaError_t launch_permute(const moe_layer_s* L, const uint16_t* x, int T, int l
   const int S = L->S;
   const int rows = T * (K + S);
   const size_t nwords = size_t(E) * W;
-  uint32_t* done = reinterpret_cast<uint32_t*>(s.counts + E);
-  cudaError_t e = launch_pdl(permute_clear_kernel, dim3(unsigned((nwords + 1023) / 1024)), dim3(256), 0, st,
-                             s.bitmap, nwords, done);
-  if (e != cudaSuccess) return e;
-  e = launch_pdl(permute_bitmap_kernel, dim3((T * K + 255) / 256), dim3(256), 0, st, idx, T, K, E, W, s.bitmap,
-                 L->status);
-  if (e != cudaSuccess) return e;
-  e = launch_pdl(permute_count_kernel, dim3(E), dim3(256), 0, st, static_cast<const uint32_t*>(s.bitmap), W,
-                 s.wprefix, s.counts, E, T, S, offsets, done);
-  if (e != cudaSuccess) return e;
+  cudaError_t e;
+  if (permute_kernels(L, T) == 2) {
+    e = launch_pdl(permute_plan_small_kernel, dim3(1), dim3(kPlanSmallThreads), 0, st, idx, T, K, E, W, S, s.bitmap,
+                   s.wprefix, s.counts, offsets, L->status);
+    if (e != cudaSuccess) return e;
+  } else {
+    uint32_t* done = reinterpret_cast<uint32_t*>(s.counts + E);
+    e = launch_pdl(permute_clear_kernel, dim3(unsigned((nwords + 1023) / 1024)), dim3(256), 0, st, s.bitmap, nwords,
+                   done);
+    if (e != cudaSuccess) return e;
+    e = launch_pdl(permute_bitmap_kernel, dim3((T * K + 255) / 256), dim3(256), 0, st, idx, T, K, E, W, s.bitmap,
+                   L->status);
+    if (e != cudaSuccess) return e;
+    e = launch_pdl(permute_count_kernel, dim3(E), dim3(256), 0, st, static_cast<const uint32_t*>(s.bitmap), W,
+                   s.wprefix, s.counts, E, T, S, offsets, done);
+    if (e != cudaSuccess) return e;
+  }
   const int nchunk = (L->HB + GATHER_GROUPS - 1) / GATHER_GROUPS;
   const long long warps = static_cast<long long>(T) * nchunk;
   return launch_pdl(permute_gather_kernel, dim3(unsigned((warps + 7) / 8)), dim3(256), 0, st, x, T, ldx, L->H, idx,

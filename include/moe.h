@@ -328,8 +328,9 @@ moe_status moe_layer_forward(moe_layer_t layer, const uint16_t* x, int T, int ld
 moe_status moe_get_device_status(moe_layer_t layer, void* stream, uint32_t* detail);
 
 /* Number of kernels moe_layer_forward launches for T tokens (route 2,
- * permute 4, gate/up 1, down 1 plus 1 when its K blocks are split, combine
- * 1); 0 for T = 0 or bad arguments. Library plumbing: no counterpart on the
+ * permute 2 when the E x ceil(T/32)-word token bitmap fits in 8192 words,
+ * else 4, gate/up 1, down 1 plus 1 when its K blocks are split, combine 1);
+ * 0 for T = 0 or bad arguments. Library plumbing: no counterpart on the
  * pages. */
 int moe_kernels_per_forward(moe_layer_t layer, int T);
 

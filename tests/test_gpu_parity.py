@@ -589,13 +589,57 @@ def test_split_k_down_exact_integers():
 
 
 def test_kernels_per_forward():
-    """The launch count bench.py reports: 9 kernels per forward, 10 when the
-    down GEMM splits its K blocks (the dense FFN at T = 64)."""
+    """The launch count bench.py reports: route 2, permute 2 while the
+    E x ceil(T/32)-word token bitmap fits one CTA (8192 words: T <= 1024 at
+    E = 256) else 4, gate/up 1, down 1 (+1 when it splits its K blocks, as
+    the dense FFN does at T = 64), combine 1."""
     _, _, c = get_case("decode")
-    assert fx.moe_kernels_per_forward(c.dev, c.T) == 9
+    assert fx.moe_kernels_per_forward(c.dev, c.T) == 7
+    assert fx.moe_kernels_per_forward(c.dev, 1024) == 7
+    assert fx.moe_kernels_per_forward(c.dev, 1025) == 9
+    assert fx.moe_kernels_per_forward(c.dev, 16384) == 9
     assert fx.moe_kernels_per_forward(c.dev, 0) == 0
     _, _, cd = get_case("dense")
-    assert fx.moe_kernels_per_forward(cd.dev, cd.T) == 10
+    assert fx.moe_kernels_per_forward(cd.dev, cd.T) == 8
+
+
+@pytest.mark.parametrize("T", [1, 31, 1024, 1025, 3000])
+def test_permute_plan_paths_on_the_full_router(T):
+    """Both plans of the permutation (one CTA while the 256-expert token
+    bitmap fits 8192 words, T <= 1024; three kernels above) give the oracle's
+    offsets, perm and inv bit-exactly on Zipf-skewed routing of the full
+    layer, and both flag an out-of-range and a repeated expert id."""
+    wl, layer, c = get_case("decode")
+    sh = layer.shape
+    rng = np.random.default_rng(T)
+    pz = 1.0 / np.arange(1, sh.E + 1) ** 1.1
+    pz /= pz.sum()
+    idx_np = np.stack([rng.choice(sh.E, sh.K, replace=False, p=pz) for _ in range(T)]).astype(np.int32)
+    x = tu.bf16_tensor(gen.make_x(T, sh.H, 77, outliers=2))
+    rows = T * (sh.K + sh.S)
+
+    def run(ix):
+        off = torch.empty(sh.E + 2, dtype=torch.int32, device="cuda")
+        perm = torch.full((rows,), -7, dtype=torch.int32, device="cuda")
+        inv = torch.empty((T, sh.K), dtype=torch.int32, device="cuda")
+        xq = torch.empty((rows, sh.H), dtype=torch.uint8, device="cuda")
+        xs = torch.empty((sh.HB, rows), dtype=torch.float32, device="cuda")
+        ws = tu.workspace(c.dev, T)
+        fx.moe_permute(c.dev, x, T, sh.H, torch.from_numpy(ix).cuda(), off, perm, inv, xq, xs, ws, ws.numel())
+        return off.cpu().numpy(), perm.cpu().numpy(), inv.cpu().numpy()
+
+    off, perm, inv = run(idx_np)
+    assert fx.moe_get_device_status(c.dev)[0] == fx.MOE_OK
+    p = moe.permute(idx_np, sh.E, sh.S)
+    assert np.array_equal(off, p.offsets) and np.array_equal(perm, p.perm) and np.array_equal(inv, p.inv)
+    bad = idx_np.copy()
+    bad[T - 1, 0] = sh.E                   # out of range
+    if T > 1:
+        bad[0, sh.K - 1] = bad[0, 0]       # repeated within token 0
+    run(bad)
+    code, bits = fx.moe_get_device_status(c.dev)
+    assert code == fx.MOE_ERR_DEVICE and bits & 1
+    assert T == 1 or bits & 2
 
 
 def test_forward_is_cuda_graph_capturable():
