@@ -1,11 +1,13 @@
 """Benchmark of the FP8 MoE-layer forward (dots3-note preview shape) on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload decode|prefill|zipf|edge|edge_f1500|...] [--no-workloads]
+                    [--workload decode|prefill|zipf|edge|edge_f1500|...] [--no-workloads] [--ep]
 
 One step = one whole forward of the layer (route, permute + quantise, gate/up
 GEMM + SwiGLU + quantise, down GEMM, combine) over one batch of T tokens
-whose inputs already sit in HBM. With N > 1 (torchrun, one rank per GPU) every
+whose inputs already sit in HBM, timed through moe_layer_forward; a second
+timed pass calls the stages one by one with CUDA events between them for the
+per-stage times and the kernel rooflines. With N > 1 (torchrun, one rank per GPU) every
 rank runs an independent replica of the layer on its own batch: the layer has
 no exchange step on one node at this scale, so the job is weak-scaled and the
 value is all ranks' tokens over the slowest rank's device time.
@@ -16,6 +18,9 @@ T=16384, edge T=4099 and its FFN=1500 variant) timed the same way, with both
 roofline fractions (measured HBM copy bandwidth; dense FP8 = 2 x the measured
 BF16 burst GEMM rate), its own clock sample and the C++ FP64 oracle timed on
 that workload's own tokens. The toy layer is a parity case only.
+
+With --ep the ranks run the layer expert-parallel instead (run_ep): a
+separate line, not the replica measurement above.
 
 Prints one JSON line (rank 0).
 """
@@ -52,6 +57,9 @@ def parse():
                             "dense"])
     p.add_argument("--no-workloads", action="store_true", help="time only --workload (no workloads block)")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--ep", action="store_true",
+                   help="expert parallelism over the ranks instead of replicas: the routed experts split into "
+                        "equal blocks, one per rank, with the all-to-alls over torch.distributed (NCCL)")
     return p.parse_args()
 
 
@@ -102,10 +110,10 @@ class Dist:
     only collectives are the barriers around the timed region and the
     reductions of the timing (max over ranks) and of the token count (sum)."""
 
-    def __init__(self, world, rank, local, backend="nccl", timeout_s=600):
+    def __init__(self, world, rank, local, backend="nccl", timeout_s=600, group_always=False):
         import torch.distributed as dist
         self.world, self.rank, self.local = world, rank, local
-        self.dist = dist if world > 1 else None
+        self.dist = dist if (world > 1 or group_always) else None
         self.device = "cuda" if backend == "nccl" else "cpu"
         if self.dist:
             from datetime import timedelta
@@ -323,34 +331,88 @@ def time_stages(st: Stages, steps: int, warmup: int, d: Dist, sampler=None):
     return total_ms, per, clocks
 
 
+def time_forward(st: Stages, steps: int, warmup: int, d: Dist, sampler=None):
+    """The whole forward as a user calls it: one moe_layer_forward per step
+    (its kernels chained by programmatic dependent launch, no event between
+    them), CUDA events on the launching stream around the timed steps. The
+    per-stage breakdown comes from time_stages, whose events between the
+    stages break that chaining."""
+    import torch
+    fx, dev, T, H = st.fx, st.dev, st.T, st.sh.H
+    for _ in range(warmup):
+        fx.moe_layer_forward(dev, st.x, T, H, st.out, H, st.ws, st.ws.numel())
+    torch.cuda.synchronize()
+    d.barrier()
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.start()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        fx.moe_layer_forward(dev, st.x, T, H, st.out, H, st.ws, st.ws.numel())
+    b.record()
+    torch.cuda.synchronize()
+    clocks = sampler.stop() if sampler else None
+    d.barrier()
+    torch.cuda.synchronize()
+    code, bits = fx.moe_get_device_status(dev)
+    if code != 0:
+        raise RuntimeError(f"device status {bits:#x}")
+    return a.elapsed_time(b), clocks
+
+
 def time_e2e(dev, sh, x_bits, steps, warmup, d: Dist):
-    """Through moe_layer_forward with host buffers: pinned host x -> device,
-    forward, device -> pinned host out, all inside the timed region."""
+    """Through moe_layer_forward with host buffers, pipelined the way a serving
+    loop runs it: step i's input is copied from pinned host memory to the
+    device, and step i's output back, on a copy stream, while the forwards
+    run in order on the compute stream (double-buffered device input and
+    output). Every step's two copies are inside the timed region, which runs
+    from before the first upload to after the last download."""
     import torch
     import fp8_expert_ffn_b200 as fx
     from fp8_expert_ffn_b200 import torch_utils as tu
     T, H = x_bits.shape
     x_host = torch.from_numpy(np.ascontiguousarray(x_bits).view(np.int16)).view(torch.bfloat16).pin_memory()
-    out_host = torch.empty((T, H), dtype=torch.bfloat16).pin_memory()
-    x_dev = torch.empty((T, H), dtype=torch.bfloat16, device="cuda")
-    out_dev = torch.empty((T, H), dtype=torch.bfloat16, device="cuda")
+    out_host = [torch.empty((T, H), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    x_dev = [torch.empty((T, H), dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+    out_dev = [torch.empty((T, H), dtype=torch.bfloat16, device="cuda") for _ in range(2)]
     ws = tu.workspace(dev, T)
+    comp, copy = torch.cuda.current_stream(), torch.cuda.Stream()
+    h2d = [torch.cuda.Event() for _ in range(2)]
+    fwd = [torch.cuda.Event() for _ in range(2)]
+    d2h = [torch.cuda.Event() for _ in range(2)]
 
-    def one():
-        x_dev.copy_(x_host, non_blocking=True)
-        fx.moe_layer_forward(dev, x_dev, T, H, out_dev, H, ws, ws.numel())
-        out_host.copy_(out_dev, non_blocking=True)
+    def run(n, start=None, end=None):
+        with torch.cuda.stream(copy):
+            if start is not None:
+                start.record(copy)
+            x_dev[0].copy_(x_host, non_blocking=True)
+            h2d[0].record(copy)
+        for i in range(n):
+            b = i & 1
+            comp.wait_event(h2d[b])
+            if i >= 2:
+                comp.wait_event(d2h[b])          # out_dev[b]'s previous download is done
+            fx.moe_layer_forward(dev, x_dev[b], T, H, out_dev[b], H, ws, ws.numel(), stream=comp)
+            fwd[b].record(comp)
+            with torch.cuda.stream(copy):
+                if i + 1 < n:                   # next step's upload, overlapping this forward
+                    if i >= 1:
+                        copy.wait_event(fwd[1 - b])   # x_dev[1-b] was read by the previous forward
+                    x_dev[1 - b].copy_(x_host, non_blocking=True)
+                    h2d[1 - b].record(copy)
+                copy.wait_event(fwd[b])
+                out_host[b].copy_(out_dev[b], non_blocking=True)
+                d2h[b].record(copy)
+        if end is not None:
+            end.record(copy)
 
-    for _ in range(warmup):
-        one()
+    run(warmup)
     torch.cuda.synchronize()
     d.barrier()
     torch.cuda.synchronize()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record()
-    for _ in range(steps):
-        one()
-    b.record()
+    run(steps, a, b)
     torch.cuda.synchronize()
     d.barrier()
     return a.elapsed_time(b), T * H * 2, T * H * 2
@@ -418,8 +480,10 @@ def measure_workload(name, d, rank, args, pk, sampler, oracle=True):
     wl, host, dev, x_bits = load_layer(name, d, rank)
     st = Stages(dev, wl.shape, wl.T, tu.bf16_tensor(x_bits))
     steps = max(10, args.steps)
-    total_ms, per, clocks = time_stages(st, steps, max(3, min(args.warmup, 5)), d, sampler)
+    warm = max(3, min(args.warmup, 5))
+    total_ms, clocks = time_forward(st, steps, warm, d, sampler)
     total_ms = d.max(total_ms)
+    _, per, _ = time_stages(st, steps, warm, d)
     off = st.offsets.cpu().numpy()
     work = algorithmic_work(wl, wl.T, off)
     counts = np.diff(off)[:wl.shape.E]
@@ -443,6 +507,15 @@ WORKLOADS = ("decode", "prefill", "zipf", "edge", "edge_f1500")
 
 # ----------------------------------------------------------------------------- arms
 
+def workload_config(wl, world, touched):
+    """The config block of a line (the same in both arms)."""
+    sh = wl.shape
+    return {"workload": f"{wl.name}: {wl.note}", "T": wl.T, "hidden": sh.H, "experts": f"{sh.E}+{sh.S}",
+            "top_k": sh.K, "ffn": sh.F, "weights": "FP8 E4M3, 128x128 fp32 block scales, seeded synthetic",
+            "l2": "inputs larger than L2 (each step streams the touched experts' weights, GBs >> 126 MB)",
+            "parallelism": f"replicas x{world}", "touched_groups": int(touched)}
+
+
 def run_ours(args):
     import torch
     world, rank, local = dist_setup(args.gpus)
@@ -457,8 +530,9 @@ def run_ours(args):
     st = Stages(dev, sh, T, x)
     visible = os.environ.get("CUDA_VISIBLE_DEVICES", "")
     sampler = ClockSampler(visible.split(",")[local] if visible else local)
-    total_ms, per, clocks = time_stages(st, args.steps, args.warmup, d, sampler)
+    total_ms, clocks = time_forward(st, args.steps, args.warmup, d, sampler)
     value, total_ms, tokens = job_throughput(d, float(T * args.steps), total_ms)
+    _, per, _ = time_stages(st, args.steps, args.warmup, d)
     off = st.offsets.cpu().numpy()
     work = algorithmic_work(wl, T, off)
     # the dominant kernel: decode-sized batches are bound by streaming the
@@ -493,15 +567,13 @@ def run_ours(args):
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 5), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "e4m3 (fp32 accumulate)", "data": "synthetic",
-        "config": {"workload": f"{wl.name}: {wl.note}", "T": T, "hidden": sh.H, "experts": f"{sh.E}+{sh.S}",
-                   "top_k": sh.K, "ffn": sh.F, "weights": "FP8 E4M3, 128x128 fp32 block scales, seeded synthetic",
-                   "l2": "inputs larger than L2 (each step streams the touched experts' weights, GBs >> 126 MB)",
-                   "parallelism": f"replicas x{world}", "touched_groups": work["touched_groups"]},
+        "config": workload_config(wl, world, work["touched_groups"]),
         "stage_ms": {k: round(v, 5) for k, v in per.items()},
         "roofline": roof,
         "e2e": {"value": round(tokens / (e2e_ms / 1e3), 1), "unit": "tokens/s", "h2d_bytes_per_step": bi,
                 "d2h_bytes_per_step": bo, "ms_per_step": round(e2e_ms / args.steps, 5)},
-        # the library's own count for one forward (10, or 11 with a split down GEMM)
+        # the library's own count for one forward (route 2, permute 2 or 4,
+        # gate/up 1, down 1 or 2, combine 1)
         "gpu_launches": st.fx.moe_kernels_per_forward(dev, T) * args.steps,
         "clocks": clocks,
     }
@@ -524,6 +596,99 @@ def run_ours(args):
     d.close()
 
 
+def run_ep(args):
+    """--ep: one expert-parallel forward per step on every rank (its own T
+    tokens of the workload; fp8_expert_ffn_b200.ep.ep_forward): route and
+    permute against all E experts, exchange the row counts, dispatch the FP8
+    rows and scales, grouped GEMMs over the rank's E/P experts plus the shared
+    expert, return the rows, combine. The exchanges are torch.distributed
+    all-to-alls (NCCL; a one-rank group when run alone). Timed like the
+    replica arm (CUDA events on the compute stream, barriers on both sides,
+    max over ranks); the orchestration's two host reads of the counts are
+    inside the timed region. Each rank's output is checked bit for bit
+    against the single-GPU forward of the whole layer on the same tokens, and
+    that forward's own time is reported beside it."""
+    import torch
+    from fp8_expert_ffn_b200 import ep
+    from fp8_expert_ffn_b200 import torch_utils as tu
+    import fp8_expert_ffn_b200 as fx
+    world, rank, local = dist_setup(args.gpus)
+    torch.cuda.set_device(local)
+    if world == 1:
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        os.environ.setdefault("MASTER_PORT", str(_free_port()))
+        os.environ.setdefault("RANK", "0")
+        os.environ.setdefault("WORLD_SIZE", "1")
+    d = Dist(world, rank, local, group_always=True)
+    wl, host, dev, x_bits = load_layer(args.workload, d, rank)
+    sh, T = wl.shape, wl.T
+    x = tu.bf16_tensor(x_bits)
+    # the single-GPU forward of the whole layer: the parity reference and the
+    # time the expert-parallel step is compared with
+    ref = torch.empty((T, sh.H), dtype=torch.bfloat16, device="cuda")
+    ws = tu.workspace(dev, T)
+    fwd = lambda: fx.moe_layer_forward(dev, x, T, sh.H, ref, sh.H, ws, ws.numel())
+    for _ in range(args.warmup):
+        fwd()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(args.steps):
+        fwd()
+    b.record()
+    torch.cuda.synchronize()
+    single_ms = d.max(a.elapsed_time(b)) / args.steps
+    route, experts = ep.rank_layers(dev, rank, world)
+    ops, ex = ep.CudaOps(route, experts, world), ep.TorchExchange()
+    for _ in range(args.warmup):
+        out = ep.ep_forward(ops, ex, x, T)
+    torch.cuda.synchronize()
+    visible = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+    sampler = ClockSampler(visible.split(",")[local] if visible else local)
+    d.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    a.record()
+    for _ in range(args.steps):
+        out = ep.ep_forward(ops, ex, x, T)
+    b.record()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    d.barrier()
+    torch.cuda.synchronize()
+    value, total_ms, tokens = job_throughput(d, float(T * args.steps), a.elapsed_time(b))
+    same = d.sum(0.0 if torch.equal(out.view(torch.int16), ref.view(torch.int16)) else 1.0)
+    for h in (route, experts, dev):
+        code, bits = fx.moe_get_device_status(h)
+        if code != fx.MOE_OK:
+            raise RuntimeError(f"device status {bits:#x}")
+    if same != 0:
+        raise RuntimeError(f"{int(same)} rank(s) differ from the single-GPU forward")
+    line = {
+        "metric": "expert-parallel MoE-layer tokens/s", "value": round(value, 1), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e4m3 (fp32 accumulate)",
+        "data": "synthetic",
+        "config": {"workload": f"{wl.name}: {wl.note}", "T_per_rank": T, "hidden": sh.H,
+                   "experts": f"{sh.E}+{sh.S}", "experts_per_rank": sh.E // world, "top_k": sh.K, "ffn": sh.F,
+                   "parallelism": f"ep{world}", "exchange": "torch.distributed all_to_all_single (NCCL)"},
+        "parity": "every rank's output bit-identical to the single-GPU forward of the whole layer",
+        "single_gpu_forward_ms_per_step": round(single_ms, 5),
+        "clocks": clocks,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del ops, route, experts
+    d.close()
+
+
+def _free_port():
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
 def run_reference(args):
     """The C++ FP64 oracle timed on this host's cores as the reference arm
     (rank 0 only): each step is one oracle_sample of the workload (the same
@@ -534,8 +699,12 @@ def run_reference(args):
         return
     import gen
     from oracle import cpp
+    from oracle import moe
     wl, host, x_bits = gen.workload_inputs(args.workload)
     cpp.build()
+    # the groups the whole batch touches (routed experts chosen by the
+    # oracle's router, plus the shared expert), as in the other arm's config
+    touched = len(np.unique(moe.route_layer(x_bits, host).idx)) + wl.shape.S
     for i in range(args.warmup):
         oracle_sample(host, x_bits, first=i * ORACLE_TOKENS)
     tokens, secs = 0, 0.0
@@ -547,8 +716,7 @@ def run_reference(args):
     line = {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(secs / args.steps * 1e3, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": f"{wl.name}: {wl.note}", "T": wl.T, "hidden": wl.shape.H,
-                       "experts": f"{wl.shape.E}+{wl.shape.S}", "top_k": wl.shape.K, "ffn": wl.shape.F},
+            "config": workload_config(wl, world, touched),
             "cpu_baseline": {"value": round(value, 4), "unit": "tokens/s", "kind": "oracle", "cores": cpp.threads(),
                              "sample": f"C++ FP64 oracle, {n1} consecutive tokens of the workload per step "
                                        f"through the whole layer"},
@@ -563,6 +731,8 @@ def main():
         raise SystemExit("--warmup must be >= 3")
     if args.impl == "reference":
         run_reference(args)
+    elif args.ep:
+        run_ep(args)
     else:
         run_ours(args)
 

@@ -139,6 +139,10 @@ class MoeLayer:
         self.H, self.E, self.K, self.F = hidden, n_routed, top_k, ffn
         self.weights = weights
         self.S = n_shared
+        self.ld_h = hidden if ld_h is None else ld_h
+        self.ld_f = ffn if ld_f is None else ld_f
+        self.routed_scaling, self.n_group, self.topk_group = routed_scaling, n_group, topk_group
+        self.norm_topk, self.router_bias = bool(norm_topk), router_bias
         d = moe_layer_desc(hidden, n_routed, n_shared, top_k, ffn, ffn, 128, routed_scaling, int(bool(norm_topk)),
                            n_group, topk_group)
         w = moe_weights(_ptr(weights.w_gate), _ptr(weights.w_up), _ptr(weights.w_down), _ptr(weights.s_gate),

@@ -45,6 +45,28 @@ def plan_dispatch(offsets, E: int, ranks: int) -> np.ndarray:
     return np.diff(off[:E + 1]).reshape(ranks, local_experts(E, ranks))
 
 
+def rank_layers(layer, rank: int, ranks: int):
+    """The two handles rank `rank` of `ranks` runs, built from a whole layer's
+    device tensors: a routing-only handle over all E experts (the layer's
+    router and its settings) and an expert handle over the rank's block
+    [rank*El, (rank+1)*El) plus the shared expert, whose weights are copied
+    out of the layer's (index_select) so that the block is contiguous."""
+    import torch
+    from . import LayerWeights, MoeLayer
+    El = local_experts(layer.E, ranks)
+    w = layer.weights
+    route = MoeLayer(layer.H, layer.E, layer.K, layer.F, LayerWeights(None, None, None, None, None, None, w.router_w),
+                     routed_scaling=layer.routed_scaling, n_shared=layer.S, n_group=layer.n_group,
+                     topk_group=layer.topk_group, norm_topk=layer.norm_topk, router_bias=layer.router_bias)
+    e0 = rank * El
+    keep = torch.tensor(list(range(e0, e0 + El)) + ([layer.E] if layer.S else []), device=w.w_gate.device)
+    pick = {k: getattr(w, k).index_select(0, keep).contiguous()
+            for k in ("w_gate", "w_up", "w_down", "s_gate", "s_up", "s_down")}
+    experts = MoeLayer(layer.H, El, layer.K, layer.F, LayerWeights(router_w=w.router_w[e0:e0 + El].contiguous(), **pick),
+                       ld_h=layer.ld_h, ld_f=layer.ld_f, n_shared=layer.S)
+    return route, experts
+
+
 @dataclass
 class Dispatch:
     """Row counts of one forward on one rank."""

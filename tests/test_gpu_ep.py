@@ -65,23 +65,6 @@ class _RankView:
         return out
 
 
-def _rank_layers(dev, sh, ranks):
-    """(routing-only handle, expert handle) per rank; the expert handle holds
-    experts [r*El, (r+1)*El) and the shared expert, contiguous."""
-    El = sh.E // ranks
-    w = dev.weights
-    route = fx.MoeLayer(sh.H, sh.E, sh.K, sh.F, fx.LayerWeights(None, None, None, None, None, None, w.router_w),
-                        n_shared=sh.S)
-    out = []
-    for r in range(ranks):
-        keep = torch.tensor(list(range(r * El, (r + 1) * El)) + [sh.E], device="cuda")
-        lw = fx.LayerWeights(*(getattr(w, k).index_select(0, keep).contiguous()
-                               for k in ("w_gate", "w_up", "w_down", "s_gate", "s_up", "s_down")),
-                             router_w=w.router_w[r * El:(r + 1) * El].contiguous())
-        out.append((route, fx.MoeLayer(sh.H, El, sh.K, sh.F, lw, ld_h=sh.H, ld_f=sh.ld_f, n_shared=sh.S)))
-    return out
-
-
 def _run(name, ranks, T, layer=None, xs=None):
     wl, layer0, _ = gen.workload_inputs(name)
     layer = layer0 if layer is None else layer
@@ -96,7 +79,7 @@ def _run(name, ranks, T, layer=None, xs=None):
         ws = tu.workspace(dev, T)
         fx.moe_layer_forward(dev, xt, T, sh.H, o, sh.H, ws, ws.numel())
         refs.append(o)
-    layers = _rank_layers(dev, sh, ranks)
+    layers = [ep.rank_layers(dev, r, ranks) for r in range(ranks)]
     ex = LocalExchange(ranks)
     outs, errs = [None] * ranks, []
 
