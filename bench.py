@@ -59,7 +59,10 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--ep", action="store_true",
                    help="expert parallelism over the ranks instead of replicas: the routed experts split into "
-                        "equal blocks, one per rank, with the all-to-alls over torch.distributed (NCCL)")
+                        "equal blocks, one per rank")
+    p.add_argument("--ep-transport", choices=["peer", "nccl"], default="peer",
+                   help="peer: the library's dispatch/combine kernels over peer memory (CUDA IPC); nccl: "
+                        "all-to-alls of the rows over torch.distributed with the regroup kernels")
     return p.parse_args()
 
 
@@ -598,11 +601,13 @@ def run_ours(args):
 
 def run_ep(args):
     """--ep: one expert-parallel forward per step on every rank (its own T
-    tokens of the workload; fp8_expert_ffn_b200.ep.ep_forward): route and
-    permute against all E experts, exchange the row counts, dispatch the FP8
-    rows and scales, grouped GEMMs over the rank's E/P experts plus the shared
-    expert, return the rows, combine. The exchanges are torch.distributed
-    all-to-alls (NCCL; a one-rank group when run alone). Timed like the
+    tokens of the workload): route against all E experts, dispatch the FP8
+    rows to the ranks that own their experts, grouped GEMMs over the rank's
+    E/P experts plus the shared expert, return the rows, combine. With the
+    peer transport (default; ep.ep_forward_peer) the library's kernels store
+    and load the rows in the owners' memory and NCCL carries only the
+    offsets and two barriers; with nccl (ep.ep_forward) the rows cross in
+    torch.distributed all-to-alls. A one-rank group when run alone. Timed like the
     replica arm (CUDA events on the compute stream, barriers on both sides,
     max over ranks); the orchestration's two host reads of the counts are
     inside the timed region. Each rank's output is checked bit for bit
@@ -639,9 +644,20 @@ def run_ep(args):
     torch.cuda.synchronize()
     single_ms = d.max(a.elapsed_time(b)) / args.steps
     route, experts = ep.rank_layers(dev, rank, world)
-    ops, ex = ep.CudaOps(route, experts, world), ep.TorchExchange()
+    comm = None
+    if args.ep_transport == "peer":
+        comm = fx.EpComm(route, rank, world, ep.peer_capacity(T, sh.K, sh.S, world))
+        if world > 1:
+            handles = [None] * world
+            d.dist.all_gather_object(handles, comm.export())
+            comm.connect(handles)
+        ops, ex = ep.PeerOps(route, experts, comm, world), ep.TorchSync()
+        step = lambda: ep.ep_forward_peer(ops, ex, x, T)
+    else:
+        ops, ex = ep.CudaOps(route, experts, world), ep.TorchExchange()
+        step = lambda: ep.ep_forward(ops, ex, x, T)
     for _ in range(args.warmup):
-        out = ep.ep_forward(ops, ex, x, T)
+        out = step()
     torch.cuda.synchronize()
     visible = os.environ.get("CUDA_VISIBLE_DEVICES", "")
     sampler = ClockSampler(visible.split(",")[local] if visible else local)
@@ -650,7 +666,7 @@ def run_ep(args):
     sampler.start()
     a.record()
     for _ in range(args.steps):
-        out = ep.ep_forward(ops, ex, x, T)
+        out = step()
     b.record()
     torch.cuda.synchronize()
     clocks = sampler.stop()
@@ -671,13 +687,20 @@ def run_ep(args):
         "data": "synthetic",
         "config": {"workload": f"{wl.name}: {wl.note}", "T_per_rank": T, "hidden": sh.H,
                    "experts": f"{sh.E}+{sh.S}", "experts_per_rank": sh.E // world, "top_k": sh.K, "ffn": sh.F,
-                   "parallelism": f"ep{world}", "exchange": "torch.distributed all_to_all_single (NCCL)"},
+                   "parallelism": f"ep{world}",
+                   "exchange": ("dispatch/combine kernels over peer memory (CUDA IPC); NCCL all-gather of the "
+                                "offsets and two barriers" if comm else
+                                "torch.distributed all_to_all_single (NCCL) + regroup kernels")},
         "parity": "every rank's output bit-identical to the single-GPU forward of the whole layer",
         "single_gpu_forward_ms_per_step": round(single_ms, 5),
         "clocks": clocks,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
+    d.barrier()
+    torch.cuda.synchronize()
+    if comm is not None:
+        comm.close()          # every rank is past its last read of the peers' buffers
     del ops, route, experts
     d.close()
 

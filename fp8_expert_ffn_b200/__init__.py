@@ -21,7 +21,11 @@ ENTRY_POINTS = ("moe_status_string", "moe_layer_create", "moe_layer_destroy", "m
                 "moe_permute", "moe_expert_ffn", "moe_combine", "moe_layer_forward", "moe_get_device_status",
                 "moe_gate_up", "moe_down", "moe_test_grouped_gemm_f32", "moe_permute_noalloc",
                 "moe_kernels_per_forward", "moe_test_inject_stall", "moe_grouped_gate_up", "moe_grouped_down",
-                "moe_ep_pack_scales", "moe_ep_regroup", "moe_ep_unregroup")
+                "moe_ep_pack_scales", "moe_ep_regroup", "moe_ep_unregroup", "moe_ep_comm_create",
+                "moe_ep_comm_export", "moe_ep_comm_connect", "moe_ep_comm_connect_local", "moe_ep_comm_buffers",
+                "moe_ep_comm_destroy", "moe_ep_plan", "moe_ep_dispatch", "moe_ep_combine")
+
+MOE_EP_HANDLE_BYTES = 64        # include/moe.h
 
 MOE_NOALLOC_MAX_TOKENS = 4096   # include/moe.h
 
@@ -85,6 +89,15 @@ def lib(build_if_missing: bool = True):
     L.moe_ep_pack_scales.argtypes = [P, P, I, P, P]
     L.moe_ep_regroup.argtypes = [P, I, P, I, P, P, P, P, I, P, P, P, P]
     L.moe_ep_unregroup.argtypes = [P, I, P, I, P, I, P, P, P]
+    L.moe_ep_comm_create.argtypes = [P, I, I, I, ctypes.POINTER(P)]
+    L.moe_ep_comm_export.argtypes = [P, ctypes.c_char_p]
+    L.moe_ep_comm_connect.argtypes = [P, ctypes.c_char_p]
+    L.moe_ep_comm_connect_local.argtypes = [ctypes.POINTER(P), I]
+    L.moe_ep_comm_buffers.argtypes = [P, ctypes.POINTER(P), ctypes.POINTER(P), ctypes.POINTER(P)]
+    L.moe_ep_comm_destroy.argtypes = [P]
+    L.moe_ep_plan.argtypes = [P, P, I, P, P, S, P]
+    L.moe_ep_dispatch.argtypes = [P, P, P, I, I, P, P, P, P, P, S, P]
+    L.moe_ep_combine.argtypes = [P, P, P, P, P, P, I, P, I, P]
     for name in ENTRY_POINTS:
         if name not in ("moe_status_string", "moe_workspace_size"):
             getattr(L, name).restype = I
@@ -195,6 +208,67 @@ def moe_ep_regroup(layer, ranks, seg_counts, n_recv, recv_q, recv_s, own_q, own_
 def moe_ep_unregroup(layer, ranks, seg_counts, n_recv, y_g, T, y_send, y_own, stream=None):
     _check("moe_ep_unregroup", lib().moe_ep_unregroup(layer.handle, ranks, _ptr(seg_counts), n_recv, _ptr(y_g), T,
                                                       _ptr(y_send), _ptr(y_own), _stream(stream)))
+
+
+class EpComm:
+    """One rank's exchange buffers for the expert-parallel dispatch and
+    combine over peer memory (moe_ep_comm_*); `capacity` rows each."""
+
+    def __init__(self, layer: MoeLayer, rank: int, ranks: int, capacity: int):
+        h = ctypes.c_void_p()
+        _check("moe_ep_comm_create", lib().moe_ep_comm_create(layer.handle, rank, ranks, capacity, ctypes.byref(h)))
+        self.handle = h.value
+        self.rank, self.ranks, self.capacity = rank, ranks, capacity
+        q, s, y = ctypes.c_void_p(), ctypes.c_void_p(), ctypes.c_void_p()
+        _check("moe_ep_comm_buffers", lib().moe_ep_comm_buffers(self.handle, ctypes.byref(q), ctypes.byref(s),
+                                                                ctypes.byref(y)))
+        self.recv_q, self.recv_s, self.y = q.value, s.value, y.value   # device addresses
+
+    def export(self) -> bytes:
+        buf = ctypes.create_string_buffer(MOE_EP_HANDLE_BYTES)
+        _check("moe_ep_comm_export", lib().moe_ep_comm_export(self.handle, buf))
+        return buf.raw
+
+    def connect(self, handles):
+        """handles: every rank's export(), in rank order."""
+        blob = b"".join(handles)
+        if len(blob) != MOE_EP_HANDLE_BYTES * self.ranks:
+            raise ValueError("one handle per rank expected")
+        _check("moe_ep_comm_connect", lib().moe_ep_comm_connect(self.handle, blob))
+
+    @staticmethod
+    def connect_local(comms):
+        arr = (ctypes.c_void_p * len(comms))(*[c.handle for c in comms])
+        _check("moe_ep_comm_connect_local", lib().moe_ep_comm_connect_local(arr, len(comms)))
+
+    def close(self):
+        if getattr(self, "handle", None):
+            lib().moe_ep_comm_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def moe_ep_plan(layer, topk_idx, T, offsets, ws, ws_bytes, stream=None):
+    _check("moe_ep_plan", lib().moe_ep_plan(layer.handle, _ptr(topk_idx), T, _ptr(offsets), _ptr(ws), ws_bytes,
+                                            _stream(stream)))
+
+
+def moe_ep_dispatch(layer, comm: EpComm, x, T, ldx, topk_idx, all_offsets, inv_ep, group_offsets, ws, ws_bytes,
+                    stream=None):
+    _check("moe_ep_dispatch", lib().moe_ep_dispatch(layer.handle, comm.handle, _ptr(x), T, ldx, _ptr(topk_idx),
+                                                    _ptr(all_offsets), _ptr(inv_ep), _ptr(group_offsets), _ptr(ws),
+                                                    ws_bytes, _stream(stream)))
+
+
+def moe_ep_combine(layer, comm: EpComm, topk_idx, inv_ep, topk_w, group_offsets, T, out, ldo, stream=None):
+    _check("moe_ep_combine", lib().moe_ep_combine(layer.handle, comm.handle, _ptr(topk_idx), _ptr(inv_ep),
+                                                  _ptr(topk_w), _ptr(group_offsets), T, _ptr(out), ldo,
+                                                  _stream(stream)))
 
 
 def moe_test_inject_stall(layer: MoeLayer, wait_limit_ns: int):

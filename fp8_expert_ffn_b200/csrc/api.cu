@@ -446,5 +446,196 @@ moe_status moe_test_grouped_gemm_f32(moe_layer_t L, int which, const uint8_t* a,
   return from_cuda(launch_test_gemm_f32(L, which, a, as, offsets, T, out, static_cast<cudaStream_t>(stream)));
 }
 
+// ---------------------------------------------------------------------------
+// Expert parallelism over peer memory
+
+static_assert(sizeof(cudaIpcMemHandle_t) == MOE_EP_HANDLE_BYTES, "IPC handle size");
+
+static moe_status ep_upload_tables(moe_ep_comm_s* c, const uint64_t* q, const uint64_t* s, const uint64_t* y) {
+  uint64_t tab[3 * kEpMaxRanks];
+  for (int i = 0; i < c->ranks; ++i) {
+    tab[i] = q[i];
+    tab[c->ranks + i] = s[i];
+    tab[2 * c->ranks + i] = y[i];
+  }
+  return from_cuda(cudaMemcpy(c->d_peer_q, tab, sizeof(uint64_t) * 3 * c->ranks, cudaMemcpyHostToDevice));
+}
+
+static void ep_own(const moe_ep_comm_s* c, const char* base, uint64_t* q, uint64_t* s, uint64_t* y) {
+  *q = reinterpret_cast<uint64_t>(base);
+  *s = reinterpret_cast<uint64_t>(base + c->off_s);
+  *y = reinterpret_cast<uint64_t>(base + c->off_y);
+}
+
+moe_status moe_ep_comm_create(moe_layer_t L, int rank, int ranks, int capacity, moe_ep_comm_t* out) {
+  if (!out) return MOE_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (!L || ranks < 1 || ranks > kEpMaxRanks || rank < 0 || rank >= ranks || capacity < 1 || capacity > kMaxT)
+    return MOE_ERR_INVALID_ARG;
+  moe_ep_comm_s* c = new (std::nothrow) moe_ep_comm_s();
+  if (!c) return MOE_ERR_CUDA;
+  if (cudaGetDevice(&c->device) != cudaSuccess) {
+    delete c;
+    return MOE_ERR_CUDA;
+  }
+  c->rank = rank;
+  c->ranks = ranks;
+  c->cap = capacity;
+  c->H = L->H;
+  c->HB = L->HB;
+  c->off_s = align_up(size_t(capacity) * L->H, 256);
+  c->off_y = c->off_s + align_up(sizeof(float) * L->HB * size_t(capacity), 256);
+  c->bytes = c->off_y + sizeof(uint16_t) * size_t(capacity) * L->H;
+  void* tab = nullptr;
+  if (cudaMalloc(&c->base, c->bytes) != cudaSuccess || cudaMalloc(&tab, sizeof(uint64_t) * 3 * ranks) != cudaSuccess) {
+    if (c->base) cudaFree(c->base);
+    delete c;
+    return MOE_ERR_CUDA;
+  }
+  c->d_peer_q = static_cast<uint64_t*>(tab);
+  c->d_peer_s = c->d_peer_q + ranks;
+  c->d_peer_y = c->d_peer_s + ranks;
+  uint64_t q[kEpMaxRanks] = {}, sc[kEpMaxRanks] = {}, y[kEpMaxRanks] = {};
+  ep_own(c, static_cast<const char*>(c->base), &q[rank], &sc[rank], &y[rank]);
+  moe_status st = ep_upload_tables(c, q, sc, y);
+  if (st != MOE_OK) {
+    cudaFree(tab);
+    cudaFree(c->base);
+    delete c;
+    return st;
+  }
+  c->connected = ranks == 1;
+  *out = c;
+  return MOE_OK;
+}
+
+moe_status moe_ep_comm_export(moe_ep_comm_t c, unsigned char handle[MOE_EP_HANDLE_BYTES]) {
+  if (!c || !handle) return MOE_ERR_INVALID_ARG;
+  cudaIpcMemHandle_t h;
+  if (cudaIpcGetMemHandle(&h, c->base) != cudaSuccess) return MOE_ERR_CUDA;
+  std::memcpy(handle, &h, sizeof(h));
+  return MOE_OK;
+}
+
+static void ep_close_opened(moe_ep_comm_s* c) {
+  for (int i = 0; i < kEpMaxRanks; ++i)
+    if (c->opened[i]) {
+      cudaIpcCloseMemHandle(c->opened[i]);
+      c->opened[i] = nullptr;
+    }
+}
+
+moe_status moe_ep_comm_connect(moe_ep_comm_t c, const unsigned char* handles) {
+  if (!c || !handles || c->connected) return MOE_ERR_INVALID_ARG;
+  uint64_t q[kEpMaxRanks] = {}, sc[kEpMaxRanks] = {}, y[kEpMaxRanks] = {};
+  for (int i = 0; i < c->ranks; ++i) {
+    if (i == c->rank) {
+      ep_own(c, static_cast<const char*>(c->base), &q[i], &sc[i], &y[i]);
+      continue;
+    }
+    cudaIpcMemHandle_t h;
+    std::memcpy(&h, handles + size_t(i) * MOE_EP_HANDLE_BYTES, sizeof(h));
+    void* p = nullptr;
+    if (cudaIpcOpenMemHandle(&p, h, cudaIpcMemLazyEnablePeerAccess) != cudaSuccess) {
+      ep_close_opened(c);
+      return MOE_ERR_CUDA;
+    }
+    c->opened[i] = p;
+    ep_own(c, static_cast<const char*>(p), &q[i], &sc[i], &y[i]);
+  }
+  moe_status st = ep_upload_tables(c, q, sc, y);
+  if (st != MOE_OK) {
+    ep_close_opened(c);
+    return st;
+  }
+  c->connected = true;
+  return MOE_OK;
+}
+
+moe_status moe_ep_comm_connect_local(moe_ep_comm_t* comms, int ranks) {
+  if (!comms || ranks < 1 || ranks > kEpMaxRanks) return MOE_ERR_INVALID_ARG;
+  for (int i = 0; i < ranks; ++i) {
+    const moe_ep_comm_s* c = comms[i];
+    if (!c || c->rank != i || c->ranks != ranks || c->cap != comms[0]->cap || c->H != comms[0]->H ||
+        c->device != comms[0]->device || c->connected != (ranks == 1))
+      return MOE_ERR_INVALID_ARG;
+  }
+  uint64_t q[kEpMaxRanks] = {}, sc[kEpMaxRanks] = {}, y[kEpMaxRanks] = {};
+  for (int i = 0; i < ranks; ++i) ep_own(comms[i], static_cast<const char*>(comms[i]->base), &q[i], &sc[i], &y[i]);
+  for (int i = 0; i < ranks; ++i) {
+    moe_status st = ep_upload_tables(comms[i], q, sc, y);
+    if (st != MOE_OK) return st;
+    comms[i]->connected = true;
+  }
+  return MOE_OK;
+}
+
+moe_status moe_ep_comm_buffers(moe_ep_comm_t c, uint8_t** recv_q, float** recv_s, uint16_t** y) {
+  if (!c) return MOE_ERR_INVALID_ARG;
+  char* b = static_cast<char*>(c->base);
+  if (recv_q) *recv_q = reinterpret_cast<uint8_t*>(b);
+  if (recv_s) *recv_s = reinterpret_cast<float*>(b + c->off_s);
+  if (y) *y = reinterpret_cast<uint16_t*>(b + c->off_y);
+  return MOE_OK;
+}
+
+moe_status moe_ep_comm_destroy(moe_ep_comm_t c) {
+  if (!c) return MOE_OK;
+  moe_status st = from_cuda(cudaDeviceSynchronize());
+  ep_close_opened(c);
+  if (cudaFree(c->d_peer_q) != cudaSuccess) st = MOE_ERR_CUDA;
+  if (cudaFree(c->base) != cudaSuccess) st = MOE_ERR_CUDA;
+  delete c;
+  return st;
+}
+
+moe_status moe_ep_plan(moe_layer_t L, const int32_t* idx, int T, int32_t* offsets, void* ws, size_t ws_bytes,
+                       void* stream) {
+  if (!L || T < 0 || T > kMaxT || !offsets) return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (T == 0) return from_cuda(cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (L->E + 2), st));
+  if (!idx) return MOE_ERR_INVALID_ARG;
+  moe_status s;
+  if ((s = check_ws(L, T, ws, ws_bytes)) != MOE_OK) return s;
+  return from_cuda(launch_ep_plan(L, idx, T, offsets, carve(L, T, ws), st));
+}
+
+static moe_status ep_check(const moe_layer_s* L, const moe_ep_comm_s* c, int T) {
+  if (!L || !c || T < 0 || T > kMaxT) return MOE_ERR_INVALID_ARG;
+  if (!c->connected || L->E % c->ranks != 0 || c->H != L->H) return MOE_ERR_INVALID_ARG;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+  if (dev != c->device) return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+
+moe_status moe_ep_dispatch(moe_layer_t L, moe_ep_comm_t c, const uint16_t* x, int T, int ldx, const int32_t* idx,
+                           const int32_t* all_offsets, int32_t* inv_ep, int32_t* group_offsets, void* ws,
+                           size_t ws_bytes, void* stream) {
+  moe_status s;
+  if ((s = ep_check(L, c, T)) != MOE_OK) return s;
+  if (!all_offsets || !group_offsets) return MOE_ERR_INVALID_ARG;
+  Scratch sc = {};
+  if (T > 0) {
+    if (!idx || !inv_ep) return MOE_ERR_INVALID_ARG;
+    if ((s = check_x(L, x, ldx)) != MOE_OK) return s;
+    if ((s = check_ws(L, T, ws, ws_bytes)) != MOE_OK) return s;
+    sc = carve(L, T, ws);
+  }
+  return from_cuda(launch_ep_dispatch(L, c, x, T, ldx, idx, all_offsets, inv_ep, group_offsets, sc,
+                                      static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_ep_combine(moe_layer_t L, moe_ep_comm_t c, const int32_t* idx, const int32_t* inv_ep, const float* w,
+                          const int32_t* group_offsets, int T, uint16_t* out, int ldo, void* stream) {
+  moe_status s;
+  if ((s = ep_check(L, c, T)) != MOE_OK) return s;
+  if (T == 0) return MOE_OK;
+  if (!idx || !inv_ep || !w || !group_offsets || !out || ldo < L->H) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(out) || (size_t(ldo) * 2) % 16 != 0) return MOE_ERR_MISALIGNED;
+  return from_cuda(launch_ep_combine(L, c, idx, inv_ep, w, group_offsets, T, out, ldo,
+                                     static_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"
 #pragma GCC visibility pop

@@ -16,36 +16,67 @@ namespace {
 
 constexpr int CB_THREADS = 128;
 
+struct CombineArgs {
+  const uint16_t* y;       // local: [rows][H], routed rows then the shared rows
+  const int32_t* inv;      // [T][K] row of (token, slot), -1 if none
+  const float* w;          // [T][K]
+  int T, K, S, H;
+  uint16_t* out;
+  int ldo;
+  // expert parallel: slot k's row is in the y buffer of its expert's owner
+  const int32_t* idx;      // [T][K]
+  const uint64_t* peer_y;  // [ranks] rows [cap][H] bf16
+  const int32_t* goff;     // [El+2] this rank's group offsets: its shared rows start at goff[El]
+  int rank, El;
+};
+
 // CTA (token, chunk of CB_THREADS*8 channels); each thread owns one
-// 8-channel (16-byte) piece and loads its K+1 rows at once.
-__global__ void __launch_bounds__(CB_THREADS) combine_kernel(const uint16_t* __restrict__ y,
-                                                             const int32_t* __restrict__ inv,
-                                                             const float* __restrict__ w, int T, int K, int S, int H,
-                                                             uint16_t* __restrict__ out, int ldo) {
+// 8-channel (16-byte) piece and loads its K+1 rows at once. With EP the rows
+// are read from their owners' buffers (a peer's memory over NVLink, plain
+// 16-byte loads).
+template <bool EP>
+__global__ void __launch_bounds__(CB_THREADS) combine_kernel(const CombineArgs a) {
   pdl_wait();
   pdl_launch_dependents();
-  const int t = blockIdx.x;
-  __shared__ int s_row[9];
+  const int t = blockIdx.x, K = a.K, H = a.H;
+  __shared__ const uint16_t* s_src[9];
   __shared__ float s_w[9];
   if (threadIdx.x < K) {
-    s_row[threadIdx.x] = inv[size_t(t) * K + threadIdx.x];
-    s_w[threadIdx.x] = w[size_t(t) * K + threadIdx.x];
+    const int r = a.inv[size_t(t) * K + threadIdx.x];
+    const uint16_t* src = nullptr;
+    if (r >= 0) {
+      const uint16_t* ybase = EP ? reinterpret_cast<const uint16_t*>(a.peer_y[a.idx[size_t(t) * K + threadIdx.x] / a.El])
+                                 : a.y;
+      src = ybase + size_t(r) * H;
+    }
+    s_src[threadIdx.x] = src;
+    s_w[threadIdx.x] = a.w[size_t(t) * K + threadIdx.x];
+  } else if (threadIdx.x == K) {
+    const uint16_t* src = nullptr;
+    if (a.S && !EP) {
+      src = a.y + (size_t(a.T) * K + t) * H;
+    } else if (a.S) {
+      // this rank's shared rows are [goff[El], goff[El+1]) of its own buffer
+      // (both 0 after an overflow: then nothing is read)
+      const int row = a.goff[a.El] + t;
+      if (row < a.goff[a.El + 1]) src = reinterpret_cast<const uint16_t*>(a.peer_y[a.rank]) + size_t(row) * H;
+    }
+    s_src[K] = src;
   }
   __syncthreads();
-  const size_t shared_row = size_t(T) * K + t;
   const int c = (blockIdx.y * CB_THREADS + threadIdx.x) * 8;
   if (c < H) {
     uint4 raws[8];
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
-      const int r = k < K ? s_row[k] : -1;
-      raws[k] = r >= 0 ? *reinterpret_cast<const uint4*>(y + size_t(r) * H + c) : make_uint4(0, 0, 0, 0);
+      const uint16_t* src = k < K ? s_src[k] : nullptr;
+      raws[k] = src ? *reinterpret_cast<const uint4*>(src + c) : make_uint4(0, 0, 0, 0);
     }
-    const uint4 raw_shared = S ? *reinterpret_cast<const uint4*>(y + shared_row * H + c) : make_uint4(0, 0, 0, 0);
+    const uint4 raw_shared = s_src[K] ? *reinterpret_cast<const uint4*>(s_src[K] + c) : make_uint4(0, 0, 0, 0);
     float acc[8] = {};
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
-      if (k >= K || s_row[k] < 0) continue;
+      if (k >= K || !s_src[k]) continue;
       const float wk = s_w[k];
       const uint4 raw = raws[k];
       const uint32_t p[4] = {raw.x, raw.y, raw.z, raw.w};
@@ -59,11 +90,11 @@ __global__ void __launch_bounds__(CB_THREADS) combine_kernel(const uint16_t* __r
     uint32_t o[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const float a = acc[2 * j] + bf16_bits_to_f32(uint16_t(p[j] & 0xFFFFu));
-      const float b = acc[2 * j + 1] + bf16_bits_to_f32(uint16_t(p[j] >> 16));
-      o[j] = uint32_t(f32_to_bf16_bits(a)) | (uint32_t(f32_to_bf16_bits(b)) << 16);
+      const float a0 = acc[2 * j] + bf16_bits_to_f32(uint16_t(p[j] & 0xFFFFu));
+      const float a1 = acc[2 * j + 1] + bf16_bits_to_f32(uint16_t(p[j] >> 16));
+      o[j] = uint32_t(f32_to_bf16_bits(a0)) | (uint32_t(f32_to_bf16_bits(a1)) << 16);
     }
-    *reinterpret_cast<uint4*>(out + size_t(t) * ldo + c) = make_uint4(o[0], o[1], o[2], o[3]);
+    *reinterpret_cast<uint4*>(a.out + size_t(t) * a.ldo + c) = make_uint4(o[0], o[1], o[2], o[3]);
   }
 }
 
@@ -71,8 +102,38 @@ __global__ void __launch_bounds__(CB_THREADS) combine_kernel(const uint16_t* __r
 
 cudaError_t launch_combine(const moe_layer_s* L, const uint16_t* y, const int32_t* inv, const float* w, int T,
                            uint16_t* out, int ldo, cudaStream_t st) {
+  CombineArgs a = {};
+  a.y = y;
+  a.inv = inv;
+  a.w = w;
+  a.T = T;
+  a.K = L->K;
+  a.S = L->S;
+  a.H = L->H;
+  a.out = out;
+  a.ldo = ldo;
   dim3 grid(T, (L->H + CB_THREADS * 8 - 1) / (CB_THREADS * 8));
-  return launch_pdl(combine_kernel, grid, dim3(CB_THREADS), 0, st, y, inv, w, T, L->K, L->S, L->H, out, ldo);
+  return launch_pdl(combine_kernel<false>, grid, dim3(CB_THREADS), 0, st, a);
+}
+
+cudaError_t launch_ep_combine(const moe_layer_s* L, const moe_ep_comm_s* c, const int32_t* idx, const int32_t* inv_ep,
+                              const float* w, const int32_t* goff, int T, uint16_t* out, int ldo, cudaStream_t st) {
+  CombineArgs a = {};
+  a.inv = inv_ep;
+  a.w = w;
+  a.T = T;
+  a.K = L->K;
+  a.S = L->S;
+  a.H = L->H;
+  a.out = out;
+  a.ldo = ldo;
+  a.idx = idx;
+  a.peer_y = c->d_peer_y;
+  a.goff = goff;
+  a.rank = c->rank;
+  a.El = L->E / c->ranks;
+  dim3 grid(T, (L->H + CB_THREADS * 8 - 1) / (CB_THREADS * 8));
+  return launch_pdl(combine_kernel<true>, grid, dim3(CB_THREADS), 0, st, a);
 }
 
 }  // namespace moe

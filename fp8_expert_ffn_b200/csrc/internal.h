@@ -35,6 +35,26 @@ struct moe_layer_s {
   mutable unsigned long long test_stall_ns;
 };
 
+// Exchange buffers of one rank for the expert-parallel dispatch and combine
+// over peer memory (ep.cu): one device allocation holding this rank's
+// receive buffers and output rows, and device tables of every rank's
+// buffers (a peer's through a CUDA IPC mapping, or a buffer of this process
+// when the ranks are emulated on one GPU).
+struct moe_ep_comm_s {
+  int device;
+  int rank, ranks;
+  int cap;             // rows of each buffer
+  int H, HB;
+  void* base;          // this rank's allocation
+  size_t bytes;
+  size_t off_s, off_y; // byte offsets of the scales and of y in an allocation
+  uint64_t* d_peer_q;  // [ranks] device table: codes [cap][H] u8
+  uint64_t* d_peer_s;  // [ranks] scales [HB][cap] f32
+  uint64_t* d_peer_y;  // [ranks] rows [cap][H] bf16
+  void* opened[64];    // IPC mappings to close (by rank), null if none
+  bool connected;
+};
+
 namespace moe {
 
 // Workspace carving shared by every entry point.
@@ -87,6 +107,18 @@ cudaError_t launch_gate_up(const moe_layer_s* L, const uint8_t* xq, const float*
                            uint8_t* h, float* hs, cudaStream_t st);
 cudaError_t launch_down(const moe_layer_s* L, const uint8_t* h, const float* hs, const int32_t* offsets, int rows,
                         uint16_t* y, cudaStream_t st);
+// Expert parallelism over peer memory: the permutation plan alone (bitmap,
+// prefixes, offsets), the dispatch (quantise and write each routed row into
+// its owner's receive buffer, the shared rows into this rank's; the owner's
+// group offsets) and the combine (read the rows back from the owners' y).
+constexpr int kEpMaxRanks = 64;
+cudaError_t launch_ep_plan(const moe_layer_s* L, const int32_t* idx, int T, int32_t* offsets, const Scratch& s,
+                           cudaStream_t st);
+cudaError_t launch_ep_dispatch(const moe_layer_s* L, const moe_ep_comm_s* c, const uint16_t* x, int T, int ldx,
+                               const int32_t* idx, const int32_t* all_off, int32_t* inv_ep, int32_t* goff,
+                               const Scratch& s, cudaStream_t st);
+cudaError_t launch_ep_combine(const moe_layer_s* L, const moe_ep_comm_s* c, const int32_t* idx, const int32_t* inv_ep,
+                              const float* w, const int32_t* goff, int T, uint16_t* out, int ldo, cudaStream_t st);
 // Expert parallelism (ep.cu): at most kEpMaxSegments = ranks x local experts.
 constexpr int kEpMaxSegments = 2048;
 cudaError_t launch_ep_pack_scales(const moe_layer_s* L, const float* xs, int T, float* out, cudaStream_t st);

@@ -186,29 +186,125 @@ __global__ void __launch_bounds__(kPlanSmallThreads) permute_plan_small_kernel(
 }
 
 constexpr int GATHER_GROUPS = 16;   // 128-channel groups per warp (4 steps of 4 groups)
+constexpr int GATHER_THREADS = 256;
+
+enum GatherMode { GATHER_LOCAL = 0, GATHER_EP = 1 };
+
+struct GatherArgs {
+  const uint16_t* x;
+  int T, ldx, H;
+  const int32_t* idx;
+  int K, E, W, S;
+  const uint32_t* bitmap;
+  const uint32_t* wprefix;
+  // GATHER_LOCAL: this GPU's grouped layout
+  const int32_t* offsets;
+  int rows;
+  int32_t* perm;
+  int32_t* inv;
+  uint8_t* xq;
+  float* xs;
+  // GATHER_EP: the rows' owners' receive buffers
+  const int32_t* all_off;   // [ranks][E+2] every rank's local offsets
+  int rank, ranks, El, cap;
+  const uint64_t* peer_q;   // [ranks] code buffers [cap][H]
+  const uint64_t* peer_s;   // [ranks] scale buffers [HB][cap]
+  int32_t* inv_ep;          // [T][K] row in the owner's buffer, -1 if none
+  int32_t* goff;            // [El+2] this rank's group offsets as an owner
+  uint32_t* status;
+};
+
+// Expert-parallel layout, computed by every CTA from the ranks' offsets.
+// Owner p holds local expert e's rows from sender 0, 1, ..., ranks-1 in turn,
+// experts in order, then its own shared rows. For a global expert g the rows
+// this rank sends start at base[g] in g's owner's buffer.
+__device__ void ep_layout(const GatherArgs& a, int* s_base, int* s_excl, int* s_wsum, int* s_nr, int* s_over) {
+  const int i = threadIdx.x, lane = i & 31, wid = i >> 5;
+  const int E = a.E, stride = E + 2;
+  int tot = 0, pre = 0;
+  bool bad = false;
+  if (i < E) {
+    for (int s = 0; s < a.ranks; ++s) {
+      const int c = a.all_off[s * stride + i + 1] - a.all_off[s * stride + i];
+      bad |= c < 0;
+      tot += c;
+      if (s < a.rank) pre += c;
+    }
+  }
+  int incl = tot;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int o = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+    if (lane >= off) incl += o;
+  }
+  if (lane == 31) s_wsum[wid] = incl;
+  if (i == 0) *s_over = 0;
+  __syncthreads();
+  if (bad) {   // offsets not ascending: nothing is dispatched
+    atomicOr(s_over, 1);
+    set_status(a.status, STATUS_BAD_PLAN);
+  }
+  int before = 0;
+  for (int j = 0; j < wid; ++j) before += s_wsum[j];
+  if (i < E) s_excl[i] = before + incl - tot;
+  if (i == E - 1) s_excl[E] = before + incl;
+  __syncthreads();
+  if (i < E) s_base[i] = s_excl[i] - s_excl[(i / a.El) * a.El] + pre;
+  if (i < a.ranks) {   // owner i's routed rows plus its own shared rows must fit its buffer
+    const int n = s_excl[(i + 1) * a.El] - s_excl[i * a.El];
+    const int sh = a.all_off[i * stride + E + 1] - a.all_off[i * stride + E];
+    if (sh < 0 || n + sh > a.cap) atomicOr(s_over, 1);
+  }
+  if (i == 0) *s_nr = s_excl[(a.rank + 1) * a.El] - s_excl[a.rank * a.El];
+  __syncthreads();
+  if (blockIdx.x == 0) {
+    const bool over = *s_over != 0;
+    const int e0 = a.rank * a.El;
+    for (int e = i; e < a.El; e += blockDim.x) a.goff[e] = over ? 0 : s_excl[e0 + e] - s_excl[e0];
+    if (i == 0) {
+      const int sh = a.all_off[a.rank * stride + E + 1] - a.all_off[a.rank * stride + E];
+      a.goff[a.El] = over ? 0 : *s_nr;
+      a.goff[a.El + 1] = over ? 0 : *s_nr + sh;
+      if (over) set_status(a.status, STATUS_EP_OVERFLOW);
+    }
+  }
+}
 
 // One warp per (token, chunk of GATHER_GROUPS groups). In each step the warp
 // covers 4 consecutive groups: lanes 8j..8j+7 hold group j of the step, 16
 // channels per lane (one 32-byte load of x, one 16-byte store of codes per
 // row), so a row's store instruction writes 512 contiguous bytes. Lane k < K
-// owns slot k's row, lane K the shared row; the chunk-0 warp writes inv and
-// perm.
-__global__ void __launch_bounds__(256) permute_gather_kernel(
-    const uint16_t* __restrict__ x, int T, int ldx, int H, const int32_t* __restrict__ idx, int K, int E, int W,
-    const uint32_t* __restrict__ bitmap, const uint32_t* __restrict__ wprefix, const int32_t* __restrict__ offsets,
-    int S, int rows, int32_t* __restrict__ perm, int32_t* __restrict__ inv, uint8_t* __restrict__ xq,
-    float* __restrict__ xs) {
+// owns slot k's row, lane K the shared row; the chunk-0 warp writes the row
+// maps. GATHER_LOCAL writes the rows of this GPU's grouped layout (and inv,
+// perm); GATHER_EP writes each routed row into its expert's owner's receive
+// buffer (a peer's memory over NVLink; every store is a plain 16- or 4-byte
+// store, no bulk or tensor copy) and the shared row into this rank's own.
+template <int MODE>
+__global__ void __launch_bounds__(GATHER_THREADS) gather_rows_kernel(const GatherArgs a) {
   pdl_wait();
   pdl_launch_dependents();
+  __shared__ int s_base[MODE == GATHER_EP ? 256 : 1];
+  __shared__ int s_excl[MODE == GATHER_EP ? 257 : 1];
+  __shared__ int s_wsum[GATHER_THREADS / 32];
+  __shared__ int s_nr, s_over;
+  __shared__ uint64_t s_peer[MODE == GATHER_EP ? 2 * kEpMaxRanks : 1];   // codes, then scales
+  if (MODE == GATHER_EP) {
+    for (int i = threadIdx.x; i < a.ranks; i += GATHER_THREADS) {
+      s_peer[i] = a.peer_q[i];
+      s_peer[kEpMaxRanks + i] = a.peer_s[i];
+    }
+    ep_layout(a, s_base, s_excl, s_wsum, &s_nr, &s_over);   // ends with a CTA barrier
+  }
+  const int T = a.T, K = a.K, E = a.E, W = a.W, H = a.H;
   const int lane = threadIdx.x & 31;
   const int gl = lane & 7, gs = lane >> 3;   // lane within its group, group slot of the step
   const int HB = H / 128;
   const int nchunk = (HB + GATHER_GROUPS - 1) / GATHER_GROUPS;
-  const int wid = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int wid = blockIdx.x * (GATHER_THREADS / 32) + (threadIdx.x >> 5);
   const int t = wid / nchunk, chunk = wid - t * nchunk;
   if (t >= T) return;
   const int g0 = chunk * GATHER_GROUPS;
-  const uint16_t* xr = x + size_t(t) * ldx;
+  const uint16_t* xr = a.x + size_t(t) * a.ldx;
   // issue the x loads of the whole chunk before anything waits on memory
   uint4 raw[4][2];
 #pragma unroll
@@ -223,24 +319,54 @@ __global__ void __launch_bounds__(256) permute_gather_kernel(
     }
   }
 
+  // this lane's row; with EP the row in its owner's buffer, packed with the
+  // owner's index (rows < 2^24, owners < 64)
   int my_row = -1;
+  const bool over = MODE == GATHER_EP && s_over != 0;
   if (lane < K) {
-    const int e = idx[size_t(t) * K + lane];
-    bool ok = (e >= 0 && e < E);
-    for (int j = 0; j < lane && ok; ++j) ok = (idx[size_t(t) * K + j] != e);  // first slot of a repeat wins
+    const int e = a.idx[size_t(t) * K + lane];
+    bool ok = (e >= 0 && e < E) && !over;
+    for (int j = 0; j < lane && ok; ++j) ok = (a.idx[size_t(t) * K + j] != e);  // first slot of a repeat wins
+    int row = -1;
     if (ok) {
-      const uint32_t word = bitmap[size_t(e) * W + (t >> 5)];
-      my_row = offsets[e] + int(wprefix[size_t(e) * W + (t >> 5)]) + __popc(word & ((1u << (t & 31)) - 1u));
+      const uint32_t word = a.bitmap[size_t(e) * W + (t >> 5)];
+      const int within = int(a.wprefix[size_t(e) * W + (t >> 5)]) + __popc(word & ((1u << (t & 31)) - 1u));
+      if (MODE == GATHER_LOCAL) {
+        row = a.offsets[e] + within;
+        my_row = row;
+      } else if (within < a.all_off[a.rank * (E + 2) + e + 1] - a.all_off[a.rank * (E + 2) + e]) {
+        // (a row beyond this rank's own count in all_offsets is not this
+        // rank's plan: skipped and flagged, so no store leaves its range)
+        row = s_base[e] + within;
+        my_row = row | ((e / a.El) << 24);
+      } else {
+        set_status(a.status, STATUS_BAD_PLAN);
+      }
     }
-    if (chunk == 0) inv[size_t(t) * K + lane] = my_row;
-  } else if (lane == K && S) {
-    my_row = offsets[E] + t;
+    if (chunk == 0) {
+      if (MODE == GATHER_LOCAL) {
+        a.inv[size_t(t) * K + lane] = row;
+        if (row >= 0) a.perm[row] = t;
+      } else {
+        a.inv_ep[size_t(t) * K + lane] = row;
+      }
+    }
+  } else if (lane == K && a.S) {
+    if (MODE == GATHER_LOCAL) {
+      my_row = a.offsets[E] + t;
+      if (chunk == 0) a.perm[my_row] = t;
+    } else if (!over) {
+      if (t < a.all_off[a.rank * (E + 2) + E + 1] - a.all_off[a.rank * (E + 2) + E])
+        my_row = (s_nr + t) | (a.rank << 24);
+      else
+        set_status(a.status, STATUS_BAD_PLAN);
+    }
   }
-  if (chunk == 0 && my_row >= 0) perm[my_row] = t;
-  // rows of this token, known to every lane
+  // the token's rows, known to every lane
   int rowv[9];
 #pragma unroll
   for (int j = 0; j < 9; ++j) rowv[j] = __shfl_sync(0xFFFFFFFFu, my_row, j);
+  const size_t sstride = MODE == GATHER_LOCAL ? size_t(a.rows) : size_t(a.cap);
 
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
@@ -277,10 +403,24 @@ __global__ void __launch_bounds__(256) permute_gather_kernel(
       if (j > K) break;
       const int r = rowv[j];
       if (r < 0) continue;
-      *reinterpret_cast<uint4*>(xq + size_t(r) * H + g * 128 + gl * 16) = q;
-      if (gl == (j & 7)) xs[size_t(g) * rows + r] = s;
+      uint8_t* qb;
+      float* sb;
+      if (MODE == GATHER_LOCAL) {
+        qb = a.xq + size_t(r) * H;
+        sb = a.xs + r;
+      } else {
+        const int p = r >> 24, rr = r & 0xFFFFFF;
+        qb = reinterpret_cast<uint8_t*>(s_peer[p]) + size_t(rr) * H;
+        sb = reinterpret_cast<float*>(s_peer[kEpMaxRanks + p]) + rr;
+      }
+      *reinterpret_cast<uint4*>(qb + g * 128 + gl * 16) = q;
+      if (gl == (j & 7)) sb[size_t(g) * sstride] = s;
     }
   }
+  // the rows written into peers' memory are complete, system-wide, before
+  // this thread finishes (the owners read them after a barrier that follows
+  // this kernel)
+  if (MODE == GATHER_EP) __threadfence_system();
 }
 
 }  // namespace
@@ -289,35 +429,98 @@ int permute_kernels(const moe_layer_s* L, int T) {
   return size_t(L->E) * ((T + 31) / 32) <= size_t(kPlanSmallWords) ? 2 : 4;
 }
 
+// The plan of the permutation: the token bitmap and its per-word prefixes in
+// the scratch, the counts, and offsets[E+2].
+static cudaError_t launch_plan(const moe_layer_s* L, const int32_t* idx, int T, int32_t* offsets, const Scratch& s,
+                        cudaStream_t st) {
+  const int K = L->K, E = L->E, W = (T + 31) / 32;
+  const int S = L->S;
+  const size_t nwords = size_t(E) * W;
+  cudaError_t e;
+  if (permute_kernels(L, T) == 2)
+    return launch_pdl(permute_plan_small_kernel, dim3(1), dim3(kPlanSmallThreads), 0, st, idx, T, K, E, W, S,
+                      s.bitmap, s.wprefix, s.counts, offsets, L->status);
+  uint32_t* done = reinterpret_cast<uint32_t*>(s.counts + E);
+  e = launch_pdl(permute_clear_kernel, dim3(unsigned((nwords + 1023) / 1024)), dim3(256), 0, st, s.bitmap, nwords,
+                 done);
+  if (e != cudaSuccess) return e;
+  e = launch_pdl(permute_bitmap_kernel, dim3((T * K + 255) / 256), dim3(256), 0, st, idx, T, K, E, W, s.bitmap,
+                 L->status);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(permute_count_kernel, dim3(E), dim3(256), 0, st, static_cast<const uint32_t*>(s.bitmap), W,
+                    s.wprefix, s.counts, E, T, S, offsets, done);
+}
+
 cudaError_t launch_permute(const moe_layer_s* L, const uint16_t* x, int T, int ldx, const int32_t* idx,
                            int32_t* offsets, int32_t* perm, int32_t* inv, uint8_t* xq, float* xs,
                            const Scratch& s, cudaStream_t st) {
   const int K = L->K, E = L->E, W = (T + 31) / 32;
   const int S = L->S;
   const int rows = T * (K + S);
-  const size_t nwords = size_t(E) * W;
-  cudaError_t e;
-  if (permute_kernels(L, T) == 2) {
-    e = launch_pdl(permute_plan_small_kernel, dim3(1), dim3(kPlanSmallThreads), 0, st, idx, T, K, E, W, S, s.bitmap,
-                   s.wprefix, s.counts, offsets, L->status);
-    if (e != cudaSuccess) return e;
-  } else {
-    uint32_t* done = reinterpret_cast<uint32_t*>(s.counts + E);
-    e = launch_pdl(permute_clear_kernel, dim3(unsigned((nwords + 1023) / 1024)), dim3(256), 0, st, s.bitmap, nwords,
-                   done);
-    if (e != cudaSuccess) return e;
-    e = launch_pdl(permute_bitmap_kernel, dim3((T * K + 255) / 256), dim3(256), 0, st, idx, T, K, E, W, s.bitmap,
-                   L->status);
-    if (e != cudaSuccess) return e;
-    e = launch_pdl(permute_count_kernel, dim3(E), dim3(256), 0, st, static_cast<const uint32_t*>(s.bitmap), W,
-                   s.wprefix, s.counts, E, T, S, offsets, done);
-    if (e != cudaSuccess) return e;
-  }
+  cudaError_t e = launch_plan(L, idx, T, offsets, s, st);
+  if (e != cudaSuccess) return e;
+  GatherArgs a = {};
+  a.x = x;
+  a.T = T;
+  a.ldx = ldx;
+  a.H = L->H;
+  a.idx = idx;
+  a.K = K;
+  a.E = E;
+  a.W = W;
+  a.S = S;
+  a.bitmap = s.bitmap;
+  a.wprefix = s.wprefix;
+  a.offsets = offsets;
+  a.rows = rows;
+  a.perm = perm;
+  a.inv = inv;
+  a.xq = xq;
+  a.xs = xs;
   const int nchunk = (L->HB + GATHER_GROUPS - 1) / GATHER_GROUPS;
   const long long warps = static_cast<long long>(T) * nchunk;
-  return launch_pdl(permute_gather_kernel, dim3(unsigned((warps + 7) / 8)), dim3(256), 0, st, x, T, ldx, L->H, idx,
-                    K, E, W, static_cast<const uint32_t*>(s.bitmap), static_cast<const uint32_t*>(s.wprefix),
-                    static_cast<const int32_t*>(offsets), S, rows, perm, inv, xq, xs);
+  const int wpc = GATHER_THREADS / 32;
+  return launch_pdl(gather_rows_kernel<GATHER_LOCAL>, dim3(unsigned((warps + wpc - 1) / wpc)), dim3(GATHER_THREADS),
+                    0, st, a);
+}
+
+cudaError_t launch_ep_plan(const moe_layer_s* L, const int32_t* idx, int T, int32_t* offsets, const Scratch& s,
+                           cudaStream_t st) {
+  return launch_plan(L, idx, T, offsets, s, st);
+}
+
+cudaError_t launch_ep_dispatch(const moe_layer_s* L, const moe_ep_comm_s* c, const uint16_t* x, int T, int ldx,
+                               const int32_t* idx, const int32_t* all_off, int32_t* inv_ep, int32_t* goff,
+                               const Scratch& s, cudaStream_t st) {
+  GatherArgs a = {};
+  a.x = x;
+  a.T = T;
+  a.ldx = ldx;
+  a.H = L->H;
+  a.idx = idx;
+  a.K = L->K;
+  a.E = L->E;
+  a.W = (T + 31) / 32;
+  a.S = L->S;
+  a.bitmap = s.bitmap;
+  a.wprefix = s.wprefix;
+  a.all_off = all_off;
+  a.rank = c->rank;
+  a.ranks = c->ranks;
+  a.El = L->E / c->ranks;
+  a.cap = c->cap;
+  a.peer_q = c->d_peer_q;
+  a.peer_s = c->d_peer_s;
+  a.inv_ep = inv_ep;
+  a.goff = goff;
+  a.status = L->status;
+  const int nchunk = (L->HB + GATHER_GROUPS - 1) / GATHER_GROUPS;
+  const long long warps = static_cast<long long>(T) * nchunk;
+  const int wpc = GATHER_THREADS / 32;
+  const long long ctas = (warps + wpc - 1) / wpc;
+  // at least one CTA: it writes the owner offsets even when this rank sends nothing
+  return launch_pdl(gather_rows_kernel<GATHER_EP>, dim3(unsigned(ctas > 0 ? ctas : 1)), dim3(GATHER_THREADS), 0, st,
+                    a);
 }
 
 // ---------------------------------------------------------------------------

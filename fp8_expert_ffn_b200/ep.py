@@ -17,9 +17,17 @@ router and the shared expert are on every rank. One forward on rank r:
   4. return each sender's rows with a third all-to-all, into the sender's
      own permuted-row order, and combine.
 
+Two transports. ep_forward + CudaOps: the rows cross in torch.distributed
+all-to-alls (NCCL between GPUs, each rank's rows landing in its own memory
+before any kernel reads them) and are regrouped by the library's kernels.
+ep_forward_peer + PeerOps: the library's dispatch kernel writes every routed
+row straight into its owner's receive buffer (a peer GPU's memory, mapped
+with CUDA IPC through EpComm) at the row the owner's GEMMs read, and the
+combine kernel reads the owners' output rows back; the only collectives are
+an all-gather of the E+2 offsets of every rank and two barriers.
+
 Host orchestration only: every step of the layer runs in the library's
-kernels (CudaOps), the exchanges in torch.distributed (NCCL between GPUs,
-each rank's rows landing in its own memory before any kernel reads them).
+kernels.
 The orchestration takes the compute and the exchange as objects, so tests
 can drive the same code with CPU ranks over gloo or with several emulated
 ranks on one GPU.
@@ -200,3 +208,104 @@ def ep_forward(ops, exchange, x, T: int):
     R = T * ops.K
     exchange.rows(y_send, disp.recv_rows, disp.send_rows, y_own[:R])
     return ops.combine(st, y_own, T)
+
+
+# ----------------------------------------------------------------------------- over peer memory
+
+class PeerOps:
+    """The layer's steps on this rank with the dispatch and combine over
+    peer memory (moe_ep_plan / moe_ep_dispatch / moe_ep_combine): routed
+    rows are written straight into their owners' receive buffers and read
+    back from the owners' output rows, so no row crosses an all-to-all and
+    no regroup is needed. `comm` is this rank's connected EpComm."""
+
+    def __init__(self, route_layer, expert_layer, comm, ranks: int):
+        import torch
+        from . import torch_utils
+        self.torch, self.tu = torch, torch_utils
+        self.route_layer, self.expert_layer, self.comm, self.ranks = route_layer, expert_layer, comm, ranks
+        self.H, self.E, self.K, self.S = route_layer.H, route_layer.E, route_layer.K, route_layer.S
+        self.El = expert_layer.E
+        assert self.El * ranks == self.E and expert_layer.S == self.S and expert_layer.K == self.K
+        assert comm.ranks == ranks
+        cap = comm.capacity
+        FB = -(-expert_layer.F // 128)
+        d = "cuda"
+        self.h = torch.empty((cap, FB * 128), dtype=torch.uint8, device=d)
+        self.hs = torch.empty((FB, cap), dtype=torch.float32, device=d)
+        self.goff = torch.empty(self.El + 2, dtype=torch.int32, device=d)
+        self.device = d
+
+    def plan(self, x, T):
+        from . import moe_ep_plan, moe_route
+        t = self.torch
+        st = {"x": x, "ws": self.tu.workspace(self.route_layer, T) if T else None,
+              "idx": t.empty((T, self.K), dtype=t.int32, device=self.device),
+              "w": t.empty((T, self.K), dtype=t.float32, device=self.device),
+              "inv": t.empty((T, self.K), dtype=t.int32, device=self.device)}
+        off = t.empty(self.E + 2, dtype=t.int32, device=self.device)
+        nb = st["ws"].numel() if T else 0
+        if T:
+            moe_route(self.route_layer, x, T, self.H, st["idx"], st["w"], None, st["ws"], nb)
+        moe_ep_plan(self.route_layer, st["idx"], T, off, st["ws"], nb)
+        return st, off
+
+    def dispatch(self, st, all_off, T):
+        from . import moe_ep_dispatch
+        nb = st["ws"].numel() if T else 0
+        moe_ep_dispatch(self.route_layer, self.comm, st["x"], T, self.H, st["idx"], all_off, st["inv"], self.goff,
+                        st["ws"], nb)
+
+    def experts(self, st):
+        from . import moe_grouped_down, moe_grouped_gate_up
+        c = self.comm
+        moe_grouped_gate_up(self.expert_layer, c.recv_q, c.recv_s, self.goff, c.capacity, self.h, self.hs)
+        moe_grouped_down(self.expert_layer, self.h, self.hs, self.goff, c.capacity, c.y)
+
+    def combine(self, st, T):
+        from . import moe_ep_combine
+        out = self.torch.empty((T, self.H), dtype=self.torch.bfloat16, device=self.device)
+        moe_ep_combine(self.route_layer, self.comm, st["idx"], st["inv"], st["w"], self.goff, T, out, self.H)
+        return out
+
+
+class TorchSync:
+    """The two collectives of the peer-memory forward over torch.distributed
+    (NCCL: both are queued on the current stream, so no host wait): an
+    all-gather of every rank's offsets and a barrier (an all-reduce of one
+    word)."""
+
+    def __init__(self, group=None, device="cuda"):
+        import torch
+        import torch.distributed as dist
+        self.torch, self.dist, self.group = torch, dist, group
+        self.ranks = dist.get_world_size(group)
+        self.word = torch.zeros(1, dtype=torch.int32, device=device)
+
+    def all_gather(self, off):
+        out = self.torch.empty((self.ranks, off.numel()), dtype=off.dtype, device=off.device)
+        self.dist.all_gather_into_tensor(out, off.contiguous(), group=self.group)
+        return out
+
+    def barrier(self):
+        self.dist.all_reduce(self.word, group=self.group)
+
+
+def peer_capacity(tokens_per_rank: int, K: int, S: int, ranks: int) -> int:
+    """Receive rows that always suffice: every rank's routed rows going to
+    one owner, plus that owner's shared rows."""
+    return max(1, ranks * tokens_per_rank * K + tokens_per_rank * S)
+
+
+def ep_forward_peer(ops, sync, x, T: int):
+    """One expert-parallel forward of this rank's T tokens over peer memory:
+    plan, all-gather the offsets, dispatch into the owners' buffers, barrier,
+    the grouped GEMMs on this rank's buffer, barrier, combine from the
+    owners' output rows. Returns the [T][H] output."""
+    st, off = ops.plan(x, T)
+    all_off = sync.all_gather(off)
+    ops.dispatch(st, all_off, T)
+    sync.barrier()
+    ops.experts(st)
+    sync.barrier()
+    return ops.combine(st, T)

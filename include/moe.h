@@ -35,7 +35,8 @@
  *     8*256*H*4 bytes (42 MB at H = 5120); and, when a router bias is
  *     given, an E*4-byte copy of it. Nothing else is allocated (the one
  *     file-scope array of moe_permute_noalloc, below, is part of the
- *     library image, not an allocation);
+ *     library image, not an allocation), except by moe_ep_comm_create,
+ *     which allocates the expert-parallel exchange buffers it describes;
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default);
  *     calls are asynchronous on that stream and never synchronise the host;
  *     the kernels are chained with programmatic dependent launch (each one's
@@ -297,6 +298,99 @@ moe_status moe_ep_regroup(moe_layer_t expert_layer, int ranks, const int32_t* se
 moe_status moe_ep_unregroup(moe_layer_t expert_layer, int ranks, const int32_t* seg_counts, int n_recv,
                             const uint16_t* y_g, int T, uint16_t* y_send, uint16_t* y_own, void* stream);
 
+/* Expert parallelism over peer memory: the dispatch and combine of the
+ * DeepEP transport (SGLang cookbook "Dots3-Note", "2. Configuration Tips")
+ * done by the library's own kernels, with no all-to-all of rows. The
+ * dispatch kernel quantises each routed row and stores it straight into
+ * the receive buffer of its expert's owner (a peer GPU's memory over
+ * NVLink, through a CUDA IPC mapping), at the row the owner's grouped GEMMs
+ * read it from; the combine kernel reads the owners' output rows back the
+ * same way. The caller exchanges only the E+2 offsets of every rank (an
+ * all-gather) and orders the phases with two barriers (a kernel never waits
+ * on another rank). Per forward, on every rank r of P:
+ *   1. moe_route (route handle), then moe_ep_plan -> offsets [E+2];
+ *   2. all-gather the offsets -> all_offsets [P][E+2] (rank order);
+ *   3. moe_ep_dispatch -> rows into the owners' buffers, inv_ep, and this
+ *      rank's group_offsets [El+2] as an owner;
+ *   4. barrier (every rank's dispatch complete);
+ *   5. moe_grouped_gate_up / moe_grouped_down (expert handle) on this
+ *      rank's buffers (moe_ep_comm_buffers) with group_offsets and
+ *      rows = capacity;
+ *   6. barrier (every owner's y complete);
+ *   7. moe_ep_combine -> out [T][H].
+ * The next forward's step 2 keeps a rank from overwriting buffers that a
+ * slower rank still reads.
+ *
+ * Owner p's buffer holds, for its local experts e = 0..El-1 in turn, the
+ * rows from sender 0, 1, ..., P-1 (each sender's in token order), then its
+ * own T*S shared rows: the rows a single-GPU forward would give those
+ * experts, regrouped. `capacity` rows bound every owner's total; a forward
+ * whose rows for some owner exceed it dispatches nothing on any rank, sets
+ * MOE_STATUS_EP_OVERFLOW and writes zero group offsets. */
+typedef struct moe_ep_comm_s* moe_ep_comm_t;
+
+#define MOE_EP_HANDLE_BYTES 64   /* one rank's exported buffer handle */
+
+/* Allocates this rank's exchange buffers on the current device (one
+ * allocation: codes [capacity][H] u8, scales [H/128][capacity] fp32, output
+ * rows [capacity][H] bf16) and the device tables of the P ranks' buffers.
+ * `layer` gives H (any handle of the layer). 1 <= ranks <= 64,
+ * 0 <= rank < ranks, 1 <= capacity <= 2^20. Library plumbing: no
+ * counterpart on the pages. */
+moe_status moe_ep_comm_create(moe_layer_t layer, int rank, int ranks, int capacity, moe_ep_comm_t* out);
+/* The handle another process passes to moe_ep_comm_connect to map this
+ * rank's buffers (cudaIpcGetMemHandle of the allocation). Library
+ * plumbing: no counterpart on the pages. */
+moe_status moe_ep_comm_export(moe_ep_comm_t comm, unsigned char handle[MOE_EP_HANDLE_BYTES]);
+/* Maps every other rank's buffers from `handles` ([ranks][MOE_EP_HANDLE_BYTES],
+ * in rank order; this rank's own entry is not used) and fills the tables.
+ * Peers must have been created with the same ranks, capacity and H.
+ * Library plumbing: no counterpart on the pages. */
+moe_status moe_ep_comm_connect(moe_ep_comm_t comm, const unsigned char* handles);
+/* Emulated ranks in one process on one device: comms[0..ranks) (rank i at
+ * index i) use one another's buffers directly. Library plumbing: no
+ * counterpart on the pages. */
+moe_status moe_ep_comm_connect_local(moe_ep_comm_t* comms, int ranks);
+/* This rank's own buffers (device pointers): codes, scales, output rows.
+ * Library plumbing: no counterpart on the pages. */
+moe_status moe_ep_comm_buffers(moe_ep_comm_t comm, uint8_t** recv_q, float** recv_s, uint16_t** y);
+/* Unmaps the peers' buffers and frees this rank's (synchronises the device;
+ * call it on every rank together, after the last forward). Library
+ * plumbing: no counterpart on the pages. */
+moe_status moe_ep_comm_destroy(moe_ep_comm_t comm);
+
+/* Step 1 of the expert-parallel forward of the SGLang cookbook
+ * "Dots3-Note" ("2. Configuration Tips"): the plan of the permutation of
+ * this rank's T tokens (route handle): offsets [E+2] as moe_permute gives them (offsets[E] = T*K
+ * routed rows, offsets[E+1] = offsets[E] + T*S), and the token bitmap and
+ * its prefixes in `ws` (moe_workspace_size(route_layer, T) bytes), which
+ * moe_ep_dispatch reads: pass it the same workspace, unchanged. T = 0 writes
+ * zero offsets. */
+moe_status moe_ep_plan(moe_layer_t route_layer, const int32_t* idx, int T, int32_t* offsets, void* ws,
+                       size_t ws_bytes, void* stream);
+/* Step 3, the DeepEP "dispatch" of the SGLang cookbook "Dots3-Note"
+ * ("2. Configuration Tips") (route handle; comm connected; route_layer
+ * n_routed divisible by the comm's ranks): quantises x [T][ldx] bf16 per token per 128 channels
+ * (as moe_permute) and writes routed row (t, k) into the buffer of expert
+ * idx[t][k]'s owner and t's shared row into this rank's; inv_ep [T][K] =
+ * the row in the owner's buffer (-1 for a skipped slot; the owner is
+ * idx[t][k] / El); group_offsets [El+2] = this rank's offsets as an owner
+ * (shared rows from group_offsets[El]). all_offsets [ranks][E+2] is every
+ * rank's moe_ep_plan output. Runs with T = 0 too (it still writes
+ * group_offsets). Offsets that are not ascending, or rows of this rank
+ * beyond its own entry of all_offsets, are skipped and set
+ * MOE_STATUS_BAD_PLAN: no store leaves the owners' buffers. */
+moe_status moe_ep_dispatch(moe_layer_t route_layer, moe_ep_comm_t comm, const uint16_t* x, int T, int ldx,
+                           const int32_t* idx, const int32_t* all_offsets, int32_t* inv_ep, int32_t* group_offsets,
+                           void* ws, size_t ws_bytes, void* stream);
+/* Step 7, the DeepEP "combine" of the SGLang cookbook "Dots3-Note"
+ * (route handle): out [T][ldo] bf16 = sum over slots k of w[t][k]
+ * times row inv_ep[t][k] of the owner's output rows (slot order, FP32),
+ * plus this rank's shared row group_offsets[El] + t, rounded once to bf16:
+ * the same arithmetic as moe_combine. */
+moe_status moe_ep_combine(moe_layer_t route_layer, moe_ep_comm_t comm, const int32_t* idx, const int32_t* inv_ep,
+                          const float* w, const int32_t* group_offsets, int T, uint16_t* out, int ldo, void* stream);
+
 /* Weighted combine of the routed experts' outputs plus the shared expert's
  * (Dots3NoteTextConfig: norm_topk_prob, routed_scaling_factor,
  * n_shared_experts 1), the "combine" of the DeepEP transport of the SGLang
@@ -320,6 +414,7 @@ moe_status moe_layer_forward(moe_layer_t layer, const uint16_t* x, int T, int ld
 #define MOE_STATUS_DUP_EXPERT 0x2u   /* an expert repeated in one token's slots */
 #define MOE_STATUS_WAIT_TIMEOUT 0x4u /* a pipeline wait gave up; that launch's outputs are incomplete */
 #define MOE_STATUS_BAD_PLAN 0x8u     /* group offsets not ascending within [0, rows]; no GEMM work done */
+#define MOE_STATUS_EP_OVERFLOW 0x10u /* an owner's rows exceed its exchange buffer; nothing dispatched */
 
 /* Synchronises `stream`, returns MOE_ERR_DEVICE if any kernel of this layer
  * flagged an error since the last call (and clears the flag), else MOE_OK.

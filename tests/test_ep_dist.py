@@ -134,3 +134,125 @@ def test_plan_dispatch_splits_rows_by_owner():
     assert d.send_rows == [3, 7, 2, 4] and d.recv_rows == [4, 2, 7, 3] and d.n_recv == 16
     with pytest.raises(ValueError):
         ep.local_experts(10, 4)
+
+
+# ----------------------------------------------------------------------------- over peer memory
+
+class HostPeerOps:
+    """ep.PeerOps's interface on CPU: every rank's receive buffers are
+    shared-memory tensors that all processes map (the stand-in for a peer
+    GPU's memory), and the steps are the oracle's. The dispatch writes each
+    routed row at the owner-side row that include/moe.h defines: owner p
+    holds, for its local experts in turn, sender 0's rows, sender 1's, ...,
+    then its own shared rows."""
+
+    def __init__(self, layer, rank, ranks, bufs):
+        self.base = HostOps(layer, rank, ranks)
+        self.moe, self.layer, self.bufs = self.base.moe, layer, bufs
+        self.E, self.K, self.S, self.H = self.base.E, self.base.K, self.base.S, self.base.H
+        self.El, self.rank, self.ranks = self.base.El, rank, ranks
+
+    def plan(self, x, T):
+        m = self.moe
+        r = m.route_layer(x, self.layer)
+        p = m.permute(r.idx, self.E, self.S)
+        tq, ts = m.quantize_tokens(x)
+        st = {"idx": r.idx, "w": r.w, "inv": p.inv, "perm": p.perm, "offsets": p.offsets, "tq": tq, "ts": ts, "T": T}
+        return st, torch.from_numpy(p.offsets.astype(np.int32))
+
+    def dispatch(self, st, all_off, T):
+        ao = np.asarray(all_off, np.int64)
+        cnt = np.diff(ao[:, :self.E + 1], axis=1)              # [sender][expert]
+        tot, pre = cnt.sum(0), cnt[:self.rank].sum(0)
+        off, El = st["offsets"], self.El
+        for g in range(self.E):
+            p, b0 = g // El, (g // El) * El
+            base = int(tot[b0:g].sum() + pre[g])
+            rows = np.arange(off[g], off[g + 1])
+            toks = st["perm"][rows]
+            self.bufs[p]["q"][base:base + len(rows)] = torch.from_numpy(st["tq"][toks])
+            self.bufs[p]["s"][base:base + len(rows)] = torch.from_numpy(st["ts"][toks])
+            st.setdefault("where", {}).update({int(r): (p, base + i) for i, r in enumerate(rows)})
+        mine = tot[self.rank * El:(self.rank + 1) * El]
+        n_r = int(mine.sum())
+        self.bufs[self.rank]["q"][n_r:n_r + T * self.S] = torch.from_numpy(st["tq"][:T])
+        self.bufs[self.rank]["s"][n_r:n_r + T * self.S] = torch.from_numpy(st["ts"][:T])
+        st["goff"] = np.concatenate([[0], np.cumsum(mine), [n_r + T * self.S]]).astype(np.int64)
+
+    def experts(self, st):
+        goff, n = st["goff"], int(st["goff"][-1])
+        b = self.bufs[self.rank]
+        y = self.moe.expert_ffn_rows(b["q"][:n].numpy(), b["s"][:n].numpy(), goff, self.base.local)["y"]
+        b["y"][:n] = torch.from_numpy(y)
+
+    def combine(self, st, T):
+        R = T * self.K
+        y_local = np.zeros((R + T * self.S, self.H))
+        for r, (p, row) in st.get("where", {}).items():
+            y_local[r] = self.bufs[p]["y"][row].numpy()
+        n_r = int(st["goff"][self.El])
+        y_local[R:] = self.bufs[self.rank]["y"][n_r:n_r + T * self.S].numpy()
+        return self.moe.combine(y_local, st["inv"], st["w"], self.S)
+
+
+class GlooSync:
+    def all_gather(self, off):
+        out = [torch.empty_like(off) for _ in range(dist.get_world_size())]
+        dist.all_gather(out, off)
+        return torch.stack(out)
+
+    def barrier(self):
+        dist.barrier()
+
+
+def _peer_worker(rank, world, port, T, bufs, q, idle_rank=-1):
+    import sys
+    sys.path.insert(0, ROOT)
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        import gen
+        from fp8_expert_ffn_b200 import ep
+        from oracle import moe
+        _, layer, _ = gen.workload_inputs("toy")
+        Tr = 0 if rank == idle_rank else T
+        x = gen.make_x(Tr, layer.shape.H, 100 + rank, outliers=2)
+        ops = HostPeerOps(layer, rank, world, bufs)
+        outs = [ep.ep_forward_peer(ops, GlooSync(), x, Tr) for _ in range(2)]   # buffers reused
+        if Tr == 0:
+            err = max(0.0 if o.shape == (0, layer.shape.H) else 1.0 for o in outs)
+        else:
+            ref = moe.layer_forward(x, layer)["out"]
+            err = max(float(np.max(np.abs(o - ref)) / np.max(np.abs(ref))) for o in outs)
+        q.put((rank, err))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,idle", [(2, -1), (4, -1), (4, 2)])
+def test_peer_transport_forward_matches_single_rank(world, idle):
+    """ep.ep_forward_peer's order of steps and collectives across processes,
+    with the ranks' buffers in shared memory: every rank's output equals the
+    oracle's single-rank layer, twice in a row on the same buffers."""
+    from fp8_expert_ffn_b200 import ep
+    import gen
+    _, layer, _ = gen.workload_inputs("toy")
+    sh = layer.shape
+    T = 24
+    cap = ep.peer_capacity(T, sh.K, sh.S, world)
+    bufs = [{"q": torch.zeros((cap, sh.H), dtype=torch.uint8).share_memory_(),
+             "s": torch.zeros((cap, sh.HB), dtype=torch.float64).share_memory_(),
+             "y": torch.zeros((cap, sh.H), dtype=torch.float64).share_memory_()} for _ in range(world)]
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_peer_worker, args=(r, world, port, T, bufs, q, idle)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=180)
+    assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]
+    res = sorted(q.get(timeout=10) for _ in range(world))
+    for rank, err in res:
+        assert err <= 1e-12, (rank, err)

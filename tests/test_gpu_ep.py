@@ -1,5 +1,6 @@
 """Expert parallelism through the library's kernels on one GPU: P emulated
-ranks run as threads, each with a routing-only handle over all experts and
+ranks run as threads (both transports: the all-to-all one and the one over
+peer memory, whose "peers" are then buffers on this GPU), each with a routing-only handle over all experts and
 an expert handle over its own block of experts plus the shared expert; an
 in-process exchange stands in for the all-to-alls (no collective, no kernel
 waits on another). Each rank's output must be bit-identical to the
@@ -148,3 +149,115 @@ def test_routing_only_handle_refuses_gemm_calls():
     with pytest.raises(fx.MoeError) as e:
         fx.moe_layer_forward(route, x, T, sh.H, out, sh.H, ws, ws.numel())
     assert e.value.code == fx.MOE_ERR_INVALID_ARG
+
+
+# ----------------------------------------------------------------------------- over peer memory
+
+class LocalSync:
+    """The offsets all-gather and the barriers between emulated ranks
+    (threads of this process; every rank's kernels are finished before it
+    reaches a barrier, so no kernel waits on another)."""
+
+    def __init__(self, ranks):
+        self.ranks = ranks
+        self.bar = threading.Barrier(ranks, timeout=300)
+        self.box = [None] * ranks
+
+    def view(self, rank):
+        return _SyncView(self, rank)
+
+
+class _SyncView:
+    def __init__(self, s, rank):
+        self.s, self.rank = s, rank
+
+    def all_gather(self, off):
+        torch.cuda.synchronize()
+        self.s.box[self.rank] = off
+        self.s.bar.wait()
+        out = torch.stack(list(self.s.box))
+        self.s.bar.wait()
+        return out
+
+    def barrier(self):
+        torch.cuda.synchronize()
+        self.s.bar.wait()
+
+
+def _run_peer(name, ranks, T, layer=None, xs=None, capacity=None, expect_overflow=False):
+    wl, layer0, _ = gen.workload_inputs(name)
+    layer = layer0 if layer is None else layer
+    sh = layer.shape
+    dev = tu.upload_layer(layer)
+    if xs is None:
+        xs = [gen.make_x(T, sh.H, 300 + r, outliers=wl.outliers) for r in range(ranks)]
+    refs = []
+    for x in xs:
+        Tr = x.shape[0]
+        o = torch.empty((Tr, sh.H), dtype=torch.bfloat16, device="cuda")
+        if Tr:
+            ws = tu.workspace(dev, Tr)
+            fx.moe_layer_forward(dev, tu.bf16_tensor(x), Tr, sh.H, o, sh.H, ws, ws.numel())
+        refs.append(o)
+    layers = [ep.rank_layers(dev, r, ranks) for r in range(ranks)]
+    cap = capacity or ep.peer_capacity(max(x.shape[0] for x in xs), sh.K, sh.S, ranks)
+    comms = [fx.EpComm(layers[r][0], r, ranks, cap) for r in range(ranks)]
+    fx.EpComm.connect_local(comms)
+    sync = LocalSync(ranks)
+    outs, errs = [None] * ranks, []
+
+    def one(r):
+        try:
+            torch.cuda.set_device(0)
+            ops = ep.PeerOps(layers[r][0], layers[r][1], comms[r], ranks)
+            outs[r] = ep.ep_forward_peer(ops, sync.view(r), tu.bf16_tensor(xs[r]), xs[r].shape[0])
+        except BaseException as e:   # noqa: BLE001 - re-raised below
+            errs.append(e)
+            sync.bar.abort()
+
+    th = [threading.Thread(target=one, args=(r,)) for r in range(ranks)]
+    for t in th:
+        t.start()
+    for t in th:
+        t.join()
+    if errs:
+        raise errs[0]
+    for r in range(ranks):
+        code, bits = fx.moe_get_device_status(layers[r][0])
+        if expect_overflow:
+            assert code == fx.MOE_ERR_DEVICE and bits == 0x10, hex(bits)
+            continue
+        assert code == fx.MOE_OK, hex(bits)
+        assert fx.moe_get_device_status(layers[r][1])[0] == fx.MOE_OK
+        assert torch.equal(outs[r].view(torch.int16), refs[r].view(torch.int16)), f"rank {r} differs"
+    for c in comms:
+        c.close()
+
+
+@pytest.mark.parametrize("ranks", [1, 2, 4])
+def test_peer_dispatch_toy_layer_matches_single_gpu(ranks):
+    """Dispatch into the owners' buffers, grouped GEMMs on each owner's
+    buffer, combine from the owners' rows: bit-identical to the single-GPU
+    forward of the whole layer on every rank's tokens."""
+    _run_peer("toy", ranks, 512)
+
+
+def test_peer_dispatch_full_layer_two_ranks():
+    """256 routed experts split 128 + 128, 64 tokens per rank (decode)."""
+    _run_peer("decode", 2, 64)
+
+
+def test_peer_dispatch_full_layer_eight_ranks_ragged():
+    """8 ranks of 32 experts with different token counts per rank (one
+    with none): owners receive from every sender, sizes not multiples of 32."""
+    wl, layer, _ = gen.workload_inputs("decode")
+    counts = [64, 1, 0, 37, 128, 5, 64, 33]
+    xs = [gen.make_x(n, layer.shape.H, 400 + r, outliers=wl.outliers) for r, n in enumerate(counts)]
+    _run_peer("decode", 8, None, xs=xs)
+
+
+def test_peer_dispatch_overflow_is_flagged_and_dispatches_nothing():
+    """A capacity below some owner's rows: every rank flags
+    MOE_STATUS_EP_OVERFLOW, writes zero group offsets (the GEMMs do
+    nothing) and no row is written out of bounds."""
+    _run_peer("toy", 2, 64, capacity=16, expect_overflow=True)
