@@ -6,7 +6,9 @@
 // Preview", Dots3NoteTextConfig: n_shared_experts 1, norm_topk_prob True,
 // routed_scaling_factor 1.0). This is the "combine" of the pages' DeepEP
 // transport (SGLang cookbook "Dots3-Note", "2. Configuration Tips"), here a
-// deterministic gather: fixed slot order, shared row last, no atomics.
+// deterministic gather: fixed slot order, shared row last, no atomics. With
+// expert parallelism over peer memory (combine_kernel<true>) each slot's row
+// is read from the output rows of its expert's owner rank.
 #include "common.cuh"
 #include "internal.h"
 

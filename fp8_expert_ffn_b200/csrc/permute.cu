@@ -12,15 +12,19 @@
 // bit of a per-expert token bitmap (atomicOr, order-independent). The row of
 // (t, k) inside expert e's group is the number of earlier tokens that chose
 // e: a prefix popcount over e's bitmap words. Kernels:
-//   1. permute_bitmap   one thread per (t, k): validate, set the bit
-//   2. permute_count    one CTA per expert: per-word prefix popcounts, count;
+//   1. permute_clear    zero the bitmap and the completion counter
+//   2. permute_bitmap   one thread per (t, k): validate, set the bit
+//   3. permute_count    one CTA per expert: per-word prefix popcounts, count;
 //                       the last CTA to finish scans the counts -> offsets[E+2]
 //   (small batches: 1-3 in one CTA, permute_plan_small, when the bitmap fits
 //   in shared memory)
-//   4. permute_gather   one warp per token and 16 groups of 128 channels:
+//   4. gather_rows      one warp per token and 16 groups of 128 channels:
 //                       rows of its K slots and its shared-expert row,
 //                       inv/perm, then the groups of x quantised once and
 //                       stored to all rows with 16-byte stores.
+// With expert parallelism over peer memory the same gather is the dispatch
+// (gather_rows<GATHER_EP>): each routed row goes to the receive buffer of
+// its expert's owner rank, at the row the owner's grouped GEMMs read.
 #include <mutex>
 
 #include "common.cuh"
@@ -241,7 +245,7 @@ __device__ void ep_layout(const GatherArgs& a, int* s_base, int* s_excl, int* s_
   if (i == 0) *s_over = 0;
   __syncthreads();
   if (bad) {   // offsets not ascending: nothing is dispatched
-    atomicOr(s_over, 1);
+    atomicOr(s_over, 2);
     set_status(a.status, STATUS_BAD_PLAN);
   }
   int before = 0;
@@ -253,7 +257,12 @@ __device__ void ep_layout(const GatherArgs& a, int* s_base, int* s_excl, int* s_
   if (i < a.ranks) {   // owner i's routed rows plus its own shared rows must fit its buffer
     const int n = s_excl[(i + 1) * a.El] - s_excl[i * a.El];
     const int sh = a.all_off[i * stride + E + 1] - a.all_off[i * stride + E];
-    if (sh < 0 || n + sh > a.cap) atomicOr(s_over, 1);
+    if (sh < 0) {
+      atomicOr(s_over, 2);
+      set_status(a.status, STATUS_BAD_PLAN);
+    } else if (n + sh > a.cap) {
+      atomicOr(s_over, 1);
+    }
   }
   if (i == 0) *s_nr = s_excl[(a.rank + 1) * a.El] - s_excl[a.rank * a.El];
   __syncthreads();
@@ -265,7 +274,7 @@ __device__ void ep_layout(const GatherArgs& a, int* s_base, int* s_excl, int* s_
       const int sh = a.all_off[a.rank * stride + E + 1] - a.all_off[a.rank * stride + E];
       a.goff[a.El] = over ? 0 : *s_nr;
       a.goff[a.El + 1] = over ? 0 : *s_nr + sh;
-      if (over) set_status(a.status, STATUS_EP_OVERFLOW);
+      if (*s_over & 1) set_status(a.status, STATUS_EP_OVERFLOW);
     }
   }
 }

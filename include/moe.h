@@ -377,9 +377,10 @@ moe_status moe_ep_plan(moe_layer_t route_layer, const int32_t* idx, int T, int32
  * idx[t][k] / El); group_offsets [El+2] = this rank's offsets as an owner
  * (shared rows from group_offsets[El]). all_offsets [ranks][E+2] is every
  * rank's moe_ep_plan output. Runs with T = 0 too (it still writes
- * group_offsets). Offsets that are not ascending, or rows of this rank
- * beyond its own entry of all_offsets, are skipped and set
- * MOE_STATUS_BAD_PLAN: no store leaves the owners' buffers. */
+ * group_offsets). Offsets that are not ascending dispatch nothing (zero
+ * group offsets, inv_ep all -1); rows of this rank beyond its own entry of
+ * all_offsets are skipped (inv_ep -1); both set MOE_STATUS_BAD_PLAN. No
+ * store leaves the owners' buffers. */
 moe_status moe_ep_dispatch(moe_layer_t route_layer, moe_ep_comm_t comm, const uint16_t* x, int T, int ldx,
                            const int32_t* idx, const int32_t* all_offsets, int32_t* inv_ep, int32_t* group_offsets,
                            void* ws, size_t ws_bytes, void* stream);

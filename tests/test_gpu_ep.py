@@ -261,3 +261,52 @@ def test_peer_dispatch_overflow_is_flagged_and_dispatches_nothing():
     MOE_STATUS_EP_OVERFLOW, writes zero group offsets (the GEMMs do
     nothing) and no row is written out of bounds."""
     _run_peer("toy", 2, 64, capacity=16, expect_overflow=True)
+
+
+@pytest.mark.parametrize("case", ["short_own_entry", "descending"])
+def test_peer_dispatch_inconsistent_offsets_flag_bad_plan(case):
+    """All-gathered offsets that do not match the plan: rows of this rank
+    beyond its own entry are skipped (the rest still dispatched), and
+    offsets that descend dispatch nothing; both set MOE_STATUS_BAD_PLAN and
+    no store leaves the owners' buffers (the GEMMs and the combine then run
+    normally on what is there)."""
+    wl, layer, _ = gen.workload_inputs("toy")
+    sh = layer.shape
+    dev = tu.upload_layer(layer)
+    ranks, T = 2, 64
+    layers = [ep.rank_layers(dev, r, ranks) for r in range(ranks)]
+    cap = ep.peer_capacity(T, sh.K, sh.S, ranks)
+    comms = [fx.EpComm(layers[r][0], r, ranks, cap) for r in range(ranks)]
+    fx.EpComm.connect_local(comms)
+    ops = [ep.PeerOps(layers[r][0], layers[r][1], comms[r], ranks) for r in range(ranks)]
+    xs = [tu.bf16_tensor(gen.make_x(T, sh.H, 600 + r, outliers=2)) for r in range(ranks)]
+    plans = [ops[r].plan(xs[r], T) for r in range(ranks)]
+    all_off = torch.stack([off for _, off in plans])
+    bad = all_off.clone()
+    if case == "short_own_entry":
+        e = int(torch.argmax(torch.diff(all_off[0][:sh.E + 1])))   # rank 0's fullest expert
+        bad[0, e + 1:] -= 1                # its count one short: one row of rank 0 is not its plan
+    else:
+        bad[1, 3] = bad[1, 4] + 5          # rank 1's offsets descend at expert 3
+    for r in range(ranks):
+        plans[r][0]["x"] = xs[r]
+        ops[r].dispatch(plans[r][0], bad, T)
+    torch.cuda.synchronize()
+    bits = [fx.moe_get_device_status(layers[r][0])[1] for r in range(ranks)]
+    if case == "short_own_entry":
+        assert bits[0] == 0x8 and bits[1] == 0, [hex(b) for b in bits]
+        inv0 = plans[0][0]["inv"]
+        assert int((inv0 < 0).sum()) == 1          # exactly the one row beyond the entry skipped
+    else:
+        assert all(b == 0x8 for b in bits), [hex(b) for b in bits]
+        assert all(int((ops[r].goff != 0).sum()) == 0 for r in range(ranks))
+        assert all(bool((plans[r][0]["inv"] < 0).all()) for r in range(ranks))
+    for r in range(ranks):
+        ops[r].experts(plans[r][0])
+        ops[r].combine(plans[r][0], T)
+    torch.cuda.synchronize()
+    for r in range(ranks):
+        for h in layers[r]:
+            assert fx.moe_get_device_status(h)[0] == fx.MOE_OK
+    for c in comms:
+        c.close()
