@@ -680,6 +680,7 @@ def run_ep(args):
             raise RuntimeError(f"device status {bits:#x}")
     if same != 0:
         raise RuntimeError(f"{int(same)} rank(s) differ from the single-GPU forward")
+    stages = ep_peer_stages(ops, ex, x, T, args.steps, d, sh, world) if comm is not None else None
     line = {
         "metric": "expert-parallel MoE-layer tokens/s", "value": round(value, 1), "unit": "tokens/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 5),
@@ -695,6 +696,8 @@ def run_ep(args):
         "single_gpu_forward_ms_per_step": round(single_ms, 5),
         "clocks": clocks,
     }
+    if stages:
+        line["stages"] = stages
     if rank == 0:
         print(json.dumps(line), flush=True)
     d.barrier()
@@ -703,6 +706,56 @@ def run_ep(args):
         comm.close()          # every rank is past its last read of the peers' buffers
     del ops, route, experts
     d.close()
+
+
+EP_STAGES = ("route_plan", "all_gather", "dispatch", "barrier_1", "experts", "barrier_2", "combine")
+
+
+def ep_peer_stages(ops, sync, x, T, steps, d: Dist, sh, world):
+    """The peer-memory forward again with CUDA events between its phases
+    (max over ranks of each phase's mean), and the dispatch and combine
+    kernels' bytes over their times: the dispatch reads x and writes every
+    token's K+S quantised rows with their scales (to the owners: over
+    NVLink for the rows of other ranks), the combine reads the K+S output
+    rows of every token and writes one; on one rank all of it is HBM
+    traffic, so their fraction of the measured HBM copy is given then."""
+    import torch
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(EP_STAGES) + 1)] for _ in range(steps)]
+    d.barrier()
+    torch.cuda.synchronize()
+    for i in range(steps):
+        e = evs[i]
+        e[0].record()
+        st, off = ops.plan(x, T)
+        e[1].record()
+        all_off = sync.all_gather(off)
+        e[2].record()
+        ops.dispatch(st, all_off, T)
+        e[3].record()
+        sync.barrier()
+        e[4].record()
+        ops.experts(st)
+        e[5].record()
+        sync.barrier()
+        e[6].record()
+        ops.combine(st, T)
+        e[7].record()
+    torch.cuda.synchronize()
+    d.barrier()
+    ms = {n: d.max(sum(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(steps)) / steps)
+          for j, n in enumerate(EP_STAGES)}
+    rows = T * (sh.K + sh.S)
+    disp_bytes = T * sh.H * 2 + rows * (sh.H + 4 * sh.HB) + T * sh.K * 8
+    comb_bytes = rows * sh.H * 2 + T * sh.H * 2 + T * sh.K * 12
+    out = {"ms": {k: round(v, 5) for k, v in ms.items()},
+           "dispatch_gbs": round(disp_bytes / (ms["dispatch"] / 1e3) / 1e9, 1),
+           "combine_gbs": round(comb_bytes / (ms["combine"] / 1e3) / 1e9, 1),
+           "bytes": {"dispatch": disp_bytes, "combine": comb_bytes}}
+    if world == 1:
+        hbm = peaks()["hbm_gbs"]
+        out["dispatch_frac_hbm"] = round(out["dispatch_gbs"] / hbm, 4)
+        out["combine_frac_hbm"] = round(out["combine_gbs"] / hbm, 4)
+    return out
 
 
 def _free_port():

@@ -92,6 +92,10 @@ Scratch carve(const moe_layer_s* L, int T, void* base) {
   s.bitmap = static_cast<uint32_t*>(take(sizeof(uint32_t) * E * W));
   s.wprefix = static_cast<uint32_t*>(take(sizeof(uint32_t) * E * W));
   s.counts = static_cast<int32_t*>(take(sizeof(int32_t) * (E + 1)));   // + the count kernel's completion counter
+  if (!L->has_experts) {   // a routing-only handle: route and permutation scratch only
+    s.total = align_up(off, 256);
+    return s;
+  }
   s.h = static_cast<uint8_t*>(take(rows * L->ld_hh));
   s.hs = static_cast<float*>(take(sizeof(float) * L->FB * rows));
   s.idx = static_cast<int32_t*>(take(sizeof(int32_t) * size_t(T) * K));

@@ -289,7 +289,7 @@ __device__ void ep_layout(const GatherArgs& a, int* s_base, int* s_excl, int* s_
 // buffer (a peer's memory over NVLink; every store is a plain 16- or 4-byte
 // store, no bulk or tensor copy) and the shared row into this rank's own.
 template <int MODE>
-__global__ void __launch_bounds__(GATHER_THREADS) gather_rows_kernel(const GatherArgs a) {
+__global__ void __launch_bounds__(GATHER_THREADS, 4) gather_rows_kernel(const GatherArgs a) {
   pdl_wait();
   pdl_launch_dependents();
   __shared__ int s_base[MODE == GATHER_EP ? 256 : 1];
@@ -297,6 +297,29 @@ __global__ void __launch_bounds__(GATHER_THREADS) gather_rows_kernel(const Gathe
   __shared__ int s_wsum[GATHER_THREADS / 32];
   __shared__ int s_nr, s_over;
   __shared__ uint64_t s_peer[MODE == GATHER_EP ? 2 * kEpMaxRanks : 1];   // codes, then scales
+  const int T = a.T, K = a.K, E = a.E, H = a.H;
+  const int lane = threadIdx.x & 31;
+  const int gl = lane & 7, gs = lane >> 3;   // lane within its group, group slot of the step
+  const int HB = H / 128;
+  const int nchunk = (HB + GATHER_GROUPS - 1) / GATHER_GROUPS;
+  const int wid = blockIdx.x * (GATHER_THREADS / 32) + (threadIdx.x >> 5);
+  const int t = wid / nchunk, chunk = wid - t * nchunk;
+  const bool has_token = t < T;
+  const int g0 = chunk * GATHER_GROUPS;
+  // issue the x loads of the whole chunk before anything waits on memory
+  // (with EP, before the layout is computed)
+  uint4 raw[4][2];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int g = g0 + 4 * i + gs;
+    if (has_token && g < HB) {
+      const uint4* src = reinterpret_cast<const uint4*>(a.x + size_t(t) * a.ldx + g * 128 + gl * 16);
+      raw[i][0] = src[0];
+      raw[i][1] = src[1];
+    } else {
+      raw[i][0] = raw[i][1] = make_uint4(0u, 0u, 0u, 0u);
+    }
+  }
   if (MODE == GATHER_EP) {
     for (int i = threadIdx.x; i < a.ranks; i += GATHER_THREADS) {
       s_peer[i] = a.peer_q[i];
@@ -304,29 +327,8 @@ __global__ void __launch_bounds__(GATHER_THREADS) gather_rows_kernel(const Gathe
     }
     ep_layout(a, s_base, s_excl, s_wsum, &s_nr, &s_over);   // ends with a CTA barrier
   }
-  const int T = a.T, K = a.K, E = a.E, W = a.W, H = a.H;
-  const int lane = threadIdx.x & 31;
-  const int gl = lane & 7, gs = lane >> 3;   // lane within its group, group slot of the step
-  const int HB = H / 128;
-  const int nchunk = (HB + GATHER_GROUPS - 1) / GATHER_GROUPS;
-  const int wid = blockIdx.x * (GATHER_THREADS / 32) + (threadIdx.x >> 5);
-  const int t = wid / nchunk, chunk = wid - t * nchunk;
-  if (t >= T) return;
-  const int g0 = chunk * GATHER_GROUPS;
-  const uint16_t* xr = a.x + size_t(t) * a.ldx;
-  // issue the x loads of the whole chunk before anything waits on memory
-  uint4 raw[4][2];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int g = g0 + 4 * i + gs;
-    if (g < HB) {
-      const uint4* src = reinterpret_cast<const uint4*>(xr + g * 128 + gl * 16);
-      raw[i][0] = src[0];
-      raw[i][1] = src[1];
-    } else {
-      raw[i][0] = raw[i][1] = make_uint4(0u, 0u, 0u, 0u);
-    }
-  }
+  if (!has_token) return;
+  const int W = a.W;
 
   // this lane's row; with EP the row in its owner's buffer, packed with the
   // owner's index (rows < 2^24, owners < 64)
@@ -427,9 +429,14 @@ __global__ void __launch_bounds__(GATHER_THREADS) gather_rows_kernel(const Gathe
     }
   }
   // the rows written into peers' memory are complete, system-wide, before
-  // this thread finishes (the owners read them after a barrier that follows
-  // this kernel)
-  if (MODE == GATHER_EP) __threadfence_system();
+  // the warp finishes (the owners read them after a barrier that follows
+  // this kernel): one system-scope fence per warp, after the warp's lanes
+  // have synchronised, orders all of the warp's stores (fences are
+  // cumulative)
+  if (MODE == GATHER_EP) {
+    __syncwarp();
+    if (lane == 0) __threadfence_system();
+  }
 }
 
 }  // namespace

@@ -236,14 +236,23 @@ class PeerOps:
         self.goff = torch.empty(self.El + 2, dtype=torch.int32, device=d)
         self.device = d
 
+    def _buffers(self, T):
+        """Per-token buffers and the routing workspace, kept between forwards
+        (stream order makes the reuse safe) and regrown for a larger T."""
+        t = self.torch
+        if getattr(self, "_T", -1) < T:
+            self._T = T
+            self._ws = self.tu.workspace(self.route_layer, T) if T else None
+            self._idx = t.empty((T, self.K), dtype=t.int32, device=self.device)
+            self._w = t.empty((T, self.K), dtype=t.float32, device=self.device)
+            self._inv = t.empty((T, self.K), dtype=t.int32, device=self.device)
+            self._off = t.empty(self.E + 2, dtype=t.int32, device=self.device)
+        return self._ws, self._idx[:T], self._w[:T], self._inv[:T], self._off
+
     def plan(self, x, T):
         from . import moe_ep_plan, moe_route
-        t = self.torch
-        st = {"x": x, "ws": self.tu.workspace(self.route_layer, T) if T else None,
-              "idx": t.empty((T, self.K), dtype=t.int32, device=self.device),
-              "w": t.empty((T, self.K), dtype=t.float32, device=self.device),
-              "inv": t.empty((T, self.K), dtype=t.int32, device=self.device)}
-        off = t.empty(self.E + 2, dtype=t.int32, device=self.device)
+        ws, idx, w, inv, off = self._buffers(T)
+        st = {"x": x, "ws": ws if T else None, "idx": idx, "w": w, "inv": inv}
         nb = st["ws"].numel() if T else 0
         if T:
             moe_route(self.route_layer, x, T, self.H, st["idx"], st["w"], None, st["ws"], nb)

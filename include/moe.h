@@ -156,8 +156,10 @@ moe_status moe_layer_create(const moe_layer_desc* desc, const moe_weights* w, mo
 moe_status moe_layer_destroy(moe_layer_t layer);
 
 /* Bytes of workspace that moe_layer_forward needs for T tokens; it also
- * covers the scratch of moe_permute and moe_expert_ffn. 0 on bad input.
- * Library plumbing: no counterpart on the pages. */
+ * covers the scratch of moe_route, moe_permute, moe_expert_ffn and the
+ * expert-parallel calls. For a routing-only handle it is the route and
+ * permutation scratch alone (a few bytes per token per expert). 0 on bad
+ * input. Library plumbing: no counterpart on the pages. */
 size_t moe_workspace_size(moe_layer_t layer, int T);
 
 /* Router: logits = x . router_w^T in FP32, p = softmax over the E experts,

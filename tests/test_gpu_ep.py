@@ -143,6 +143,8 @@ def test_routing_only_handle_refuses_gemm_calls():
     route = fx.MoeLayer(sh.H, sh.E, sh.K, sh.F, fx.LayerWeights(None, None, None, None, None, None,
                                                                  dev.weights.router_w), n_shared=sh.S)
     T = 8
+    # a routing-only handle's workspace is the route and permutation scratch alone
+    assert 0 < fx.moe_workspace_size(route, 4096) < fx.moe_workspace_size(dev, 4096) // 10
     x = torch.zeros((T, sh.H), dtype=torch.bfloat16, device="cuda")
     out = torch.empty_like(x)
     ws = tu.workspace(route, T)
