@@ -256,3 +256,62 @@ def test_peer_transport_forward_matches_single_rank(world, idle):
     res = sorted(q.get(timeout=10) for _ in range(world))
     for rank, err in res:
         assert err <= 1e-12, (rank, err)
+
+
+def _failing_worker(rank, world, port, T, bufs, q, dead_rank):
+    """dead_rank leaves between steps (after the first forward, before the
+    second: nothing of its own in flight); the others must see an error from
+    their next collective, not hang."""
+    import sys
+    from datetime import timedelta
+    sys.path.insert(0, ROOT)
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=20))
+    import gen
+    from fp8_expert_ffn_b200 import ep
+    _, layer, _ = gen.workload_inputs("toy")
+    x = gen.make_x(T, layer.shape.H, 100 + rank, outliers=2)
+    ops = HostPeerOps(layer, rank, world, bufs)
+    ep.ep_forward_peer(ops, GlooSync(), x, T)
+    if rank == dead_rank:
+        os._exit(3)                      # the rank is gone: no goodbye to the others
+    try:
+        ep.ep_forward_peer(ops, GlooSync(), x, T)
+        q.put((rank, "no error"))
+    except Exception as e:               # noqa: BLE001 - the failure is the expected outcome
+        q.put((rank, type(e).__name__))
+    q.close()
+    q.join_thread()                      # the message is sent before the process leaves
+    os._exit(0)
+
+
+def test_peer_transport_reports_a_dead_rank():
+    """A rank that dies between forwards: every other rank's next forward
+    fails in its first collective (the offsets all-gather) with an error
+    instead of waiting for ever; no kernel is involved (host stand-ins)."""
+    from fp8_expert_ffn_b200 import ep
+    import gen
+    import time
+    _, layer, _ = gen.workload_inputs("toy")
+    sh = layer.shape
+    world, T, dead = 4, 16, 1
+    cap = ep.peer_capacity(T, sh.K, sh.S, world)
+    bufs = [{"q": torch.zeros((cap, sh.H), dtype=torch.uint8).share_memory_(),
+             "s": torch.zeros((cap, sh.HB), dtype=torch.float64).share_memory_(),
+             "y": torch.zeros((cap, sh.H), dtype=torch.float64).share_memory_()} for _ in range(world)]
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_failing_worker, args=(r, world, port, T, bufs, q, dead)) for r in range(world)]
+    t0 = time.time()
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+    assert all(p.exitcode is not None for p in procs), "a rank hung"
+    assert procs[dead].exitcode == 3
+    res = sorted(q.get(timeout=10) for _ in range(world - 1))
+    assert [r for r, _ in res] == [r for r in range(world) if r != dead]
+    assert all(outcome in ("RuntimeError", "DistBackendError", "DistNetworkError", "DistError") for _, outcome in res), res
+    assert time.time() - t0 < 120
