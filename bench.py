@@ -5,7 +5,8 @@
 
 One step = one whole forward of the layer (route, permute + quantise, gate/up
 GEMM + SwiGLU + quantise, down GEMM, combine) over one batch of T tokens
-whose inputs already sit in HBM, timed through moe_layer_forward; a second
+whose inputs already sit in HBM, timed through moe_layer_forward (one call
+captured in a CUDA graph, replayed once per step); a second
 timed pass calls the stages one by one with CUDA events between them for the
 per-stage times and the kernel rooflines. With N > 1 (torchrun, one rank per GPU) every
 rank runs an independent replica of the layer on its own batch: the layer has
@@ -335,15 +336,28 @@ def time_stages(st: Stages, steps: int, warmup: int, d: Dist, sampler=None):
 
 
 def time_forward(st: Stages, steps: int, warmup: int, d: Dist, sampler=None):
-    """The whole forward as a user calls it: one moe_layer_forward per step
-    (its kernels chained by programmatic dependent launch, no event between
-    them), CUDA events on the launching stream around the timed steps. The
+    """The whole forward as a serving loop runs it: one moe_layer_forward
+    captured once in a CUDA graph (its kernels chained by programmatic
+    dependent launch, no event between them) and replayed once per step,
+    CUDA events on the launching stream around the timed steps. The
     per-stage breakdown comes from time_stages, whose events between the
     stages break that chaining."""
     import torch
     fx, dev, T, H = st.fx, st.dev, st.T, st.sh.H
-    for _ in range(warmup):
+
+    def fwd():
         fx.moe_layer_forward(dev, st.x, T, H, st.out, H, st.ws, st.ws.numel())
+
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        fwd()
+    torch.cuda.current_stream().wait_stream(side)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        fwd()
+    for _ in range(warmup):
+        graph.replay()
     torch.cuda.synchronize()
     d.barrier()
     torch.cuda.synchronize()
@@ -352,12 +366,13 @@ def time_forward(st: Stages, steps: int, warmup: int, d: Dist, sampler=None):
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record()
     for _ in range(steps):
-        fx.moe_layer_forward(dev, st.x, T, H, st.out, H, st.ws, st.ws.numel())
+        graph.replay()
     b.record()
     torch.cuda.synchronize()
     clocks = sampler.stop() if sampler else None
     d.barrier()
     torch.cuda.synchronize()
+    del graph
     code, bits = fx.moe_get_device_status(dev)
     if code != 0:
         raise RuntimeError(f"device status {bits:#x}")
@@ -578,6 +593,7 @@ def run_ours(args):
         # the library's own count for one forward (route 2, permute 2 or 4,
         # gate/up 1, down 1 or 2, combine 1)
         "gpu_launches": st.fx.moe_kernels_per_forward(dev, T) * args.steps,
+        "launch": "one moe_layer_forward captured in a CUDA graph, replayed once per step",
         "clocks": clocks,
     }
     del st
