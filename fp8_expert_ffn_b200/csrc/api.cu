@@ -455,6 +455,21 @@ moe_status moe_test_grouped_gemm_f32(moe_layer_t L, int which, const uint8_t* a,
 
 static_assert(sizeof(cudaIpcMemHandle_t) == MOE_EP_HANDLE_BYTES, "IPC handle size");
 
+// Makes the comm's device current for the scope of a call (IPC mappings and
+// the tables belong to it) and restores the caller's device.
+struct DeviceScope {
+  int prev = -1;
+  bool ok = false;
+  explicit DeviceScope(int dev) {
+    if (cudaGetDevice(&prev) != cudaSuccess) return;
+    ok = prev == dev || cudaSetDevice(dev) == cudaSuccess;
+  }
+  ~DeviceScope() {
+    int cur = -1;
+    if (prev >= 0 && cudaGetDevice(&cur) == cudaSuccess && cur != prev) cudaSetDevice(prev);
+  }
+};
+
 static moe_status ep_upload_tables(moe_ep_comm_s* c, const uint64_t* q, const uint64_t* s, const uint64_t* y) {
   uint64_t tab[3 * kEpMaxRanks];
   for (int i = 0; i < c->ranks; ++i) {
@@ -515,6 +530,8 @@ moe_status moe_ep_comm_create(moe_layer_t L, int rank, int ranks, int capacity, 
 
 moe_status moe_ep_comm_export(moe_ep_comm_t c, unsigned char handle[MOE_EP_HANDLE_BYTES]) {
   if (!c || !handle) return MOE_ERR_INVALID_ARG;
+  DeviceScope scope(c->device);
+  if (!scope.ok) return MOE_ERR_CUDA;
   cudaIpcMemHandle_t h;
   if (cudaIpcGetMemHandle(&h, c->base) != cudaSuccess) return MOE_ERR_CUDA;
   std::memcpy(handle, &h, sizeof(h));
@@ -531,6 +548,8 @@ static void ep_close_opened(moe_ep_comm_s* c) {
 
 moe_status moe_ep_comm_connect(moe_ep_comm_t c, const unsigned char* handles) {
   if (!c || !handles || c->connected) return MOE_ERR_INVALID_ARG;
+  DeviceScope scope(c->device);
+  if (!scope.ok) return MOE_ERR_CUDA;
   uint64_t q[kEpMaxRanks] = {}, sc[kEpMaxRanks] = {}, y[kEpMaxRanks] = {};
   for (int i = 0; i < c->ranks; ++i) {
     if (i == c->rank) {
@@ -585,7 +604,8 @@ moe_status moe_ep_comm_buffers(moe_ep_comm_t c, uint8_t** recv_q, float** recv_s
 
 moe_status moe_ep_comm_destroy(moe_ep_comm_t c) {
   if (!c) return MOE_OK;
-  moe_status st = from_cuda(cudaDeviceSynchronize());
+  DeviceScope scope(c->device);
+  moe_status st = scope.ok ? from_cuda(cudaDeviceSynchronize()) : MOE_ERR_CUDA;
   ep_close_opened(c);
   if (cudaFree(c->d_peer_q) != cudaSuccess) st = MOE_ERR_CUDA;
   if (cudaFree(c->base) != cudaSuccess) st = MOE_ERR_CUDA;
