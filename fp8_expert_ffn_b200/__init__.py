@@ -12,7 +12,9 @@ import os
 from dataclasses import dataclass
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libfp8moe.so")
+# FP8MOE_CHECKED=1 selects the bounds-checked build (-DMOE_CHECKS)
+CHECKED = os.environ.get("FP8MOE_CHECKED", "") == "1"
+LIB_PATH = os.path.join(HERE, "libfp8moe_checked.so" if CHECKED else "libfp8moe.so")
 
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_MISALIGNED, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, \
     MOE_ERR_DEVICE = range(7)
@@ -60,8 +62,8 @@ def lib(build_if_missing: bool = True):
         return _lib
     if build_if_missing:
         from . import build as _build
-        if _build.stale():
-            _build.build()
+        if _build.stale(CHECKED):
+            _build.build(checked=CHECKED)
     if not os.path.exists(LIB_PATH):
         raise RuntimeError(f"fp8_expert_ffn_b200: CUDA library not built ({LIB_PATH})")
     L = ctypes.CDLL(LIB_PATH)

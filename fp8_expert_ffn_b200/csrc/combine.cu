@@ -30,6 +30,8 @@ struct CombineArgs {
   const uint64_t* peer_y;  // [ranks] rows [cap][H] bf16
   const int32_t* goff;     // [El+2] this rank's group offsets: its shared rows start at goff[El]
   int rank, El;
+  int rows_limit;          // rows of each y buffer (bounds-checked build)
+  uint32_t* status;
 };
 
 // CTA (token, chunk of CB_THREADS*8 channels); each thread owns one
@@ -44,7 +46,13 @@ __global__ void __launch_bounds__(CB_THREADS) combine_kernel(const CombineArgs a
   __shared__ const uint16_t* s_src[9];
   __shared__ float s_w[9];
   if (threadIdx.x < K) {
-    const int r = a.inv[size_t(t) * K + threadIdx.x];
+    int r = a.inv[size_t(t) * K + threadIdx.x];
+#ifdef MOE_CHECKS
+    if (r >= a.rows_limit) {
+      set_status(a.status, STATUS_BOUNDS);
+      r = -1;
+    }
+#endif
     const uint16_t* src = nullptr;
     if (r >= 0) {
       const uint16_t* ybase = EP ? reinterpret_cast<const uint16_t*>(a.peer_y[a.idx[size_t(t) * K + threadIdx.x] / a.El])
@@ -61,7 +69,14 @@ __global__ void __launch_bounds__(CB_THREADS) combine_kernel(const CombineArgs a
       // this rank's shared rows are [goff[El], goff[El+1]) of its own buffer
       // (both 0 after an overflow: then nothing is read)
       const int row = a.goff[a.El] + t;
-      if (row < a.goff[a.El + 1]) src = reinterpret_cast<const uint16_t*>(a.peer_y[a.rank]) + size_t(row) * H;
+      bool ok = row < a.goff[a.El + 1];
+#ifdef MOE_CHECKS
+      if (ok && (row < 0 || row >= a.rows_limit)) {
+        set_status(a.status, STATUS_BOUNDS);
+        ok = false;
+      }
+#endif
+      if (ok) src = reinterpret_cast<const uint16_t*>(a.peer_y[a.rank]) + size_t(row) * H;
     }
     s_src[K] = src;
   }
@@ -114,6 +129,8 @@ cudaError_t launch_combine(const moe_layer_s* L, const uint16_t* y, const int32_
   a.H = L->H;
   a.out = out;
   a.ldo = ldo;
+  a.rows_limit = T * (L->K + L->S);
+  a.status = L->status;
   dim3 grid(T, (L->H + CB_THREADS * 8 - 1) / (CB_THREADS * 8));
   return launch_pdl(combine_kernel<false>, grid, dim3(CB_THREADS), 0, st, a);
 }
@@ -134,6 +151,8 @@ cudaError_t launch_ep_combine(const moe_layer_s* L, const moe_ep_comm_s* c, cons
   a.goff = goff;
   a.rank = c->rank;
   a.El = L->E / c->ranks;
+  a.rows_limit = c->cap;
+  a.status = L->status;
   dim3 grid(T, (L->H + CB_THREADS * 8 - 1) / (CB_THREADS * 8));
   return launch_pdl(combine_kernel<true>, grid, dim3(CB_THREADS), 0, st, a);
 }

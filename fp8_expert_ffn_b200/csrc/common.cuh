@@ -16,6 +16,7 @@ enum : uint32_t {
   STATUS_WAIT_TIMEOUT = 1u << 2,   // a pipeline wait exceeded its time limit
   STATUS_BAD_PLAN = 1u << 3,       // tile plan inconsistent with offsets
   STATUS_EP_OVERFLOW = 1u << 4,    // an expert-parallel owner's rows exceed its buffer
+  STATUS_BOUNDS = 1u << 5,         // (checked build) an input index fell outside its buffer
 };
 
 // Upper bound on any single pipeline wait before the kernel gives up.

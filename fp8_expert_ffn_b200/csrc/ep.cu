@@ -109,7 +109,7 @@ __global__ void __launch_bounds__(EP_THREADS) ep_regroup_kernel(
     const int32_t* __restrict__ cnt, int P, int El, int N, const uint8_t* __restrict__ recv_q,
     const float* __restrict__ recv_s, const uint8_t* __restrict__ own_q, const float* __restrict__ own_s,
     int own_rows, int R, int T_shared, int H, int HB, uint8_t* __restrict__ out_q, float* __restrict__ out_s,
-    int32_t* __restrict__ out_offsets) {
+    int32_t* __restrict__ out_offsets, uint32_t* status) {
   pdl_wait();
   pdl_launch_dependents();
   __shared__ int s_in[EP_SCAN], s_out[EP_SCAN + 1], s_w[EP_THREADS / 32];
@@ -131,6 +131,12 @@ __global__ void __launch_bounds__(EP_THREADS) ep_regroup_kernel(
       const int k = seg_of(s_out, n, o);
       const int e = k / P, s = k - e * P;
       const int in = s_in[s * El + e] + (o - s_out[k]);
+#ifdef MOE_CHECKS
+      if (in < 0 || in >= N) {   // counts that do not describe the received rows
+        if (lane == 0) set_status(status, STATUS_BOUNDS);
+        continue;
+      }
+#endif
       src_q = recv_q + size_t(in) * H;
       src_s = recv_s + size_t(in) * HB;
       src_stride_s = 1;
@@ -150,7 +156,7 @@ __global__ void __launch_bounds__(EP_THREADS) ep_regroup_kernel(
 __global__ void __launch_bounds__(EP_THREADS) ep_unregroup_kernel(const int32_t* __restrict__ cnt, int P, int El,
                                                                   int N, const uint16_t* __restrict__ y_g, int R,
                                                                   int T_shared, int H, uint16_t* __restrict__ y_send,
-                                                                  uint16_t* __restrict__ y_own) {
+                                                                  uint16_t* __restrict__ y_own, uint32_t* status) {
   pdl_wait();
   pdl_launch_dependents();
   __shared__ int s_in[EP_SCAN], s_out[EP_SCAN + 1], s_w[EP_THREADS / 32];
@@ -164,7 +170,14 @@ __global__ void __launch_bounds__(EP_THREADS) ep_unregroup_kernel(const int32_t*
     if (o < N) {
       const int k = seg_of(s_out, n, o);
       const int e = k / P, s = k - e * P;
-      dst = y_send + size_t(s_in[s * El + e] + (o - s_out[k])) * H;
+      const int in = s_in[s * El + e] + (o - s_out[k]);
+#ifdef MOE_CHECKS
+      if (in < 0 || in >= N) {
+        if (lane == 0) set_status(status, STATUS_BOUNDS);
+        continue;
+      }
+#endif
+      dst = y_send + size_t(in) * H;
     } else {
       dst = y_own + size_t(R + (o - N)) * H;
     }
@@ -193,14 +206,15 @@ cudaError_t launch_ep_regroup(const moe_layer_s* L, int P, const int32_t* cnt, i
                               float* out_s, int32_t* out_offsets, cudaStream_t st) {
   const int Ts = T * L->S;
   return launch_pdl(ep_regroup_kernel, dim3(ep_grid(N + Ts)), dim3(EP_THREADS), 0, st, cnt, P, L->E, N, recv_q,
-                    recv_s, own_q, own_s, T * (L->K + L->S), T * L->K, Ts, L->H, L->HB, out_q, out_s, out_offsets);
+                    recv_s, own_q, own_s, T * (L->K + L->S), T * L->K, Ts, L->H, L->HB, out_q, out_s, out_offsets,
+                    L->status);
 }
 
 cudaError_t launch_ep_unregroup(const moe_layer_s* L, int P, const int32_t* cnt, int N, const uint16_t* y_g, int T,
                                 uint16_t* y_send, uint16_t* y_own, cudaStream_t st) {
   const int Ts = T * L->S;
   return launch_pdl(ep_unregroup_kernel, dim3(ep_grid(N + Ts)), dim3(EP_THREADS), 0, st, cnt, P, L->E, N, y_g,
-                    T * L->K, Ts, L->H, y_send, y_own);
+                    T * L->K, Ts, L->H, y_send, y_own, L->status);
 }
 
 }  // namespace moe

@@ -344,6 +344,12 @@ __global__ void __launch_bounds__(GATHER_THREADS, 4) gather_rows_kernel(const Ga
       const int within = int(a.wprefix[size_t(e) * W + (t >> 5)]) + __popc(word & ((1u << (t & 31)) - 1u));
       if (MODE == GATHER_LOCAL) {
         row = a.offsets[e] + within;
+#ifdef MOE_CHECKS
+        if (row < 0 || row >= a.rows) {
+          set_status(a.status, STATUS_BOUNDS);
+          row = -1;
+        }
+#endif
         my_row = row;
       } else if (within < a.all_off[a.rank * (E + 2) + e + 1] - a.all_off[a.rank * (E + 2) + e]) {
         // (a row beyond this rank's own count in all_offsets is not this
@@ -365,7 +371,13 @@ __global__ void __launch_bounds__(GATHER_THREADS, 4) gather_rows_kernel(const Ga
   } else if (lane == K && a.S) {
     if (MODE == GATHER_LOCAL) {
       my_row = a.offsets[E] + t;
-      if (chunk == 0) a.perm[my_row] = t;
+#ifdef MOE_CHECKS
+      if (my_row < 0 || my_row >= a.rows) {
+        set_status(a.status, STATUS_BOUNDS);
+        my_row = -1;
+      }
+#endif
+      if (chunk == 0 && my_row >= 0) a.perm[my_row] = t;
     } else if (!over) {
       if (t < a.all_off[a.rank * (E + 2) + E + 1] - a.all_off[a.rank * (E + 2) + E])
         my_row = (s_nr + t) | (a.rank << 24);
@@ -493,6 +505,7 @@ cudaError_t launch_permute(const moe_layer_s* L, const uint16_t* x, int T, int l
   a.inv = inv;
   a.xq = xq;
   a.xs = xs;
+  a.status = L->status;
   const int nchunk = (L->HB + GATHER_GROUPS - 1) / GATHER_GROUPS;
   const long long warps = static_cast<long long>(T) * nchunk;
   const int wpc = GATHER_THREADS / 32;

@@ -418,6 +418,9 @@ moe_status moe_layer_forward(moe_layer_t layer, const uint16_t* x, int T, int ld
 #define MOE_STATUS_WAIT_TIMEOUT 0x4u /* a pipeline wait gave up; that launch's outputs are incomplete */
 #define MOE_STATUS_BAD_PLAN 0x8u     /* group offsets not ascending within [0, rows]; no GEMM work done */
 #define MOE_STATUS_EP_OVERFLOW 0x10u /* an owner's rows exceed its exchange buffer; nothing dispatched */
+#define MOE_STATUS_BOUNDS 0x20u      /* bounds-checked build only: a row index taken from the inputs
+                                      (inv, offsets, segment counts) fell outside its buffer; the
+                                      access was skipped */
 
 /* Synchronises `stream`, returns MOE_ERR_DEVICE if any kernel of this layer
  * flagged an error since the last call (and clears the flag), else MOE_OK.
