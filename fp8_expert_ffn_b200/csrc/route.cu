@@ -304,9 +304,20 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const TopkArgs a) {
   for (int j = 0; j < 8; ++j) l[j] = 0.0f;
   const float* pt = a.partial + size_t(t) * E + lane;
   const size_t ps = size_t(a.T) * E;
-  // four split slices in flight at a time; the sum stays in split order
+  // eight split slices in flight at a time; the sum stays in split order
   int s = 0;
-  for (; s + 4 <= a.S; s += 4) {
+  for (; s + 8 <= a.S; s += 8) {
+    float v[8][8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[u][j] = (lane + 32 * j < E) ? __ldg(pt + (s + u) * ps + 32 * j) : 0.0f;
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+#pragma unroll
+      for (int j = 0; j < 8; ++j) l[j] += v[u][j];
+  }
+  if (s + 4 <= a.S) {
     float v[4][8];
 #pragma unroll
     for (int u = 0; u < 4; ++u)
@@ -316,6 +327,7 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const TopkArgs a) {
     for (int u = 0; u < 4; ++u)
 #pragma unroll
       for (int j = 0; j < 8; ++j) l[j] += v[u][j];
+    s += 4;
   }
   for (; s < a.S; ++s) {
     float v[8];
