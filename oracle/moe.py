@@ -338,11 +338,15 @@ def layer_forward(x_bits: np.ndarray, layer) -> dict:
     return {"route": r, "perm": p, "xq": xq, "xs": xs, **f, "out": out}
 
 
-def token_outputs(x_bits: np.ndarray, layer, tokens, idx=None, w=None) -> np.ndarray:
+def token_outputs(x_bits: np.ndarray, layer, tokens, idx=None, w=None, y_bf16: bool = False) -> np.ndarray:
     """Direct per-token evaluation (no permutation) for a subset of tokens:
     out[t] = sum_k w_k FFN_{e_k}(x_t) + FFN_shared(x_t). Routing is the
     oracle's unless idx/w (full [T, K] tables) are given. Each expert is
-    dequantised once for all the sampled tokens that use it."""
+    dequantised once for all the sampled tokens that use it. With y_bf16,
+    each expert's output row is rounded to bf16 before it is weighted: the
+    layer keeps the down projection's output y as a bf16 tensor (the model's
+    activation dtype) and the combine sums those rows; everything else
+    stays FP64."""
     sh = layer.shape
     tokens = np.asarray(tokens)
     xb = np.asarray(x_bits)[tokens]
@@ -368,6 +372,8 @@ def token_outputs(x_bits: np.ndarray, layer, tokens, idx=None, w=None) -> np.nda
         hg = expert_gate_up(a[rows], layer.w_gate[g], layer.s_gate[g], layer.w_up[g], layer.s_up[g], sh.F, sh.H)
         q, s = quantize_rows(hg.astype(np.float32))
         yg = expert_down(dequant_rows(q, s, sh.F), layer.w_down[g], layer.s_down[g], sh.H, sh.F)
+        if y_bf16:
+            yg = f64_to_bf16_f64(yg)
         return rows, wt[:, None] * yg
 
     for rows, contrib in _pool_map(one, sorted(users.items())):

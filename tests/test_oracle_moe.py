@@ -311,6 +311,20 @@ def test_permuted_path_equals_direct_per_token(O, toy):
     assert np.max(np.abs(d - r["out"])) <= 1e-12 * np.max(np.abs(r["out"]))
 
 
+def test_direct_path_with_bf16_expert_rows_equals_combine_of_rounded_y(toy):
+    """token_outputs(y_bf16=True) rounds each expert's output row to bf16
+    before weighting it: equal to the permuted path's combine applied to the
+    bf16-rounded y rows (the pinned f64 -> bf16 rounding), and different
+    from the unrounded sum."""
+    from oracle import moe
+    _, layer, x = toy
+    r = moe.layer_forward(x, layer)
+    want = moe.combine(moe.f64_to_bf16_f64(r["y"]), r["perm"].inv, r["route"].w, layer.shape.S)
+    got = moe.token_outputs(x, layer, np.arange(x.shape[0]), y_bf16=True)
+    assert np.max(np.abs(got - want)) <= 1e-12 * np.max(np.abs(want))
+    assert np.max(np.abs(got - r["out"])) > 1e-6 * np.max(np.abs(want))
+
+
 def test_partial_blocks_equal_zero_padded_layer(O):
     """F=250 (not a multiple of 128) equals the same layer zero-padded to F=256."""
     layer, sh = small_layer(H=256, E=4, K=2, F=250, ld_f=256, seed=11)
