@@ -312,3 +312,32 @@ def test_peer_dispatch_inconsistent_offsets_flag_bad_plan(case):
             assert fx.moe_get_device_status(h)[0] == fx.MOE_OK
     for c in comms:
         c.close()
+
+
+def test_peer_dispatch_zipf_skewed_routing_four_ranks():
+    """The Zipf-biased router of the long prefill (the hottest expert about
+    ten times the mean load, some experts empty), 1024 tokens on each of 4
+    ranks: the owners of the hot experts receive far more rows than the
+    others, all within the default capacity."""
+    wl, layer, _ = gen.workload_inputs("zipf")
+    xs = [gen.make_x(1024, layer.shape.H, 700 + r, outliers=wl.outliers, zipf=True) for r in range(4)]
+    _run_peer("zipf", 4, None, xs=xs)
+
+
+@pytest.mark.parametrize("transport", ["peer", "all_to_all"])
+def test_expert_parallel_router_variants(transport):
+    """Group-limited top-k, a selection-only bias, norm_topk_prob off and
+    routed_scaling 2 on the toy layer: the routing-only handle of every rank
+    carries the layer's router settings (ep.rank_layers), so each rank's
+    output stays bit-identical to the single-GPU forward."""
+    wl, layer0, _ = gen.workload_inputs("toy")
+    sh = layer0.shape
+    layer = gen.Layer(sh, layer0.router_w, layer0.w_gate, layer0.s_gate, layer0.w_up, layer0.s_up,
+                      layer0.w_down, layer0.s_down)
+    layer.n_group, layer.topk_group, layer.norm_topk, layer.routed_scaling = 8, 3, False, 2.0
+    layer.router_bias = np.random.default_rng(31).normal(0, 1.0 / sh.E, sh.E).astype(np.float32)
+    xs = [gen.make_x(256, sh.H, 800 + r, outliers=2) for r in range(2)]
+    if transport == "peer":
+        _run_peer("toy", 2, None, layer=layer, xs=xs)
+    else:
+        _run("toy", 2, 256, layer=layer, xs=xs)
