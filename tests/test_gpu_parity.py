@@ -725,3 +725,29 @@ def test_inconsistent_offsets_set_bad_plan_and_do_no_work():
         assert bool((h == 0x5A).all()) and bool((hs == 7.0).all())
     fx.moe_gate_up(c.dev, c.xq, c.xs, c.offsets, T, h, hs)
     assert fx.moe_get_device_status(c.dev) == (fx.MOE_OK, 0)
+
+
+def test_strided_activations_outputs_and_weight_rows():
+    """Row strides beyond the hidden size: x read from a [T][H+128] buffer,
+    the output written into a [T][H+64] buffer (its pad left untouched), and
+    gate/up weight rows stored with a padded stride ld_h = H + 128. The
+    result equals the contiguous forward bit for bit."""
+    wl, layer, c = get_case("toy")
+    sh, T = layer.shape, c.T
+    x_wide = torch.zeros((T, sh.H + 128), dtype=torch.bfloat16, device="cuda")
+    x_wide[:, :sh.H] = c.x
+    out_wide = torch.full((T, sh.H + 64), 7.0, dtype=torch.bfloat16, device="cuda")
+    ws = tu.workspace(c.dev, T)
+    fx.moe_layer_forward(c.dev, x_wide, T, sh.H + 128, out_wide, sh.H + 64, ws, ws.numel())
+    assert torch.equal(out_wide[:, :sh.H].contiguous().view(torch.int16), c.out.view(torch.int16))
+    assert bool((out_wide[:, sh.H:] == 7.0).all())
+    # gate/up rows with a padded stride (pad bytes hold garbage that must not be read)
+    w = c.dev.weights
+    pad = lambda t: torch.cat([t, torch.full(t.shape[:2] + (128,), 0x7E, dtype=t.dtype, device=t.device)], 2)
+    lw = fx.LayerWeights(pad(w.w_gate), pad(w.w_up), w.w_down, w.s_gate, w.s_up, w.s_down, w.router_w)
+    wide = fx.MoeLayer(sh.H, sh.E, sh.K, sh.F, lw, ld_h=sh.H + 128, ld_f=sh.ld_f, n_shared=sh.S)
+    o2 = torch.empty_like(c.out)
+    ws2 = tu.workspace(wide, T)
+    fx.moe_layer_forward(wide, c.x, T, sh.H, o2, sh.H, ws2, ws2.numel())
+    assert fx.moe_get_device_status(wide)[0] == fx.MOE_OK
+    assert torch.equal(o2.view(torch.int16), c.out.view(torch.int16))
