@@ -622,6 +622,9 @@ def run_ours(args):
         wls["toy"] = {"workload": "toy: T=32, hidden 512, 16+1 experts, top-4, FFN 256",
                       "purpose": "parity only (every value checked against the oracle), not timed"}
         line["workloads"] = wls
+        wl_d, _, dev_d, xb_d = load_layer("decode", d, rank)
+        line["expert_parallel_one_rank"] = measure_ep_one_rank(dev_d, wl_d.shape, wl_d.T, tu.bf16_tensor(xb_d),
+                                                               max(10, args.steps), max(3, min(args.warmup, 5)), d)
         line["peaks"] = {"hbm_gbs": pk["hbm_gbs"], "fp8_tflops_burst": round(fp8, 1),
                          "fp8_tflops_sustained": round(FP8_OVER_BF16 * pk["bf16_tflops_sustained"], 1),
                          "source": f"{pk['source']}: HBM copy; FP8 = {FP8_OVER_BF16} x BF16 GEMM (nominal ratio)"}
@@ -737,6 +740,56 @@ def run_ep(args):
         comm.close()          # every rank is past its last read of the peers' buffers
     del ops, route, experts
     d.close()
+
+
+class OneRankSync:
+    """The peer-memory forward's collectives for a single rank: the
+    all-gather is the rank's own offsets and there is nothing to wait for."""
+
+    def all_gather(self, off):
+        return off.unsqueeze(0)
+
+    def barrier(self):
+        pass
+
+
+def measure_ep_one_rank(dev, sh, T, x, steps, warmup, d: Dist):
+    """The expert-parallel forward over peer memory with one rank (every
+    expert local, the exchange buffer its own): what its kernels cost over
+    the fused forward, with the per-phase breakdown. Checked bit for bit
+    against the fused forward."""
+    import torch
+    import fp8_expert_ffn_b200 as fx
+    from fp8_expert_ffn_b200 import ep
+    from fp8_expert_ffn_b200 import torch_utils as tu
+    ref = torch.empty((T, sh.H), dtype=torch.bfloat16, device="cuda")
+    ws = tu.workspace(dev, T)
+    fx.moe_layer_forward(dev, x, T, sh.H, ref, sh.H, ws, ws.numel())
+    route, experts = ep.rank_layers(dev, 0, 1)
+    comm = fx.EpComm(route, 0, 1, ep.peer_capacity(T, sh.K, sh.S, 1))
+    ops, sync = ep.PeerOps(route, experts, comm, 1), OneRankSync()
+    for _ in range(warmup):
+        out = ep.ep_forward_peer(ops, sync, x, T)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        out = ep.ep_forward_peer(ops, sync, x, T)
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / steps
+    same = torch.equal(out.view(torch.int16), ref.view(torch.int16))
+    stages = ep_peer_stages(ops, sync, x, T, steps, d, sh, 1)
+    for h in (route, experts):
+        code, bits = fx.moe_get_device_status(h)
+        if code != fx.MOE_OK:
+            raise RuntimeError(f"device status {bits:#x}")
+    if not same:
+        raise RuntimeError("expert-parallel forward differs from the fused forward")
+    comm.close()
+    return {"ranks": 1, "transport": "dispatch/combine kernels over peer memory (one rank: its own buffer)",
+            "ms_per_step": round(ms, 5), "tokens_per_s": round(T / (ms / 1e3), 1), "stages": stages,
+            "parity": "bit-identical to the fused forward"}
 
 
 EP_STAGES = ("route_plan", "all_gather", "dispatch", "barrier_1", "experts", "barrier_2", "combine")
