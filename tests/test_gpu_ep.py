@@ -341,3 +341,44 @@ def test_expert_parallel_router_variants(transport):
         _run_peer("toy", 2, None, layer=layer, xs=xs)
     else:
         _run("toy", 2, 256, layer=layer, xs=xs)
+
+
+class _OneRank:
+    def all_gather(self, off):
+        return off.unsqueeze(0)
+
+    def barrier(self):
+        pass
+
+
+def test_peer_forward_has_no_host_sync_and_replays_in_a_graph():
+    """The peer-memory forward of one rank reads nothing back to the host: it
+    captures into a CUDA graph (a host read would break the capture), and
+    replays give the fused forward's bytes for new inputs."""
+    wl, layer, _ = gen.workload_inputs("toy")
+    sh, T = layer.shape, 256
+    dev = tu.upload_layer(layer)
+    route, experts = ep.rank_layers(dev, 0, 1)
+    comm = fx.EpComm(route, 0, 1, ep.peer_capacity(T, sh.K, sh.S, 1))
+    ops, sync = ep.PeerOps(route, experts, comm, 1), _OneRank()
+    x = tu.bf16_tensor(gen.make_x(T, sh.H, 900, outliers=2))
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        ep.ep_forward_peer(ops, sync, x, T)          # buffers allocated outside the capture
+    torch.cuda.current_stream().wait_stream(side)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        out = ep.ep_forward_peer(ops, sync, x, T)
+    ref = torch.empty_like(out)
+    ws = tu.workspace(dev, T)
+    for seed in (901, 902):
+        x.copy_(tu.bf16_tensor(gen.make_x(T, sh.H, seed, outliers=2)))
+        g.replay()
+        fx.moe_layer_forward(dev, x, T, sh.H, ref, sh.H, ws, ws.numel())
+        torch.cuda.synchronize()
+        assert torch.equal(out.view(torch.int16), ref.view(torch.int16))
+    for h in (route, experts):
+        assert fx.moe_get_device_status(h)[0] == fx.MOE_OK
+    del g
+    comm.close()
