@@ -680,11 +680,7 @@ def run_ep(args):
     route, experts = ep.rank_layers(dev, rank, world)
     comm = None
     if args.ep_transport == "peer":
-        comm = fx.EpComm(route, rank, world, ep.peer_capacity(T, sh.K, sh.S, world))
-        if world > 1:
-            handles = [None] * world
-            d.dist.all_gather_object(handles, comm.export())
-            comm.connect(handles)
+        comm = ep.connect_peers(fx.EpComm(route, rank, world, ep.peer_capacity(T, sh.K, sh.S, world)))
         ops, ex = ep.PeerOps(route, experts, comm, world), ep.TorchSync()
         step = lambda: ep.ep_forward_peer(ops, ex, x, T)
     else:

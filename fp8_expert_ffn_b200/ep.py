@@ -300,6 +300,22 @@ class TorchSync:
         self.dist.all_reduce(self.word, group=self.group)
 
 
+def connect_peers(comm, group=None):
+    """Maps every other rank's exchange buffers into this one (EpComm):
+    the ranks swap their buffer handles with torch.distributed (any backend)
+    and each opens the others'. Call on every rank of the group together."""
+    import torch.distributed as dist
+    ranks = dist.get_world_size(group)
+    if ranks != comm.ranks or dist.get_rank(group) != comm.rank:
+        raise ValueError("the comm's rank and ranks must be this process's in the group")
+    if ranks == 1:
+        return comm
+    handles = [None] * ranks
+    dist.all_gather_object(handles, comm.export(), group=group)
+    comm.connect(handles)
+    return comm
+
+
 def peer_capacity(tokens_per_rank: int, K: int, S: int, ranks: int) -> int:
     """Receive rows that always suffice: every rank's routed rows going to
     one owner, plus that owner's shared rows."""

@@ -69,10 +69,7 @@ def _worker(rank, world, port, T, q):
         ws = tu.workspace(dev, T)
         fx.moe_layer_forward(dev, x, T, sh.H, ref, sh.H, ws, ws.numel())
         route, experts = ep.rank_layers(dev, rank, world)
-        comm = fx.EpComm(route, rank, world, ep.peer_capacity(T, sh.K, sh.S, world))
-        handles = [None] * world
-        dist.all_gather_object(handles, comm.export())
-        comm.connect(handles)
+        comm = ep.connect_peers(fx.EpComm(route, rank, world, ep.peer_capacity(T, sh.K, sh.S, world)))
         sync = HostSync(dist)
         ops = ep.PeerOps(route, experts, comm, world)
         outs = [ep.ep_forward_peer(ops, sync, x, T) for _ in range(2)]   # twice: buffers reused
