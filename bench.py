@@ -501,6 +501,21 @@ def fractions(work, per, total_ms, pk):
     return out
 
 
+def count_near_ties(st: Stages) -> int:
+    """Tokens whose K-th and (K+1)-th routing probabilities (softmax of the
+    library's FP32 logits, taken in FP64) are less than 1e-6 apart: the
+    tokens whose choice of experts rounding may decide."""
+    import torch
+    sh, T = st.sh, st.T
+    if sh.K >= sh.E:
+        return 0
+    logits = torch.empty((T, sh.E), dtype=torch.float32, device="cuda")
+    st.fx.moe_route(st.dev, st.x, T, sh.H, st.idx, st.w, logits, st.ws, st.ws.numel())
+    p = torch.softmax(logits.double(), dim=1)
+    top = torch.topk(p, sh.K + 1, dim=1).values
+    return int((top[:, sh.K - 1] - top[:, sh.K] < 1e-6).sum().item())
+
+
 def measure_workload(name, d, rank, args, pk, sampler, oracle=True):
     """One workload: its stages timed over the same number of steps as the
     headline (at least 10; a timed region of 0.01-0.15 s, like the burst
@@ -517,13 +532,14 @@ def measure_workload(name, d, rank, args, pk, sampler, oracle=True):
     off = st.offsets.cpu().numpy()
     work = algorithmic_work(wl, wl.T, off)
     counts = np.diff(off)[:wl.shape.E]
+    near_ties = count_near_ties(st)
     entry = {"workload": f"{wl.name}: {wl.note}", "T": wl.T, "steps": steps,
              "tokens_per_s": round(d.sum(float(wl.T * steps)) / (total_ms / 1e3), 1),
              "ms_per_step": round(total_ms / steps, 5), "stage_ms": {k: round(v, 5) for k, v in per.items()},
              "roofline": fractions(work, per, total_ms / steps, pk), "clocks": clocks,
              "touched_groups": work["touched_groups"],
              "load_max_over_mean": round(float(counts.max() / max(counts.mean(), 1e-9)), 2),
-             "empty_experts": int((counts == 0).sum())}
+             "empty_experts": int((counts == 0).sum()), "near_tie_tokens": near_ties}
     if oracle and rank == 0:
         n, dt = oracle_sample(host, x_bits)
         entry["oracle"] = {"tokens_per_s": round(n / dt, 3), "tokens": n, "seconds": round(dt, 2),
