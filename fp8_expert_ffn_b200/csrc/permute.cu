@@ -18,7 +18,8 @@
 //                       the last CTA to finish scans the counts -> offsets[E+2]
 //   (small batches: 1-3 in one CTA, permute_plan_small, when the bitmap fits
 //   in shared memory)
-//   4. gather_rows      one warp per token and 16 groups of 128 channels:
+//   4. gather_rows      one warp per token and 16 groups of 128 channels (4
+//                       for small batches):
 //                       rows of its K slots and its shared-expert row,
 //                       inv/perm, then the groups of x quantised once and
 //                       stored to all rows with 16-byte stores.
@@ -189,7 +190,12 @@ __global__ void __launch_bounds__(kPlanSmallThreads) permute_plan_small_kernel(
   }
 }
 
-constexpr int GATHER_GROUPS = 16;   // 128-channel groups per warp (4 steps of 4 groups)
+// 128-channel groups per warp (steps of 4 groups): 16 for large batches;
+// 4 while the batch is small (a decode batch of 64 tokens then spreads over
+// 640 warps instead of 192, and each warp's chain of loads is shorter)
+constexpr int GATHER_GROUPS_LARGE = 16;
+constexpr int GATHER_GROUPS_SMALL = 4;
+constexpr int kGatherSmallT = 512;
 constexpr int GATHER_THREADS = 256;
 
 enum GatherMode { GATHER_LOCAL = 0, GATHER_EP = 1 };
@@ -288,7 +294,7 @@ __device__ void ep_layout(const GatherArgs& a, int* s_base, int* s_excl, int* s_
 // perm); GATHER_EP writes each routed row into its expert's owner's receive
 // buffer (a peer's memory over NVLink; every store is a plain 16- or 4-byte
 // store, no bulk or tensor copy) and the shared row into this rank's own.
-template <int MODE>
+template <int MODE, int GATHER_GROUPS>
 __global__ void __launch_bounds__(GATHER_THREADS, 4) gather_rows_kernel(const GatherArgs a) {
   pdl_wait();
   pdl_launch_dependents();
@@ -308,9 +314,9 @@ __global__ void __launch_bounds__(GATHER_THREADS, 4) gather_rows_kernel(const Ga
   const int g0 = chunk * GATHER_GROUPS;
   // issue the x loads of the whole chunk before anything waits on memory
   // (with EP, before the layout is computed)
-  uint4 raw[4][2];
+  uint4 raw[GATHER_GROUPS / 4][2];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
+  for (int i = 0; i < GATHER_GROUPS / 4; ++i) {
     const int g = g0 + 4 * i + gs;
     if (has_token && g < HB) {
       const uint4* src = reinterpret_cast<const uint4*>(a.x + size_t(t) * a.ldx + g * 128 + gl * 16);
@@ -392,7 +398,7 @@ __global__ void __launch_bounds__(GATHER_THREADS, 4) gather_rows_kernel(const Ga
   const size_t sstride = MODE == GATHER_LOCAL ? size_t(a.rows) : size_t(a.cap);
 
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
+  for (int i = 0; i < GATHER_GROUPS / 4; ++i) {
     const int g = g0 + 4 * i + gs;
     const bool valid = g < HB;   // uniform over the 8 lanes of a group
     const uint32_t w32[8] = {raw[i][0].x, raw[i][0].y, raw[i][0].z, raw[i][0].w,
@@ -457,6 +463,20 @@ int permute_kernels(const moe_layer_s* L, int T) {
   return size_t(L->E) * ((T + 31) / 32) <= size_t(kPlanSmallWords) ? 2 : 4;
 }
 
+// One warp per (token, chunk of groups); at least one CTA (with EP it writes
+// the owner offsets even when this rank sends nothing).
+template <int MODE>
+static cudaError_t launch_gather(const GatherArgs& a, int HB, int T, cudaStream_t st) {
+  const bool small = T <= kGatherSmallT;
+  const int groups = small ? GATHER_GROUPS_SMALL : GATHER_GROUPS_LARGE;
+  const long long warps = static_cast<long long>(T) * ((HB + groups - 1) / groups);
+  const int wpc = GATHER_THREADS / 32;
+  const long long ctas = (warps + wpc - 1) / wpc;
+  const dim3 grid(unsigned(ctas > 0 ? ctas : 1));
+  if (small) return launch_pdl(gather_rows_kernel<MODE, GATHER_GROUPS_SMALL>, grid, dim3(GATHER_THREADS), 0, st, a);
+  return launch_pdl(gather_rows_kernel<MODE, GATHER_GROUPS_LARGE>, grid, dim3(GATHER_THREADS), 0, st, a);
+}
+
 // The plan of the permutation: the token bitmap and its per-word prefixes in
 // the scratch, the counts, and offsets[E+2].
 static cudaError_t launch_plan(const moe_layer_s* L, const int32_t* idx, int T, int32_t* offsets, const Scratch& s,
@@ -506,11 +526,7 @@ cudaError_t launch_permute(const moe_layer_s* L, const uint16_t* x, int T, int l
   a.xq = xq;
   a.xs = xs;
   a.status = L->status;
-  const int nchunk = (L->HB + GATHER_GROUPS - 1) / GATHER_GROUPS;
-  const long long warps = static_cast<long long>(T) * nchunk;
-  const int wpc = GATHER_THREADS / 32;
-  return launch_pdl(gather_rows_kernel<GATHER_LOCAL>, dim3(unsigned((warps + wpc - 1) / wpc)), dim3(GATHER_THREADS),
-                    0, st, a);
+  return launch_gather<GATHER_LOCAL>(a, L->HB, T, st);
 }
 
 cudaError_t launch_ep_plan(const moe_layer_s* L, const int32_t* idx, int T, int32_t* offsets, const Scratch& s,
@@ -543,13 +559,7 @@ cudaError_t launch_ep_dispatch(const moe_layer_s* L, const moe_ep_comm_s* c, con
   a.inv_ep = inv_ep;
   a.goff = goff;
   a.status = L->status;
-  const int nchunk = (L->HB + GATHER_GROUPS - 1) / GATHER_GROUPS;
-  const long long warps = static_cast<long long>(T) * nchunk;
-  const int wpc = GATHER_THREADS / 32;
-  const long long ctas = (warps + wpc - 1) / wpc;
-  // at least one CTA: it writes the owner offsets even when this rank sends nothing
-  return launch_pdl(gather_rows_kernel<GATHER_EP>, dim3(unsigned(ctas > 0 ? ctas : 1)), dim3(GATHER_THREADS), 0, st,
-                    a);
+  return launch_gather<GATHER_EP>(a, L->HB, T, st);
 }
 
 // ---------------------------------------------------------------------------
