@@ -363,8 +363,9 @@ moe_status moe_ep_comm_destroy(moe_ep_comm_t comm);
 
 /* Step 1 of the expert-parallel forward of the SGLang cookbook
  * "Dots3-Note" ("2. Configuration Tips"): the plan of the permutation of
- * this rank's T tokens (route handle): offsets [E+2] as moe_permute gives them (offsets[E] = T*K
- * routed rows, offsets[E+1] = offsets[E] + T*S), and the token bitmap and
+ * this rank's T tokens (route handle): offsets [E+2] as moe_permute gives
+ * them (offsets[E] = T*K routed rows, offsets[E+1] = offsets[E] + T*S),
+ * and the token bitmap and
  * its prefixes in `ws` (moe_workspace_size(route_layer, T) bytes), which
  * moe_ep_dispatch reads: pass it the same workspace, unchanged. T = 0 writes
  * zero offsets. */
@@ -372,8 +373,9 @@ moe_status moe_ep_plan(moe_layer_t route_layer, const int32_t* idx, int T, int32
                        size_t ws_bytes, void* stream);
 /* Step 3, the DeepEP "dispatch" of the SGLang cookbook "Dots3-Note"
  * ("2. Configuration Tips") (route handle; comm connected; route_layer
- * n_routed divisible by the comm's ranks): quantises x [T][ldx] bf16 per token per 128 channels
- * (as moe_permute) and writes routed row (t, k) into the buffer of expert
+ * n_routed divisible by the comm's ranks): quantises x [T][ldx] bf16 per
+ * token per 128 channels (as moe_permute) and writes routed row (t, k)
+ * into the buffer of expert
  * idx[t][k]'s owner and t's shared row into this rank's; inv_ep [T][K] =
  * the row in the owner's buffer (-1 for a skipped slot; the owner is
  * idx[t][k] / El); group_offsets [El+2] = this rank's offsets as an owner
