@@ -451,7 +451,7 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const TopkArgs a) {
 int route_splits(const moe_layer_s* L, int T) {
   const int nkb = L->H / RK;
   const int tiles = ((T + RM - 1) / RM) * ((L->E + RN - 1) / RN);
-  int s = (L->num_sms + tiles - 1) / tiles;
+  int s = L->num_sms / tiles;               // one wave: tiles * s <= SMs
   s = s > nkb / 4 ? nkb / 4 : s;          // at least 4 K blocks per split
   return s < 1 ? 1 : s;
 }
