@@ -641,6 +641,9 @@ def run_ours(args):
         wl_d, _, dev_d, xb_d = load_layer("decode", d, rank)
         line["expert_parallel_one_rank"] = measure_ep_one_rank(dev_d, wl_d.shape, wl_d.T, tu.bf16_tensor(xb_d),
                                                                max(10, args.steps), max(3, min(args.warmup, 5)), d)
+        # the serving recipe's shape: 8 ranks of 128 tokens, emulated on this GPU
+        line["expert_parallel_8_emulated"] = measure_ep_emulated(dev_d, wl_d.shape, wl_d, 8, 128,
+                                                                 max(10, args.steps), 3)
         line["peaks"] = {"hbm_gbs": pk["hbm_gbs"], "fp8_tflops_burst": round(fp8, 1),
                          "fp8_tflops_sustained": round(FP8_OVER_BF16 * pk["bf16_tflops_sustained"], 1),
                          "source": f"{pk['source']}: HBM copy; FP8 = {FP8_OVER_BF16} x BF16 GEMM (nominal ratio)"}
@@ -802,6 +805,85 @@ def measure_ep_one_rank(dev, sh, T, x, steps, warmup, d: Dist):
     return {"ranks": 1, "transport": "dispatch/combine kernels over peer memory (one rank: its own buffer)",
             "ms_per_step": round(ms, 5), "tokens_per_s": round(T / (ms / 1e3), 1), "stages": stages,
             "parity": "bit-identical to the fused forward"}
+
+
+def measure_ep_emulated(dev, sh, wl, ranks: int, T: int, steps: int, warmup: int):
+    """The expert-parallel forward over peer memory with `ranks` ranks
+    emulated on this one GPU (each rank's buffers in this GPU's memory, its
+    tokens its own seeded batch): every phase runs for all ranks in turn on
+    one stream, which orders the phases as the barriers would. Reports the
+    time of one forward of all ranks, each phase summed over the ranks, and
+    the owners' grouped-GEMM phase per rank against the weights it streams
+    (its E/ranks experts plus the shared one). Each rank's output is checked
+    bit for bit against the fused forward of the whole layer on its tokens.
+    No NVLink is involved, so the exchange is not what this measures."""
+    import torch
+    import gen
+    import fp8_expert_ffn_b200 as fx
+    from fp8_expert_ffn_b200 import ep
+    from fp8_expert_ffn_b200 import torch_utils as tu
+    layers = [ep.rank_layers(dev, r, ranks) for r in range(ranks)]
+    cap = ep.peer_capacity(T, sh.K, sh.S, ranks)
+    comms = [fx.EpComm(layers[r][0], r, ranks, cap) for r in range(ranks)]
+    fx.EpComm.connect_local(comms)
+    ops = [ep.PeerOps(layers[r][0], layers[r][1], comms[r], ranks) for r in range(ranks)]
+    xs = [tu.bf16_tensor(gen.make_x(T, sh.H, 5000 + r, wl.outliers, wl.zipf)) for r in range(ranks)]
+
+    def forward(ev=None):
+        plans = [ops[r].plan(xs[r], T) for r in range(ranks)]
+        if ev: ev[0].record()
+        all_off = torch.stack([off for _, off in plans])
+        for r in range(ranks):
+            ops[r].dispatch(plans[r][0], all_off, T)
+        if ev: ev[1].record()
+        for r in range(ranks):
+            ops[r].experts(plans[r][0])
+        if ev: ev[2].record()
+        return [ops[r].combine(plans[r][0], T) for r in range(ranks)]
+
+    for _ in range(warmup):
+        outs = forward()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        outs = forward()
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    for i in range(steps):
+        evs[i][3].record()
+        forward(evs[i][:3])
+    torch.cuda.synchronize()
+    ph = {"route_plan": sum(evs[i][3].elapsed_time(evs[i][0]) for i in range(steps)) / steps,
+          "dispatch": sum(evs[i][0].elapsed_time(evs[i][1]) for i in range(steps)) / steps,
+          "experts": sum(evs[i][1].elapsed_time(evs[i][2]) for i in range(steps)) / steps}
+    ws = tu.workspace(dev, T)
+    ref = torch.empty((T, sh.H), dtype=torch.bfloat16, device="cuda")
+    same = True
+    for r in range(ranks):
+        fx.moe_layer_forward(dev, xs[r], T, sh.H, ref, sh.H, ws, ws.numel())
+        same &= torch.equal(outs[r].view(torch.int16), ref.view(torch.int16))
+    for lr in layers:
+        for h in lr:
+            code, bits = fx.moe_get_device_status(h)
+            if code != fx.MOE_OK:
+                raise RuntimeError(f"device status {bits:#x}")
+    if not same:
+        raise RuntimeError("an emulated rank differs from the fused forward")
+    for c in comms:
+        c.close()
+    El = sh.E // ranks
+    owner_bytes = (El + sh.S) * (3 * sh.F * sh.H + 3 * sh.FB * sh.HB * 4)
+    per_owner_ms = ph["experts"] / ranks
+    return {"ranks": ranks, "tokens_per_rank": T, "transport": "dispatch/combine kernels over peer memory, ranks "
+            "emulated on one GPU (their buffers in its memory)", "ms_per_forward_all_ranks": round(ms, 5),
+            "phase_ms_all_ranks": {k: round(v, 5) for k, v in ph.items()},
+            "owner_grouped_gemms_ms_per_rank": round(per_owner_ms, 5),
+            "owner_weight_bytes_per_rank": owner_bytes,
+            "owner_weight_stream_frac_hbm": round(owner_bytes / (per_owner_ms / 1e3) / 1e9 / peaks()["hbm_gbs"], 4),
+            "parity": "every rank bit-identical to the fused forward on its tokens"}
 
 
 EP_STAGES = ("route_plan", "all_gather", "dispatch", "barrier_1", "experts", "barrier_2", "combine")
